@@ -1,0 +1,158 @@
+"""numpy front end of the CPU oracle (oracle/lrs_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by the package's smoke check and
+by the benchmark's CPU-baseline leg. The product library never imports it.
+
+All arrays are C-contiguous numpy arrays in the oracle's logical layout
+(one int8 code per element; see lrs_oracle.h). Functions that update the state
+do so in place, like the library they are compared with.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+ROUND_RTN, ROUND_SR, ROUND_BDR = 0, 1, 2
+UPDATE_GATED, UPDATE_DELTA = 0, 1
+GATE_SCALAR, GATE_PER_KEY = 0, 1
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i32, i64, u32, u64 = ctypes.c_int, ctypes.c_int64, ctypes.c_uint32, ctypes.c_uint64
+        L.orc_splitmix64.argtypes = [u64]
+        L.orc_splitmix64.restype = u64
+        L.orc_hash.argtypes = [u64, u64, u32, u32, u32, u32]
+        L.orc_hash.restype = u64
+        L.orc_uniform.argtypes = [u64]
+        L.orc_uniform.restype = ctypes.c_float
+        L.orc_step.argtypes = [i32, P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P,
+                               P, u64, u64, i32]
+        L.orc_step.restype = i32
+        L.orc_fp32_step.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P, P, i32]
+        L.orc_fp32_step.restype = i32
+        L.orc_import.argtypes = [i32, P, i32, i32, i32, P, P, P, P]
+        L.orc_import.restype = i32
+        L.orc_dequant.argtypes = [i32, i32, i32, i32, P, P, P]
+        L.orc_dequant.restype = i32
+        L.orc_decay_means.argtypes = [i64, i32, i64, P, P]
+        L.orc_decay_means.restype = None
+        L.orc_precision_map.argtypes = [i32, P, i32, P]
+        L.orc_precision_map.restype = i32
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f32(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float32)
+
+
+def splitmix64(z):
+    return int(lib().orc_splitmix64(z & (2**64 - 1)))
+
+
+def hash64(seed, step, b, h, i, j):
+    return int(lib().orc_hash(seed, step, b, h, i, j))
+
+
+def uniform(r):
+    return float(lib().orc_uniform(r))
+
+
+def default_threads():
+    return os.cpu_count() or 1
+
+
+def step(codes, scales, q, k, v, gates, beta, prec_map, tile_b, tile_h, *, group,
+         update_kind, gate_kind, mode, seed=0, step=0, nthreads=1):
+    """One quantized decode step for ntiles tiles; codes/scales updated in place.
+
+    codes int8 [n][d_k][d_v]; scales f32 [n][G][d_v]; q, k [n][d_k]; v [n][d_v];
+    gates [n][d_k] or [n]; beta [n] or None; prec_map u8 [H]; tile_b, tile_h [n].
+    Returns out f32 [n][d_v].
+    """
+    n, d_k, d_v = codes.shape
+    assert codes.dtype == np.int8 and scales.dtype == np.float32
+    q, k, v, gates, beta = map(_f32, (q, k, v, gates, beta))
+    prec_map = np.ascontiguousarray(prec_map, dtype=np.uint8)
+    tile_b = np.ascontiguousarray(tile_b, dtype=np.int32)
+    tile_h = np.ascontiguousarray(tile_h, dtype=np.int32)
+    out = np.zeros((n, d_v), np.float32)
+    rc = lib().orc_step(n, _p(tile_b), _p(tile_h), d_k, d_v, group, update_kind, gate_kind, mode,
+                        _p(prec_map), _p(codes), _p(scales), _p(q), _p(k), _p(v), _p(gates),
+                        _p(beta), _p(out), seed, step, nthreads)
+    if rc != 0:
+        raise ValueError("orc_step rejected its arguments (%d)" % rc)
+    return out
+
+
+def fp32_step(S, q, k, v, gates, beta, *, update_kind, gate_kind, nthreads=1):
+    """The same recurrence on an fp32 state S [n][d_k][d_v] (updated in place)."""
+    n, d_k, d_v = S.shape
+    assert S.dtype == np.float32
+    q, k, v, gates, beta = map(_f32, (q, k, v, gates, beta))
+    out = np.zeros((n, d_v), np.float32)
+    rc = lib().orc_fp32_step(n, d_k, d_v, update_kind, gate_kind, _p(S), _p(q), _p(k), _p(v),
+                             _p(gates), _p(beta), _p(out), nthreads)
+    if rc != 0:
+        raise ValueError("orc_fp32_step rejected its arguments (%d)" % rc)
+    return out
+
+
+def import_fp32(S0, prec_map, tile_h, *, group):
+    """Round-to-nearest quantization of S0 [n][d_k][d_v] -> (codes, scales)."""
+    S0 = _f32(S0)
+    n, d_k, d_v = S0.shape
+    prec_map = np.ascontiguousarray(prec_map, dtype=np.uint8)
+    tile_h = np.ascontiguousarray(tile_h, dtype=np.int32)
+    codes = np.zeros((n, d_k, d_v), np.int8)
+    scales = np.zeros((n, d_k // group, d_v), np.float32)
+    rc = lib().orc_import(n, _p(tile_h), d_k, d_v, group, _p(prec_map), _p(S0), _p(codes),
+                          _p(scales))
+    if rc != 0:
+        raise ValueError("orc_import rejected its arguments (%d)" % rc)
+    return codes, scales
+
+
+def dequant(codes, scales, *, group):
+    n, d_k, d_v = codes.shape
+    S = np.zeros((n, d_k, d_v), np.float32)
+    rc = lib().orc_dequant(n, d_k, d_v, group, _p(np.ascontiguousarray(codes)),
+                           _p(np.ascontiguousarray(scales, dtype=np.float32)), _p(S))
+    if rc != 0:
+        raise ValueError("orc_dequant rejected its arguments (%d)" % rc)
+    return S
+
+
+def decay_means(decay):
+    """decay f32 [outer][H][inner] -> f64 [H]."""
+    decay = _f32(decay)
+    outer, H, inner = decay.shape
+    means = np.zeros(H, np.float64)
+    lib().orc_decay_means(outer, H, inner, _p(decay), _p(means))
+    return means
+
+
+def precision_map(means, n_int8):
+    means = np.ascontiguousarray(means, dtype=np.float64)
+    H = means.shape[0]
+    pm = np.zeros(H, np.uint8)
+    rc = lib().orc_precision_map(H, _p(means), n_int8, _p(pm))
+    if rc != 0:
+        raise ValueError("orc_precision_map rejected its arguments (%d)" % rc)
+    return pm

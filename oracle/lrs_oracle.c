@@ -1,0 +1,374 @@
+/*
+ * lrs_oracle.c -- plain CPU oracle for the quantized recurrent-state decode step.
+ *
+ * TEST INFRASTRUCTURE ONLY (tests, smoke check, CPU baseline). Independent of
+ * the CUDA library; see lrs_oracle.h for the sources and the data layout.
+ *
+ * One step for one (batch, head) tile, in the order the method states it:
+ *   1. dequantize  deq_ij = c_ij * s[i/group][j]                     [LoReS]
+ *   2. update      x = g (.) deq + k w^T, where w = v (gated form) or
+ *                  w = beta (v - alpha k^T deq) (delta rule)          [LRB/BDR]
+ *   3. output      o_j = sum_i q_i x_ij over the updated state
+ *   4. new scales  per (group of key rows, value column): absmax / qmax
+ *                                                      [LoReS value-axis grouping]
+ *   5. requantize  round-to-nearest, stochastic rounding  [LoReS], or
+ *                  Bounded Directional Rounding           [LRB/BDR]
+ */
+#include "lrs_oracle.h"
+
+#include <float.h>
+#include <math.h>
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+
+#if !defined(FLT_EVAL_METHOD) || FLT_EVAL_METHOD != 0
+#error "the oracle needs binary32 evaluation of float expressions (SSE, not x87)"
+#endif
+
+/* A column group whose largest magnitude is below this is stored as zero.
+ * (Reading: the sources are silent; without it qmax/A overflows.) */
+#define ORC_TINY 0x1p-100f
+
+/* ---------------------------------------------------------------- hash --- */
+
+uint64_t orc_splitmix64(uint64_t z)
+{
+    /* [SplitMix64]: advance by the golden gamma, then the variant-13 mixer. */
+    z += 0x9E3779B97F4A7C15ULL;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+    return z ^ (z >> 31);
+}
+
+uint64_t orc_hash(uint64_t seed, uint64_t step, uint32_t b, uint32_t h, uint32_t i, uint32_t j)
+{
+    uint64_t k0 = orc_splitmix64(seed);
+    uint64_t k1 = orc_splitmix64(k0 ^ step);
+    uint64_t k2 = orc_splitmix64(k1 ^ (((uint64_t)b << 32) | (uint64_t)h));
+    return orc_splitmix64(k2 ^ (((uint64_t)i << 32) | (uint64_t)j));
+}
+
+float orc_uniform(uint64_t r)
+{
+    /* 23-bit integer, exactly representable, times 2^-23 (exact). */
+    return (float)(r >> 41) * 0x1p-23f;
+}
+
+/* ---------------------------------------------------------- rounding --- */
+
+/* Code for one element. x: the updated value; deq: its value before the
+ * update (dequantized old state); y = x * inv; s_new: the new scale. */
+static int round_element(int mode, float x, float deq, float y, float s_new, int qmax,
+                         uint64_t r)
+{
+    float c;
+    if (mode == ORC_ROUND_SR) {
+        /* [LoReS] stochastic rounding: up with probability equal to the
+         * fractional part. */
+        float f = floorf(y);
+        float fr = y - f;
+        float u = orc_uniform(r);
+        c = (u < fr) ? f + 1.0f : f;
+    } else if (mode == ORC_ROUND_BDR) {
+        /* [LRB/BDR]: the update is delta = x - deq; the move the stored value
+         * would make is m = c0*s_new - deq. When the two point in opposite
+         * directions the element is rounded toward the update instead. */
+        float c0 = rintf(y);
+        float delta = x - deq;
+        float m = c0 * s_new - deq;
+        if (delta > 0.0f && m < 0.0f)
+            c = ceilf(y);
+        else if (delta < 0.0f && m > 0.0f)
+            c = floorf(y);
+        else
+            c = c0;
+    } else {
+        c = rintf(y); /* round half to even (default rounding mode) */
+    }
+    if (c > (float)qmax) c = (float)qmax;
+    if (c < (float)-qmax) c = (float)-qmax;
+    return (int)c;
+}
+
+/* Steps 4 and 5 for one tile: new scales from x, then codes. deq may be NULL
+ * for RTN (import). */
+static void requantize_tile(int d_k, int d_v, int group, int qmax, int mode, const float *x,
+                            const float *deq, int8_t *codes, float *scales, uint64_t seed,
+                            uint64_t step, uint32_t b, uint32_t h)
+{
+    int G = d_k / group;
+    for (int g = 0; g < G; ++g) {
+        for (int j = 0; j < d_v; ++j) {
+            float A = 0.0f;
+            for (int i = g * group; i < (g + 1) * group; ++i) {
+                float a = fabsf(x[i * d_v + j]);
+                if (a > A) A = a;
+            }
+            float s_new, inv;
+            if (A < ORC_TINY) {
+                s_new = 0.0f;
+                inv = 0.0f;
+            } else {
+                s_new = A / (float)qmax;
+                inv = (float)qmax / A;
+            }
+            scales[g * d_v + j] = s_new;
+            for (int i = g * group; i < (g + 1) * group; ++i) {
+                float xv = x[i * d_v + j];
+                float y = xv * inv;
+                uint64_t r = 0;
+                if (mode == ORC_ROUND_SR) r = orc_hash(seed, step, b, h, (uint32_t)i, (uint32_t)j);
+                float dv = deq ? deq[i * d_v + j] : 0.0f;
+                codes[i * d_v + j] = (int8_t)round_element(mode, xv, dv, y, s_new, qmax, r);
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------ update --- */
+
+/* Steps 2 and 3 for one tile, shared by the quantized and the fp32 step.
+ * S_old [d_k][d_v] is the state before the update (deq for the quantized
+ * state). Writes x and out. gate points at d_k values (per key) or one. */
+static void update_tile(int d_k, int d_v, int update_kind, int gate_kind, const float *S_old,
+                        const float *q, const float *k, const float *v, const float *gate,
+                        float beta, float *w, float *x, float *out)
+{
+    if (update_kind == ORC_UPDATE_DELTA) {
+        /* Delta rule alpha (I - beta k k^T) S + beta k v^T, written as
+         * alpha S + k w^T with w = beta (v - alpha k^T S). */
+        float alpha = gate[0];
+        for (int j = 0; j < d_v; ++j) {
+            float u = 0.0f;
+            for (int i = 0; i < d_k; ++i) u = fmaf(k[i], S_old[i * d_v + j], u);
+            float t = alpha * u;
+            float d = v[j] - t;
+            w[j] = beta * d;
+        }
+    } else {
+        for (int j = 0; j < d_v; ++j) w[j] = v[j];
+    }
+    for (int i = 0; i < d_k; ++i) {
+        float gi = (gate_kind == ORC_GATE_PER_KEY) ? gate[i] : gate[0];
+        for (int j = 0; j < d_v; ++j) {
+            float kw = k[i] * w[j];
+            x[i * d_v + j] = fmaf(gi, S_old[i * d_v + j], kw);
+        }
+    }
+    for (int j = 0; j < d_v; ++j) {
+        float acc = 0.0f;
+        for (int i = 0; i < d_k; ++i) acc = fmaf(q[i], x[i * d_v + j], acc);
+        out[j] = acc;
+    }
+}
+
+/* ------------------------------------------------------------ checks --- */
+
+static int check_shape(int d_k, int d_v, int group, int update_kind, int gate_kind)
+{
+    if (d_k <= 0 || d_v <= 0 || group <= 0 || d_k % group != 0) return -1;
+    if (update_kind != ORC_UPDATE_GATED && update_kind != ORC_UPDATE_DELTA) return -1;
+    if (gate_kind != ORC_GATE_SCALAR && gate_kind != ORC_GATE_PER_KEY) return -1;
+    if (update_kind == ORC_UPDATE_DELTA && gate_kind != ORC_GATE_SCALAR) return -1;
+    return 0;
+}
+
+static int qmax_of(uint8_t bits)
+{
+    return bits == 8 ? 127 : (bits == 4 ? 7 : -1);
+}
+
+/* ---------------------------------------------------- tile-parallel loop --- */
+
+typedef struct {
+    int ntiles, d_k, d_v, group, update_kind, gate_kind, mode, nthreads, tid;
+    const int32_t *tile_b, *tile_h;
+    const uint8_t *prec_map;
+    int8_t *codes;
+    float *scales, *S;
+    const float *q, *k, *v, *gates, *beta;
+    float *out;
+    uint64_t seed, step;
+    int quantized;
+} work_t;
+
+static void *worker(void *arg)
+{
+    work_t *W = (work_t *)arg;
+    int d_k = W->d_k, d_v = W->d_v, G = d_k / W->group;
+    size_t n = (size_t)d_k * d_v;
+    float *deq = (float *)malloc(n * sizeof(float));
+    float *x = (float *)malloc(n * sizeof(float));
+    float *w = (float *)malloc((size_t)d_v * sizeof(float));
+    if (!deq || !x || !w) {
+        free(deq); free(x); free(w);
+        return (void *)1;
+    }
+    size_t gate_len = (W->gate_kind == ORC_GATE_PER_KEY) ? (size_t)d_k : 1;
+    for (int t = W->tid; t < W->ntiles; t += W->nthreads) {
+        const float *q = W->q + (size_t)t * d_k;
+        const float *k = W->k + (size_t)t * d_k;
+        const float *v = W->v + (size_t)t * d_v;
+        const float *gate = W->gates + (size_t)t * gate_len;
+        float beta = W->beta ? W->beta[t] : 0.0f;
+        float *out = W->out + (size_t)t * d_v;
+        if (W->quantized) {
+            int8_t *c = W->codes + (size_t)t * n;
+            float *s = W->scales + (size_t)t * G * d_v;
+            int qmax = qmax_of(W->prec_map[W->tile_h[t]]);
+            /* 1. dequantize with the value-axis group scales */
+            for (int i = 0; i < d_k; ++i)
+                for (int j = 0; j < d_v; ++j)
+                    deq[i * d_v + j] = (float)c[i * d_v + j] * s[(i / W->group) * d_v + j];
+            /* 2-3. update and output */
+            update_tile(d_k, d_v, W->update_kind, W->gate_kind, deq, q, k, v, gate, beta, w, x, out);
+            /* 4-5. new scales and codes */
+            requantize_tile(d_k, d_v, W->group, qmax, W->mode, x, deq, c, s, W->seed, W->step,
+                            (uint32_t)W->tile_b[t], (uint32_t)W->tile_h[t]);
+        } else {
+            float *S = W->S + (size_t)t * n;
+            update_tile(d_k, d_v, W->update_kind, W->gate_kind, S, q, k, v, gate, beta, w, x, out);
+            memcpy(S, x, n * sizeof(float));
+        }
+    }
+    free(deq); free(x); free(w);
+    return NULL;
+}
+
+static int run_tiles(work_t *proto, int nthreads)
+{
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > proto->ntiles) nthreads = proto->ntiles > 0 ? proto->ntiles : 1;
+    work_t *ws = (work_t *)calloc((size_t)nthreads, sizeof(work_t));
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!ws || !th) { free(ws); free(th); return -2; }
+    int rc = 0;
+    for (int t = 0; t < nthreads; ++t) {
+        ws[t] = *proto;
+        ws[t].tid = t;
+        ws[t].nthreads = nthreads;
+    }
+    if (nthreads == 1) {
+        if (worker(&ws[0]) != NULL) rc = -2;
+    } else {
+        int started = 0;
+        for (int t = 0; t < nthreads; ++t) {
+            if (pthread_create(&th[t], NULL, worker, &ws[t]) != 0) { rc = -2; break; }
+            ++started;
+        }
+        for (int t = 0; t < started; ++t) {
+            void *ret = NULL;
+            pthread_join(th[t], &ret);
+            if (ret != NULL) rc = -2;
+        }
+    }
+    free(ws); free(th);
+    return rc;
+}
+
+/* ------------------------------------------------------------ public --- */
+
+int orc_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int d_k, int d_v,
+             int group, int update_kind, int gate_kind, int mode, const uint8_t *prec_map,
+             int8_t *codes, float *scales, const float *q, const float *k, const float *v,
+             const float *gates, const float *beta, float *out, uint64_t seed, uint64_t step,
+             int nthreads)
+{
+    if (ntiles < 0 || check_shape(d_k, d_v, group, update_kind, gate_kind) != 0) return -1;
+    if (mode != ORC_ROUND_RTN && mode != ORC_ROUND_SR && mode != ORC_ROUND_BDR) return -1;
+    if (ntiles == 0) return 0;
+    if (!tile_b || !tile_h || !prec_map || !codes || !scales || !q || !k || !v || !gates || !out)
+        return -1;
+    if (update_kind == ORC_UPDATE_DELTA && !beta) return -1;
+    for (int t = 0; t < ntiles; ++t)
+        if (tile_h[t] < 0 || qmax_of(prec_map[tile_h[t]]) < 0) return -1;
+    work_t W;
+    memset(&W, 0, sizeof W);
+    W.ntiles = ntiles; W.d_k = d_k; W.d_v = d_v; W.group = group;
+    W.update_kind = update_kind; W.gate_kind = gate_kind; W.mode = mode;
+    W.tile_b = tile_b; W.tile_h = tile_h; W.prec_map = prec_map;
+    W.codes = codes; W.scales = scales;
+    W.q = q; W.k = k; W.v = v; W.gates = gates; W.beta = beta; W.out = out;
+    W.seed = seed; W.step = step; W.quantized = 1;
+    return run_tiles(&W, nthreads);
+}
+
+int orc_fp32_step(int ntiles, int d_k, int d_v, int update_kind, int gate_kind, float *S,
+                  const float *q, const float *k, const float *v, const float *gates,
+                  const float *beta, float *out, int nthreads)
+{
+    if (ntiles < 0 || check_shape(d_k, d_v, d_k, update_kind, gate_kind) != 0) return -1;
+    if (ntiles == 0) return 0;
+    if (!S || !q || !k || !v || !gates || !out) return -1;
+    if (update_kind == ORC_UPDATE_DELTA && !beta) return -1;
+    work_t W;
+    memset(&W, 0, sizeof W);
+    W.ntiles = ntiles; W.d_k = d_k; W.d_v = d_v; W.group = d_k;
+    W.update_kind = update_kind; W.gate_kind = gate_kind;
+    W.S = S; W.q = q; W.k = k; W.v = v; W.gates = gates; W.beta = beta; W.out = out;
+    W.quantized = 0;
+    return run_tiles(&W, nthreads);
+}
+
+int orc_import(int ntiles, const int32_t *tile_h, int d_k, int d_v, int group,
+               const uint8_t *prec_map, const float *S0, int8_t *codes, float *scales)
+{
+    if (ntiles < 0 || check_shape(d_k, d_v, group, ORC_UPDATE_GATED, ORC_GATE_SCALAR) != 0)
+        return -1;
+    if (ntiles == 0) return 0;
+    if (!tile_h || !prec_map || !S0 || !codes || !scales) return -1;
+    size_t n = (size_t)d_k * d_v;
+    int G = d_k / group;
+    for (int t = 0; t < ntiles; ++t) {
+        int qmax = qmax_of(prec_map[tile_h[t]]);
+        if (qmax < 0) return -1;
+        requantize_tile(d_k, d_v, group, qmax, ORC_ROUND_RTN, S0 + (size_t)t * n, NULL,
+                        codes + (size_t)t * n, scales + (size_t)t * G * d_v, 0, 0, 0, 0);
+    }
+    return 0;
+}
+
+int orc_dequant(int ntiles, int d_k, int d_v, int group, const int8_t *codes,
+                const float *scales, float *S)
+{
+    if (ntiles < 0 || check_shape(d_k, d_v, group, ORC_UPDATE_GATED, ORC_GATE_SCALAR) != 0)
+        return -1;
+    size_t n = (size_t)d_k * d_v;
+    int G = d_k / group;
+    for (int t = 0; t < ntiles; ++t)
+        for (int i = 0; i < d_k; ++i)
+            for (int j = 0; j < d_v; ++j)
+                S[t * n + (size_t)i * d_v + j] = (float)codes[t * n + (size_t)i * d_v + j] *
+                                                 scales[(size_t)t * G * d_v + (i / group) * d_v + j];
+    return 0;
+}
+
+void orc_decay_means(int64_t outer, int heads, int64_t inner, const float *decay, double *means)
+{
+    for (int h = 0; h < heads; ++h) {
+        double sum = 0.0;
+        for (int64_t o = 0; o < outer; ++o)
+            for (int64_t c = 0; c < inner; ++c)
+                sum += (double)decay[(o * heads + h) * inner + c];
+        means[h] = sum / (double)(outer * inner);
+    }
+}
+
+int orc_precision_map(int heads, const double *means, int n_int8, uint8_t *prec_map)
+{
+    if (heads <= 0 || n_int8 < 0 || n_int8 > heads) return -1;
+    /* [LoReS] decay-based mixed precision: rank heads by mean decay, largest
+     * first (slowest decay), ties to the lower index; selection by repeated
+     * scan keeps this obviously correct for the head counts involved. */
+    for (int h = 0; h < heads; ++h) prec_map[h] = 4;
+    for (int n = 0; n < n_int8; ++n) {
+        int best = -1;
+        for (int h = 0; h < heads; ++h) {
+            if (prec_map[h] == 8) continue;
+            if (best < 0 || means[h] > means[best]) best = h;
+        }
+        prec_map[best] = 8;
+    }
+    return 0;
+}

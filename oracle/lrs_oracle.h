@@ -1,0 +1,90 @@
+/*
+ * lrs_oracle.h -- plain CPU oracle for the quantized recurrent-state decode step.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing in the product path includes, links or calls
+ * this code; only the tests, the package's smoke check and the benchmark's CPU
+ * baseline leg do. It shares no source, header, table or helper with the CUDA
+ * library: everything here is written out independently, in the order in which
+ * the method is stated, so that a reader can check it against the sources:
+ *
+ *   [LoReS]  "Quantizing Recurrent Language Models Is Easier Than You Think",
+ *            abstract: value-axis scale grouping, decay-based mixed precision
+ *            for slowly decaying heads, stochastic rounding against error
+ *            accumulation under repeated requantization.
+ *   [LRB/BDR] "Preserving Updates in Low-Bit Recurrent State Quantization",
+ *            abstract: the state is updated and requantized at every step;
+ *            Bounded Directional Rounding rounds an element that would move
+ *            opposite to its update toward that update instead.
+ *   [SplitMix64] Steele, Lea & Flood, "Fast Splittable Pseudorandom Number
+ *            Generators", OOPSLA 2014 (the published generator and mixer).
+ *
+ * Arithmetic: IEEE binary32 with one round-to-nearest-even per written
+ * operation; the only fused operations are the explicit fmaf() calls. Build
+ * with -ffp-contract=off and without fast-math (see oracle/build.py).
+ *
+ * Data layout (logical, one code per byte, independent of any packed format):
+ *   codes  int8  [ntiles][d_k][d_v]   code c_ij in [-qmax, qmax]
+ *   scales float [ntiles][G][d_v]     G = d_k / group
+ *   q, k   float [ntiles][d_k];  v, out float [ntiles][d_v]
+ *   gates  float [ntiles][d_k] (per-key) or [ntiles] (scalar)
+ *   beta   float [ntiles]       (delta rule only)
+ * Tile t is head tile_h[t] of batch row tile_b[t]; (b, h) enter the hash and
+ * select the precision prec_map[h] in {4, 8}.
+ */
+#ifndef LRS_ORACLE_H
+#define LRS_ORACLE_H
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum { ORC_ROUND_RTN = 0, ORC_ROUND_SR = 1, ORC_ROUND_BDR = 2 };
+enum { ORC_UPDATE_GATED = 0, ORC_UPDATE_DELTA = 1 };
+enum { ORC_GATE_SCALAR = 0, ORC_GATE_PER_KEY = 1 };
+
+/* SplitMix64 output for generator state z: the state is advanced by the golden
+ * gamma and then mixed. A generator seeded with s returns mix(s), mix(s+g), ... */
+uint64_t orc_splitmix64(uint64_t z);
+
+/* Counter hash of one state element: a chain of SplitMix64 mixes over
+ * (seed, step, (b,h), (i,j)). */
+uint64_t orc_hash(uint64_t seed, uint64_t step, uint32_t b, uint32_t h, uint32_t i, uint32_t j);
+
+/* Uniform in [0,1) on the 2^-23 grid taken from the top 23 bits of r. */
+float orc_uniform(uint64_t r);
+
+/* One decode step, in place on codes and scales, writing out. Returns 0, or a
+ * negative value for invalid arguments (nothing is written then). */
+int orc_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h,
+             int d_k, int d_v, int group, int update_kind, int gate_kind, int mode,
+             const uint8_t *prec_map, int8_t *codes, float *scales,
+             const float *q, const float *k, const float *v, const float *gates,
+             const float *beta, float *out, uint64_t seed, uint64_t step, int nthreads);
+
+/* The same recurrence on an fp32 state S [ntiles][d_k][d_v], no quantization:
+ * S <- x, out = x^T q. */
+int orc_fp32_step(int ntiles, int d_k, int d_v, int update_kind, int gate_kind, float *S,
+                  const float *q, const float *k, const float *v, const float *gates,
+                  const float *beta, float *out, int nthreads);
+
+/* Quantize an fp32 state with round-to-nearest into codes and scales. */
+int orc_import(int ntiles, const int32_t *tile_h, int d_k, int d_v, int group,
+               const uint8_t *prec_map, const float *S0, int8_t *codes, float *scales);
+
+/* Dequantize codes and scales into S [ntiles][d_k][d_v]. */
+int orc_dequant(int ntiles, int d_k, int d_v, int group, const int8_t *codes,
+                const float *scales, float *S);
+
+/* Mean decay per head, accumulated in binary64 in index order.
+ * decay [outer][heads][inner]; means [heads]. */
+void orc_decay_means(int64_t outer, int heads, int64_t inner, const float *decay, double *means);
+
+/* Mixed precision: the n_int8 heads with the largest mean decay (ties to the
+ * lower head index) get 8-bit codes, the rest 4-bit. */
+int orc_precision_map(int heads, const double *means, int n_int8, uint8_t *prec_map);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
