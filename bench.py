@@ -1,0 +1,495 @@
+"""Throughput of the quantized recurrent-state decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lrs|reference]
+                    [--workload NAME] [--layers L] [--mode rtn|sr|bdr] [--no-extras]
+
+A step is one decode step of one layer's state: every (batch, head) tile of
+the workload is dequantized, updated, read out and requantized once (one
+kernel launch). Steps rotate over L independent layer states whose total size
+is far above the 126 MB L2, as in a model where the other layers run between
+two steps of one layer, so every step reads its state from HBM.
+
+Prints one JSON line (rank 0). Under torchrun each rank runs its own batch of
+the workload (weak scaling, no collective on the data path); the time is the
+slowest rank's.
+
+--impl reference times the CPU oracle on the host cores on a bounded sample of
+tiles per step and reports the same metric for the whole workload.
+"""
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantized-state decode steps/s and state GB/s (% of HBM peak), B=256 32h 128×128"
+DEFAULT_WORKLOAD = "gla_rtn_int8_b256h32_128"
+MODES = {"rtn": 0, "sr": 1, "bdr": 2}
+KERNEL_SOURCES = ["quantized_recurrent_state_decode_b200/csrc/step_kernel.cuh",
+                  "quantized_recurrent_state_decode_b200/csrc/lrs_device.cuh",
+                  "quantized_recurrent_state_decode_b200/csrc/step_rtn.cu"]
+PROFILE = os.path.join(ROOT, "profiles", "step_kernel_gla_rtn_int8_b256h32.md")
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the step kernel from the committed ncu summary,
+    if it was taken on the current kernel source; else None."""
+    try:
+        text = open(PROFILE).read()
+    except OSError:
+        return None
+    m = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
+    t = re.search(r"dram_bytes_per_launch_full_workload:\s*([0-9.eE+]+)", text)
+    if not m or not t or m.group(1) != kernel_source_hash():
+        return None
+    return float(t.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self):
+        return time.time()
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(2)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [l for (ts, l) in self.lines if t0 <= ts <= t1] or \
+            [l for (_, l) in self.lines[-5:]]
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            f = [x.strip() for x in r.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# --------------------------------------------------------------- reference ---
+
+def run_reference(args, w):
+    """The CPU oracle on the host cores: each step runs a bounded sample of
+    tiles, and the metric is scaled to the whole workload."""
+    import numpy as np
+    import oracle
+    from quantized_recurrent_state_decode_b200 import inputs as I
+
+    nthreads = oracle.default_threads()
+    mode = MODES[args.mode] if args.mode else w.mode
+    pm = I.uniform_prec_map(w).numpy()
+    # calibrate: time per tile with all threads
+    ntiles_all = w.batch * w.heads
+    rng = np.random.default_rng(0)
+    per_step = max(nthreads, 8)
+    tiles = rng.choice(ntiles_all, size=per_step, replace=False)
+    tb = (tiles // w.heads).astype(np.int32)
+    th = (tiles % w.heads).astype(np.int32)
+    S0 = I.initial_state(w)[tb, th].numpy()
+    codes, scales = oracle.import_fp32(S0, pm, th, group=w.group)
+    x0 = I.step_inputs(w, 0)
+    sel = {n: (None if v is None else v[tb, th].numpy().reshape(len(tiles), -1))
+           for n, v in x0.items()}
+
+    def one(t):
+        oracle.step(codes, scales, sel["q"], sel["k"], sel["v"], sel["gates"],
+                    None if sel["beta"] is None else sel["beta"].reshape(-1), pm, tb, th,
+                    group=w.group, update_kind=w.update_kind, gate_kind=w.gate_kind, mode=mode,
+                    seed=1, step=t, nthreads=nthreads)
+
+    t0 = time.perf_counter()
+    one(0)
+    t_sample = time.perf_counter() - t0
+    budget = 120.0
+    reps = max(1, int(budget / max(t_sample, 1e-6) / max(args.steps + args.warmup, 1)))
+    reps = min(reps, 64)
+    for t in range(args.warmup):
+        for _ in range(reps):
+            one(t)
+    t0 = time.perf_counter()
+    for t in range(args.steps):
+        for _ in range(reps):
+            one(t)
+    el = time.perf_counter() - t0
+    sec_per_tile = el / (args.steps * reps * len(tiles))
+    sec_per_step = sec_per_tile * ntiles_all
+    steps_per_s = 1.0 / sec_per_step
+    sample = ("%d of %d tiles x %d repeats per step, %d threads, extrapolated to the whole "
+              "workload" % (len(tiles), ntiles_all, reps, nthreads))
+    line = {"metric": METRIC, "impl": "reference", "value": steps_per_s, "unit": "steps/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec_per_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": config_of(w, mode, args.layers, args.gpus),
+            "cpu_baseline": {"value": steps_per_s, "unit": "steps/s", "cores": nthreads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": steps_per_s, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def config_of(w, mode, layers, n):
+    from quantized_recurrent_state_decode_b200 import inputs as I
+    prec = {"int8": "int8", "int4": "int4", "mixed": "mixed int8/int4"}[w.precision]
+    return {"workload": w.name, "family": w.family, "batch_per_gpu": w.batch,
+            "global_batch": w.batch * n, "heads": w.heads, "d_k": w.d_k, "d_v": w.d_v,
+            "group": w.group, "state": prec,
+            "rounding": {0: "rtn", 1: "sr", 2: "bdr"}[mode],
+            "layers_rotated": layers,
+            "l2": "inputs larger than L2: %d layer states rotated per step" % layers,
+            "parallelism": "dp%d" % n}
+
+
+# -------------------------------------------------------------------- GPU ---
+
+def state_bytes(w, prec_bits=8):
+    G = w.d_k // w.group
+    return w.batch * w.heads * (w.d_k * w.d_v * prec_bits // 8 + G * w.d_v * 4)
+
+
+def run_gpu(args, w):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from quantized_recurrent_state_decode_b200 import inputs as I
+    from quantized_recurrent_state_decode_b200 import lrs
+    from quantized_recurrent_state_decode_b200.shard import batch_slice, max_over_ranks
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    mode = MODES[args.mode] if args.mode else w.mode
+
+    # weak scaling: every rank owns a batch slice of size w.batch of a global
+    # batch of w.batch * world rows
+    wg = w.with_batch(w.batch * world)
+    off, nb = batch_slice(wg.batch, rank, world)
+    wl = w.with_batch(nb)
+    pm = I.uniform_prec_map(w).numpy()
+    shp = lrs.shape(nb, w.heads, w.d_k, w.d_v, w.group, w.update_kind, w.gate_kind)
+    L = args.layers
+    states = [lrs.lrs_state_alloc(shp, pm) for _ in range(L)]
+    S0 = I.initial_state(wg, off, nb, device=dev)
+    for st in states:
+        lrs.lrs_state_import_fp32(st, S0)
+    del S0
+    NI = 8
+    xs = [I.step_inputs(wg, t, off, nb, device=dev) for t in range(NI)]
+    out = torch.empty(nb, w.heads, w.d_v, device=dev)
+    seed = I.sr_seed(w)
+    torch.cuda.synchronize()
+    # all work runs on one non-default stream (graph capture needs one)
+    stream = torch.cuda.Stream()
+    pick = lambda i: (states[i % L], xs[i % NI], i)
+
+    with torch.cuda.stream(stream):
+        for t in range(args.warmup):                    # warm-up, eager launches
+            st, x, _ = pick(t)
+            lrs.lrs_decode_step(st, st.state_codes, st.scales, st.prec_map, x["q"], x["k"],
+                                x["v"], x["gates"], x["beta"], out, seed, t, mode, stream)
+        lrs.lrs_sync(stream)
+        # the timed steps: CUDA graphs of `chunk` launches, replayed
+        chunk = min(args.steps, 64)
+        full, rem = divmod(args.steps, chunk)
+        g_chunk = _capture_on(stream, chunk, pick, lrs, out, seed, mode)
+        g_rem = _capture_on(stream, rem, pick, lrs, out, seed, mode) if rem else None
+        g_chunk.replay()                                # one untimed replay
+        torch.cuda.synchronize()
+
+        sampler = ClockSampler(local)
+        if rank == 0:
+            sampler.start()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t_wall0 = time.time()
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(full):
+            g_chunk.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        t_wall1 = time.time()
+        if world > 1:
+            dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    lrs.lrs_sync(stream)
+    del g_chunk, g_rem
+    ms_max = max_over_ranks(ms, device=dev)
+    clocks = sampler.summary(t_wall0, t_wall1) if rank == 0 else None
+    if rank == 0:
+        sampler.stop()
+
+    steps_per_s = world * args.steps / (ms_max / 1e3)
+    bytes_step = state_bytes(wl)
+    launch_s = ms / 1e3 / args.steps
+    achieved = bytes_step / launch_s / 1e9
+    peak, peak_kind = measured_peaks()
+
+    # end to end: host inputs in pinned memory, copies inside the timed region
+    e2e_steps = min(args.steps, 256)
+    xh = [{n: (None if v is None else v.cpu().pin_memory()) for n, v in x.items()} for x in xs]
+    out_h = torch.empty(nb, w.heads, w.d_v).pin_memory()
+    st0 = states[0]
+    with torch.cuda.stream(stream):
+        for t in range(min(args.warmup, 8)):
+            x = xh[t % NI]
+            lrs.lrs_decode_step_host(st0, x["q"], x["k"], x["v"], x["gates"], x["beta"], out_h,
+                                     seed, t, mode, stream)
+        lrs.lrs_sync(stream)
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for t in range(e2e_steps):
+            st = states[t % L]
+            x = xh[t % NI]
+            lrs.lrs_decode_step_host(st, x["q"], x["k"], x["v"], x["gates"], x["beta"], out_h,
+                                     seed, t, mode, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    lrs.lrs_sync(stream)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), device=dev)
+    h2d = sum(v.numel() * 4 for v in xh[0].values() if v is not None)
+    d2h = out_h.numel() * 4
+
+    extras = {}
+    if not args.no_extras and rank == 0:
+        with torch.cuda.stream(stream):
+            extras = run_extras(args, w, wl, states, xs, out, seed, stream, L, NI, mode, dev)
+
+    for st in states:
+        lrs.lrs_state_free(st)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    line = {
+        "metric": METRIC, "value": steps_per_s, "unit": "steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded draws with the workload's distributions)",
+        "config": config_of(w, mode, L, world),
+        "state_gbs": achieved,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind + " (hbm_gbs, burst copy)",
+                     "traffic": profiled_traffic(),
+                     "algorithmic_bytes_per_launch": bytes_step,
+                     "kernel": "lrs::step_kernel<4,32,gated,per_key,%s>" % (
+                         {0: "rtn", 1: "sr", 2: "bdr"}[mode])},
+        "e2e": {"value": world * e2e_steps / (e2e_ms / 1e3), "unit": "steps/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "api": "lrs_decode_step_host"},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    line.update(extras)
+    if args.cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, mode)
+    print(json.dumps(line))
+
+
+def _capture_on(stream, n, pick, lrs, out, seed, mode):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            st, x, t = pick(i)
+            lrs.lrs_decode_step(st, st.state_codes, st.scales, st.prec_map, x["q"], x["k"],
+                                x["v"], x["gates"], x["beta"], out, seed, t, mode, stream)
+    return g
+
+
+def run_extras(args, w, wl, states, xs, out, seed, stream, L, NI, mode, dev):
+    """Other rounding modes on the same state, and the fp32-state kernel on the
+    same inputs (rank 0 only, not part of the headline number)."""
+    import torch
+    from quantized_recurrent_state_decode_b200 import lrs
+    res = {}
+    n = 640
+    for name, m in (("sr", 1), ("bdr", 2), ("rtn", 0)):
+        if m == mode:
+            continue
+        for i in range(8):   # eager launches before capture
+            st, x, t = states[i % L], xs[i % NI], i
+            lrs.lrs_decode_step(st, st.state_codes, st.scales, st.prec_map, x["q"], x["k"],
+                                x["v"], x["gates"], x["beta"], out, seed, t, m, stream)
+        g = _capture_on(stream, n, lambda i: (states[i % L], xs[i % NI], i), lrs, out, seed, m)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / n
+        res["mode_" + name] = {"ms_per_step": ms, "steps_per_s": 1e3 / ms,
+                               "state_gbs": state_bytes(wl) / (ms / 1e3) / 1e9}
+        del g
+    lrs.lrs_sync()
+    # fp32 state kernel: 4 rotated fp32 states
+    shp = lrs.shape(wl.batch, w.heads, w.d_k, w.d_v, w.group, w.update_kind, w.gate_kind)
+    Ls = 4
+    Ss = [torch.zeros(wl.batch, w.heads, w.d_k, w.d_v, device=dev) for _ in range(Ls)]
+    nf = 256
+    for i in range(4):
+        x = xs[i % NI]
+        lrs.lrs_fp32_decode_step(shp, Ss[i % Ls], x["q"], x["k"], x["v"], x["gates"], x["beta"],
+                                 out, stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(nf):
+            x = xs[i % NI]
+            lrs.lrs_fp32_decode_step(shp, Ss[i % Ls], x["q"], x["k"], x["v"], x["gates"],
+                                     x["beta"], out, stream)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / nf
+    fb = wl.batch * w.heads * w.d_k * w.d_v * 4 * 2
+    res["fp32_state_kernel"] = {"ms_per_step": ms, "steps_per_s": 1e3 / ms,
+                                "state_gbs": fb / (ms / 1e3) / 1e9, "bytes_per_step": fb}
+    del g, Ss
+    return res
+
+
+def cpu_baseline(w, mode):
+    """The oracle on the host cores, a bounded sample of tiles for ~10-20 s."""
+    import numpy as np
+    import oracle
+    from quantized_recurrent_state_decode_b200 import inputs as I
+    nthreads = oracle.default_threads()
+    ntiles_all = w.batch * w.heads
+    n = min(ntiles_all, max(nthreads * 16, 256))
+    rng = np.random.default_rng(1)
+    tiles = np.sort(rng.choice(ntiles_all, size=n, replace=False))
+    tb = (tiles // w.heads).astype(np.int32)
+    th = (tiles % w.heads).astype(np.int32)
+    pm = I.uniform_prec_map(w).numpy()
+    S0 = I.initial_state(w)[tb, th].numpy()
+    codes, scales = oracle.import_fp32(S0, pm, th, group=w.group)
+    reps, el = 0, 0.0
+    t_end = time.perf_counter() + 12.0
+    while time.perf_counter() < t_end or reps == 0:
+        x = I.step_inputs(w, reps)
+        sel = {k: (None if v is None else v[tb, th].numpy().reshape(n, -1)) for k, v in x.items()}
+        t0 = time.perf_counter()
+        oracle.step(codes, scales, sel["q"], sel["k"], sel["v"], sel["gates"],
+                    None if sel["beta"] is None else sel["beta"].reshape(-1), pm, tb, th,
+                    group=w.group, update_kind=w.update_kind, gate_kind=w.gate_kind, mode=mode,
+                    seed=1, step=reps, nthreads=nthreads)
+        el += time.perf_counter() - t0
+        reps += 1
+    sec_step = el / reps / n * ntiles_all
+    return {"value": 1.0 / sec_step, "unit": "steps/s", "cores": nthreads, "kind": "oracle",
+            "sample": "%d of %d tiles for %d steps (%.1f s of oracle time), scaled to the whole "
+                      "workload" % (n, ntiles_all, reps, el)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=6400)
+    ap.add_argument("--warmup", type=int, default=64)
+    ap.add_argument("--impl", default="lrs", choices=["lrs", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--mode", default=None, choices=sorted(MODES))
+    ap.add_argument("--layers", type=int, default=4)
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    from quantized_recurrent_state_decode_b200 import inputs as I
+    w = I.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        run_reference(args, w)
+        return
+    run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,393 @@
+// aux_kernels.cu -- the state's set-up and inspection kernels, the fp32-state
+// decode step used as the uncompressed baseline, and the per-head mean decay.
+//
+// The quantizing kernels here share the step kernel's rounding and packing
+// (round_code / encode_word), so an imported state is exactly the state a step
+// with x = S would produce.
+#include "lrs_internal.h"
+#include "step_kernel.cuh"
+
+namespace lrs {
+
+namespace {
+
+constexpr int kAuxWarps = 8;
+
+// Byte offset, inside a tile, of the 16-byte unit `u` of lane `lane`.
+__device__ __forceinline__ int unit_offset(int u, int lane) { return (u * 32 + lane) * 16; }
+
+struct TileRef {
+    uint8_t* codes;   // tile base
+    int prec;         // 4 or 8, 0 when the layout is inconsistent
+};
+
+__device__ __forceinline__ TileRef tile_ref(const LayoutArgs& a, int tile) {
+    const int h = tile % a.H, b = tile / a.H;
+    const int prec = a.prec_map[h];
+    const int64_t off = a.head_offsets[h];
+    const int64_t end = (h + 1 < a.H) ? a.head_offsets[h + 1] : a.batch_stride;
+    const int64_t bytes = static_cast<int64_t>(a.d_k) * a.d_v * prec / 8;
+    TileRef t;
+    t.prec = ((prec == 4 || prec == 8) && off >= 0 && off + bytes <= end) ? prec : 0;
+    t.codes = a.codes + static_cast<int64_t>(b) * a.batch_stride + off;
+    return t;
+}
+
+// Quantize x[GROUP][C] (this lane's columns of one group) with round to
+// nearest into the tile's group block and scales row.
+template <int C, int GROUP, int BITS>
+__device__ void quantize_group_rtn(const float (&x)[GROUP][C], uint8_t* gcodes, float* gscales,
+                                   int lane) {
+    constexpr int EPW = 32 / BITS;
+    constexpr int UNITS = GROUP * C * BITS / 8 / 16;
+    constexpr float QMAX = BITS == 8 ? 127.0f : 7.0f;
+    float snew[C], inv[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        float A = 0.0f;
+#pragma unroll
+        for (int r = 0; r < GROUP; ++r) A = fmaxf(A, fabsf(x[r][c]));
+        const bool zero = A < kTiny;
+        snew[c] = zero ? 0.0f : __fdiv_rn(A, QMAX);
+        inv[c] = zero ? 0.0f : __fdiv_rn(QMAX, A);
+        gscales[lane * C + c] = snew[c];
+    }
+#pragma unroll
+    for (int un = 0; un < UNITS; ++un) {
+        uint32_t ow[4];
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+            float t[EPW];
+#pragma unroll
+            for (int e = 0; e < EPW; ++e) {
+                const int el = (un * 4 + wi) * EPW + e;
+                const int r = el / C, c = el % C;
+                t[e] = round_code<kRTN, BITS>(__fmul_rn(x[r][c], inv[c]), 0.f, 0.f, 0.f, 0ull, 0u,
+                                              0u);
+            }
+            ow[wi] = encode_word<BITS>(t);
+        }
+        *reinterpret_cast<uint4*>(gcodes + unit_offset(un, lane)) =
+            make_uint4(ow[0], ow[1], ow[2], ow[3]);
+    }
+}
+
+// Signed codes of one group block, code[r][c] for this lane's columns.
+template <int C, int GROUP, int BITS>
+__device__ void decode_group(const uint8_t* gcodes, int lane, float (&code)[GROUP][C]) {
+    constexpr int EPW = 32 / BITS;
+    constexpr int UNITS = GROUP * C * BITS / 8 / 16;
+#pragma unroll
+    for (int un = 0; un < UNITS; ++un) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(gcodes + unit_offset(un, lane));
+        const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+            float f[EPW];
+            decode_word<BITS>(wd[wi], f);
+#pragma unroll
+            for (int e = 0; e < EPW; ++e) {
+                const int el = (un * 4 + wi) * EPW + e;
+                code[el / C][el % C] = f[e];
+            }
+        }
+    }
+}
+
+enum { kOpFillZero, kOpImportFp32, kOpExportFp32, kOpExportCodes, kOpImportCodes };
+
+template <int C, int GROUP, int BITS>
+__device__ void layout_op_tile(const LayoutArgs& a, int op, int tile, uint8_t* tcodes,
+                               const float* S, float* So, int8_t* Co, const int8_t* Ci,
+                               const float* Si, int lane) {
+    constexpr int DV = 32 * C;
+    constexpr int QMAX = BITS == 8 ? 127 : 7;
+    const int G = a.d_k / GROUP;
+    const int64_t tile_elems = static_cast<int64_t>(a.d_k) * DV;
+    for (int g = 0; g < G; ++g) {
+        uint8_t* gcodes = tcodes + static_cast<int64_t>(g) * GROUP * DV * BITS / 8;
+        float* gscales = a.scales + (static_cast<int64_t>(tile) * G + g) * DV;
+        const int64_t base = tile * tile_elems + static_cast<int64_t>(g) * GROUP * DV + lane * C;
+        if (op == kOpFillZero || op == kOpImportFp32 || op == kOpImportCodes) {
+            float x[GROUP][C];
+            if (op == kOpImportFp32) {
+#pragma unroll
+                for (int r = 0; r < GROUP; ++r)
+#pragma unroll
+                    for (int c = 0; c < C; ++c) x[r][c] = S[base + r * DV + c];
+                quantize_group_rtn<C, GROUP, BITS>(x, gcodes, gscales, lane);
+            } else {
+                // zero state, or given codes: the codes are written as they are
+                // (clamped), the scales copied.
+#pragma unroll
+                for (int r = 0; r < GROUP; ++r)
+#pragma unroll
+                    for (int c = 0; c < C; ++c) {
+                        float cv = 0.0f;
+                        if (op == kOpImportCodes) {
+                            int ci = Ci[base + r * DV + c];
+                            if (ci > QMAX || ci < -QMAX) {
+                                atomicOr(a.err, kErrRange);
+                                ci = ci > QMAX ? QMAX : -QMAX;
+                            }
+                            cv = static_cast<float>(ci);
+                        }
+                        x[r][c] = cv;
+                    }
+                constexpr int EPW = 32 / BITS;
+                constexpr int UNITS = GROUP * C * BITS / 8 / 16;
+#pragma unroll
+                for (int un = 0; un < UNITS; ++un) {
+                    uint32_t ow[4];
+#pragma unroll
+                    for (int wi = 0; wi < 4; ++wi) {
+                        float t[EPW];
+#pragma unroll
+                        for (int e = 0; e < EPW; ++e) {
+                            const int el = (un * 4 + wi) * EPW + e;
+                            t[e] = round_code<kRTN, BITS>(x[el / C][el % C], 0.f, 0.f, 0.f, 0ull,
+                                                          0u, 0u);
+                        }
+                        ow[wi] = encode_word<BITS>(t);
+                    }
+                    *reinterpret_cast<uint4*>(gcodes + unit_offset(un, lane)) =
+                        make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                }
+#pragma unroll
+                for (int c = 0; c < C; ++c)
+                    gscales[lane * C + c] = op == kOpImportCodes ? Si[(static_cast<int64_t>(tile) * G + g) * DV + lane * C + c] : 0.0f;
+            }
+        } else {
+            float code[GROUP][C];
+            decode_group<C, GROUP, BITS>(gcodes, lane, code);
+#pragma unroll
+            for (int r = 0; r < GROUP; ++r)
+#pragma unroll
+                for (int c = 0; c < C; ++c) {
+                    if (op == kOpExportFp32)
+                        So[base + r * DV + c] = __fmul_rn(code[r][c], gscales[lane * C + c]);
+                    else
+                        Co[base + r * DV + c] = static_cast<int8_t>(static_cast<int>(code[r][c]));
+                }
+        }
+    }
+}
+
+template <int C, int GROUP>
+__global__ void __launch_bounds__(kAuxWarps * 32) layout_kernel(const LayoutArgs a, int op,
+                                                                 const float* S, float* So,
+                                                                 int8_t* Co, const int8_t* Ci,
+                                                                 const float* Si) {
+    const int lane = threadIdx.x & 31;
+    const int ntiles = a.B * a.H;
+    for (int tile = blockIdx.x * kAuxWarps + (threadIdx.x >> 5); tile < ntiles;
+         tile += gridDim.x * kAuxWarps) {
+        const TileRef t = tile_ref(a, tile);
+        if (t.prec == 0) {
+            if (lane == 0) atomicOr(a.err, kErrLayout);
+            continue;
+        }
+        if (t.prec == 8)
+            layout_op_tile<C, GROUP, 8>(a, op, tile, t.codes, S, So, Co, Ci, Si, lane);
+        else
+            layout_op_tile<C, GROUP, 4>(a, op, tile, t.codes, S, So, Co, Ci, Si, lane);
+    }
+}
+
+cudaError_t launch_layout(const LayoutArgs& a, int op, const float* S, float* So, int8_t* Co,
+                          const int8_t* Ci, const float* Si, cudaStream_t s) {
+    const int ntiles = a.B * a.H;
+    if (ntiles == 0) return cudaSuccess;
+    const int grid = (ntiles + kAuxWarps - 1) / kAuxWarps;
+    const int C = a.d_v / 32;
+#define LRS_LAYOUT_CASE(CC, GG)                                                              \
+    if (C == CC && a.group == GG) {                                                          \
+        layout_kernel<CC, GG><<<grid, kAuxWarps * 32, 0, s>>>(a, op, S, So, Co, Ci, Si);     \
+        return cudaGetLastError();                                                           \
+    }
+    LRS_LAYOUT_CASE(4, 16)
+    LRS_LAYOUT_CASE(4, 32)
+    LRS_LAYOUT_CASE(2, 16)
+    LRS_LAYOUT_CASE(2, 32)
+    LRS_LAYOUT_CASE(2, 64)
+#undef LRS_LAYOUT_CASE
+    return cudaErrorInvalidValue;
+}
+
+// ------------------------------------------------------------ fp32 step ---
+
+// One warp per tile, lane t owns columns [t*C, t*C + C) of every row, rows in
+// key order: the same arithmetic, in the same order, as the quantized step
+// with deq replaced by the fp32 state.
+template <int C, int UPD, int GATE>
+__global__ void __launch_bounds__(kAuxWarps * 32) fp32_step_kernel(
+    int ntiles, int d_k, float* S, const float* q, const float* k, const float* v,
+    const float* gates, const float* beta, float* out) {
+    constexpr int DV = 32 * C;
+    constexpr int UNR = 8;
+    const int lane = threadIdx.x & 31;
+    for (int tile = blockIdx.x * kAuxWarps + (threadIdx.x >> 5); tile < ntiles;
+         tile += gridDim.x * kAuxWarps) {
+        float* St = S + static_cast<int64_t>(tile) * d_k * DV + lane * C;
+        const float* qt = q + static_cast<int64_t>(tile) * d_k;
+        const float* kt = k + static_cast<int64_t>(tile) * d_k;
+        const float* gt = gates + (GATE == kGatePerKey ? static_cast<int64_t>(tile) * d_k : tile);
+        float w[C], o[C];
+        const float alpha = GATE == kGate ? __ldg(gt) : 0.0f;
+        if (UPD == kDelta) {
+            float u[C];
+#pragma unroll
+            for (int c = 0; c < C; ++c) u[c] = 0.0f;
+            for (int i0 = 0; i0 < d_k; i0 += UNR) {
+                float s[UNR][C];
+#pragma unroll
+                for (int r = 0; r < UNR; ++r) {
+                    const float* row = St + static_cast<int64_t>(i0 + r) * DV;
+                    if constexpr (C == 4) {
+                        const float4 t = *reinterpret_cast<const float4*>(row);
+                        s[r][0] = t.x; s[r][1] = t.y; s[r][2] = t.z; s[r][3] = t.w;
+                    } else {
+                        const float2 t = *reinterpret_cast<const float2*>(row);
+                        s[r][0] = t.x; s[r][1] = t.y;
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < UNR; ++r) {
+                    const float ki = __ldg(kt + i0 + r);
+#pragma unroll
+                    for (int c = 0; c < C; ++c) u[c] = __fmaf_rn(ki, s[r][c], u[c]);
+                }
+            }
+            const float b = __ldg(beta + tile);
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                const float t = __fmul_rn(alpha, u[c]);
+                const float d = __fsub_rn(__ldg(v + static_cast<int64_t>(tile) * DV + lane * C + c), t);
+                w[c] = __fmul_rn(b, d);
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < C; ++c) w[c] = __ldg(v + static_cast<int64_t>(tile) * DV + lane * C + c);
+        }
+#pragma unroll
+        for (int c = 0; c < C; ++c) o[c] = 0.0f;
+        for (int i0 = 0; i0 < d_k; i0 += UNR) {
+            float s[UNR][C];
+#pragma unroll
+            for (int r = 0; r < UNR; ++r) {
+                const float* row = St + static_cast<int64_t>(i0 + r) * DV;
+                if constexpr (C == 4) {
+                    const float4 t = __ldcs(reinterpret_cast<const float4*>(row));
+                    s[r][0] = t.x; s[r][1] = t.y; s[r][2] = t.z; s[r][3] = t.w;
+                } else {
+                    const float2 t = __ldcs(reinterpret_cast<const float2*>(row));
+                    s[r][0] = t.x; s[r][1] = t.y;
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < UNR; ++r) {
+                const int i = i0 + r;
+                const float gi = GATE == kGatePerKey ? __ldg(gt + i) : alpha;
+                const float ki = __ldg(kt + i), qi = __ldg(qt + i);
+                float x[C];
+#pragma unroll
+                for (int c = 0; c < C; ++c) {
+                    x[c] = __fmaf_rn(gi, s[r][c], __fmul_rn(ki, w[c]));
+                    o[c] = __fmaf_rn(qi, x[c], o[c]);
+                }
+                float* row = St + static_cast<int64_t>(i) * DV;
+                if constexpr (C == 4)
+                    __stcs(reinterpret_cast<float4*>(row), make_float4(x[0], x[1], x[2], x[3]));
+                else
+                    __stcs(reinterpret_cast<float2*>(row), make_float2(x[0], x[1]));
+            }
+        }
+        float* op = out + static_cast<int64_t>(tile) * DV + lane * C;
+#pragma unroll
+        for (int c = 0; c < C; ++c) op[c] = o[c];
+    }
+}
+
+// ----------------------------------------------------------- decay mean ---
+
+// One block per head; a fixed assignment of elements to threads and a fixed
+// reduction tree make the binary64 sum deterministic.
+__global__ void decay_mean_kernel(const float* decay, int64_t outer, int heads, int64_t inner,
+                                  double* means) {
+    __shared__ double part[256];
+    const int h = blockIdx.x;
+    const int64_t n = outer * inner;
+    double acc = 0.0;
+    for (int64_t e = threadIdx.x; e < n; e += blockDim.x) {
+        const int64_t o = e / inner, c = e % inner;
+        acc += static_cast<double>(decay[(o * heads + h) * inner + c]);
+    }
+    part[threadIdx.x] = acc;
+    __syncthreads();
+    for (int s = 128; s > 0; s >>= 1) {
+        if (threadIdx.x < s) part[threadIdx.x] += part[threadIdx.x + s];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) means[h] = part[0] / static_cast<double>(n);
+}
+
+}  // namespace
+
+bool layout_kernels_support(int d_v, int group) {
+    const int C = d_v / 32;
+    return (C == 4 && (group == 16 || group == 32)) ||
+           (C == 2 && (group == 16 || group == 32 || group == 64));
+}
+
+cudaError_t launch_fill_zero(const LayoutArgs& a, cudaStream_t s) {
+    return launch_layout(a, kOpFillZero, nullptr, nullptr, nullptr, nullptr, nullptr, s);
+}
+cudaError_t launch_import_fp32(const LayoutArgs& a, const float* S, cudaStream_t s) {
+    return launch_layout(a, kOpImportFp32, S, nullptr, nullptr, nullptr, nullptr, s);
+}
+cudaError_t launch_export_fp32(const LayoutArgs& a, float* S, cudaStream_t s) {
+    return launch_layout(a, kOpExportFp32, nullptr, S, nullptr, nullptr, nullptr, s);
+}
+cudaError_t launch_export_codes(const LayoutArgs& a, int8_t* codes, cudaStream_t s) {
+    return launch_layout(a, kOpExportCodes, nullptr, nullptr, codes, nullptr, nullptr, s);
+}
+cudaError_t launch_import_codes(const LayoutArgs& a, const int8_t* codes, const float* scales,
+                                cudaStream_t s) {
+    return launch_layout(a, kOpImportCodes, nullptr, nullptr, nullptr, codes, scales, s);
+}
+
+cudaError_t launch_fp32_step(int B, int H, int d_k, int d_v, int update_kind, int gate_kind,
+                             float* S, const float* q, const float* k, const float* v,
+                             const float* gates, const float* beta, float* out, cudaStream_t s) {
+    const int ntiles = B * H;
+    if (ntiles == 0) return cudaSuccess;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int grid = (ntiles + kAuxWarps - 1) / kAuxWarps;
+    grid = grid < sms * 8 ? grid : sms * 8;
+    const int C = d_v / 32;
+#define LRS_FP32_CASE(CC, UU, GG)                                                           \
+    if (C == CC && update_kind == UU && gate_kind == GG) {                                  \
+        fp32_step_kernel<CC, UU, GG><<<grid, kAuxWarps * 32, 0, s>>>(ntiles, d_k, S, q, k, v, \
+                                                                    gates, beta, out);      \
+        return cudaGetLastError();                                                          \
+    }
+    LRS_FP32_CASE(4, kGated, kGatePerKey)
+    LRS_FP32_CASE(4, kGated, kGate)
+    LRS_FP32_CASE(4, kDelta, kGate)
+    LRS_FP32_CASE(2, kGated, kGatePerKey)
+    LRS_FP32_CASE(2, kGated, kGate)
+    LRS_FP32_CASE(2, kDelta, kGate)
+#undef LRS_FP32_CASE
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decay_means(const float* decay, int64_t outer, int heads, int64_t inner,
+                               double* means, cudaStream_t s) {
+    if (heads == 0) return cudaSuccess;
+    decay_mean_kernel<<<heads, 256, 0, s>>>(decay, outer, heads, inner, means);
+    return cudaGetLastError();
+}
+
+}  // namespace lrs

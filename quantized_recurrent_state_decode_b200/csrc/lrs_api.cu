@@ -1,0 +1,610 @@
+// lrs_api.cu -- the C ABI of liblrs (declared in include/lrs.h): argument
+// validation, the state's layout and memory, kernel selection and launch.
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "lrs.h"
+#include "lrs_internal.h"
+#include "step_kernel.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+lrs_status fail(lrs_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = std::string(lrs_status_string(s)) + ": " + buf;
+    return s;
+}
+
+lrs_status ok() {
+    g_last_error.clear();
+    return LRS_OK;
+}
+
+lrs_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(e == cudaErrorMemoryAllocation ? LRS_ERR_OOM : LRS_ERR_CUDA, "%s: %s", what,
+                cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------- per-device context ---
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceCtx {
+    unsigned* err = nullptr;  // device error word
+    int sms = 0;
+};
+
+std::mutex g_ctx_mu;
+DeviceCtx g_ctx[kMaxDevices];
+
+lrs_status device_ctx(DeviceCtx** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(LRS_ERR_UNSUPPORTED, "device index %d", dev);
+    std::lock_guard<std::mutex> lk(g_ctx_mu);
+    DeviceCtx& c = g_ctx[dev];
+    if (!c.err) {
+        e = cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        unsigned* p = nullptr;
+        e = cudaMalloc(&p, 256);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(error word)");
+        e = cudaMemset(p, 0, 256);
+        if (e != cudaSuccess) {
+            cudaFree(p);
+            return cuda_fail(e, "cudaMemset(error word)");
+        }
+        c.err = p;
+    }
+    *out = &c;
+    return LRS_OK;
+}
+
+// Fault injection (tests of the error path only).
+std::mutex g_inject_mu;
+bool g_inject = false;
+uint64_t g_inject_timeout_ns = 0;
+
+// Launch shape of the step kernel: warps per CTA (0 = derived from shared
+// memory). LRS_STEP_WARPS overrides it for launch-shape sweeps.
+int step_warps_override() {
+    static int v = [] {
+        const char* s = getenv("LRS_STEP_WARPS");
+        return s ? atoi(s) : 0;
+    }();
+    return v;
+}
+
+struct StatePriv {
+    int device = -1;
+    std::vector<uint8_t> prec_host;
+    std::vector<int64_t> offsets_host;
+    // device staging for lrs_decode_step_host (allocated on first use)
+    float* stage = nullptr;
+    size_t stage_floats = 0;
+};
+
+// ------------------------------------------------------------- layout ---
+
+lrs_status check_shape(const lrs_shape* s) {
+    if (!s) return fail(LRS_ERR_INVALID_ARG, "shape is NULL");
+    if (s->batch < 0 || s->heads < 1 || s->d_k < 1 || s->d_v < 1 || s->group < 1)
+        return fail(LRS_ERR_INVALID_ARG, "non-positive dimension (B=%d H=%d d_k=%d d_v=%d group=%d)",
+                    s->batch, s->heads, s->d_k, s->d_v, s->group);
+    if (s->update_kind != LRS_UPDATE_GATED && s->update_kind != LRS_UPDATE_DELTA)
+        return fail(LRS_ERR_INVALID_ARG, "update_kind %d", s->update_kind);
+    if (s->gate_kind != LRS_GATE_SCALAR && s->gate_kind != LRS_GATE_PER_KEY)
+        return fail(LRS_ERR_INVALID_ARG, "gate_kind %d", s->gate_kind);
+    if (s->update_kind == LRS_UPDATE_DELTA && s->gate_kind != LRS_GATE_SCALAR)
+        return fail(LRS_ERR_UNSUPPORTED, "the delta rule takes a scalar decay");
+    if (s->d_v != 64 && s->d_v != 128)
+        return fail(LRS_ERR_UNSUPPORTED, "d_v=%d (supported: 64, 128)", s->d_v);
+    if (s->group != 16 && s->group != 32 && s->group != 64)
+        return fail(LRS_ERR_UNSUPPORTED, "group=%d (supported: 16, 32, 64)", s->group);
+    if (s->group * s->d_v > 4096)
+        return fail(LRS_ERR_UNSUPPORTED, "group*d_v=%d exceeds 4096", s->group * s->d_v);
+    if (s->d_k % s->group != 0 || s->d_k < 16 || s->d_k > 256)
+        return fail(LRS_ERR_UNSUPPORTED, "d_k=%d (a multiple of group=%d in [16, 256])", s->d_k,
+                    s->group);
+    if (static_cast<int64_t>(s->batch) * s->heads > INT32_MAX / 2)
+        return fail(LRS_ERR_UNSUPPORTED, "batch*heads too large");
+    return LRS_OK;
+}
+
+lrs_status compute_layout(const lrs_shape* s, const uint8_t* prec, int64_t* offsets,
+                          int64_t* stride, int64_t* scale_count) {
+    lrs_status st = check_shape(s);
+    if (st != LRS_OK) return st;
+    if (!prec) return fail(LRS_ERR_INVALID_ARG, "prec_map is NULL");
+    int64_t off = 0;
+    for (int h = 0; h < s->heads; ++h) {
+        if (prec[h] != 4 && prec[h] != 8)
+            return fail(LRS_ERR_INVALID_ARG, "prec_map[%d]=%d (must be 4 or 8)", h, prec[h]);
+        if (offsets) offsets[h] = off;
+        off += static_cast<int64_t>(s->d_k) * s->d_v * prec[h] / 8;
+    }
+    if (stride) *stride = off;
+    if (scale_count)
+        *scale_count = static_cast<int64_t>(s->batch) * s->heads * (s->d_k / s->group) * s->d_v;
+    return LRS_OK;
+}
+
+lrs_status check_state(const lrs_state* st) {
+    if (!st || !st->priv) return fail(LRS_ERR_INVALID_ARG, "state is NULL or not allocated");
+    const StatePriv* pv = static_cast<const StatePriv*>(st->priv);
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev != pv->device)
+        return fail(LRS_ERR_INVALID_ARG, "state lives on device %d, current device is %d",
+                    pv->device, dev);
+    return check_shape(&st->shape);
+}
+
+lrs::LayoutArgs layout_args(const lrs_state* st, unsigned* err) {
+    lrs::LayoutArgs a;
+    a.codes = static_cast<uint8_t*>(st->state_codes);
+    a.scales = st->scales;
+    a.prec_map = st->prec_map;
+    a.head_offsets = st->head_offsets;
+    a.batch_stride = st->batch_stride_bytes;
+    a.B = st->shape.batch;
+    a.H = st->shape.heads;
+    a.d_k = st->shape.d_k;
+    a.d_v = st->shape.d_v;
+    a.group = st->shape.group;
+    a.err = err;
+    return a;
+}
+
+#define LRS_REQUIRE_PTR(p)                                                          \
+    do {                                                                            \
+        if (!(p)) return fail(LRS_ERR_INVALID_ARG, "%s is NULL", #p);               \
+        if (!aligned16(p)) return fail(LRS_ERR_ALIGNMENT, "%s is not 16-byte aligned", #p); \
+    } while (0)
+
+}  // namespace
+
+namespace lrs {
+
+const void* find_step_kernel(int C, int group, int update_kind, int gate_kind, int mode) {
+    switch (mode) {
+        case kRTN: return find_step_kernel_rtn(C, group, update_kind, gate_kind);
+        case kSR: return find_step_kernel_sr(C, group, update_kind, gate_kind);
+        case kBDR: return find_step_kernel_bdr(C, group, update_kind, gate_kind);
+        default: return nullptr;
+    }
+}
+
+int step_warp_smem(int C, int group, int gate_kind, int G) {
+#define LRS_SLOT(CC, GG)                                                                 \
+    if (C == CC && group == GG)                                                          \
+        return gate_kind == kGatePerKey ? Slot<CC, GG, kGatePerKey>::warp_bytes(G)       \
+                                        : Slot<CC, GG, kGate>::warp_bytes(G);
+    LRS_SLOT(4, 16)
+    LRS_SLOT(4, 32)
+    LRS_SLOT(2, 16)
+    LRS_SLOT(2, 32)
+    LRS_SLOT(2, 64)
+#undef LRS_SLOT
+    return -1;
+}
+
+}  // namespace lrs
+
+extern "C" {
+
+const char* lrs_status_string(lrs_status s) {
+    switch (s) {
+        case LRS_OK: return "LRS_OK";
+        case LRS_ERR_INVALID_ARG: return "LRS_ERR_INVALID_ARG";
+        case LRS_ERR_ALIGNMENT: return "LRS_ERR_ALIGNMENT";
+        case LRS_ERR_UNSUPPORTED: return "LRS_ERR_UNSUPPORTED";
+        case LRS_ERR_OOM: return "LRS_ERR_OOM";
+        case LRS_ERR_CUDA: return "LRS_ERR_CUDA";
+        case LRS_ERR_DEVICE_TIMEOUT: return "LRS_ERR_DEVICE_TIMEOUT";
+        case LRS_ERR_DEVICE_LAYOUT: return "LRS_ERR_DEVICE_LAYOUT";
+        case LRS_ERR_DEVICE_RANGE: return "LRS_ERR_DEVICE_RANGE";
+    }
+    return "LRS_ERR_UNKNOWN";
+}
+
+const char* lrs_last_error(void) { return g_last_error.c_str(); }
+
+int32_t lrs_version(void) { return LRS_VERSION; }
+
+lrs_status lrs_layout_query(const lrs_shape* shape, const uint8_t* prec_map_host,
+                            int64_t* head_offsets_host, int64_t* batch_stride_bytes,
+                            int64_t* scale_count) {
+    lrs_status s = compute_layout(shape, prec_map_host, head_offsets_host, batch_stride_bytes,
+                                  scale_count);
+    return s == LRS_OK ? ok() : s;
+}
+
+lrs_status lrs_state_alloc(const lrs_shape* shape, const uint8_t* prec_map_host, lrs_state* out) {
+    if (!out) return fail(LRS_ERR_INVALID_ARG, "out is NULL");
+    memset(out, 0, sizeof *out);
+    lrs_status s = check_shape(shape);
+    if (s != LRS_OK) return s;
+    std::vector<int64_t> offs(shape->heads);
+    int64_t stride = 0, nscales = 0;
+    s = compute_layout(shape, prec_map_host, offs.data(), &stride, &nscales);
+    if (s != LRS_OK) return s;
+    DeviceCtx* ctx = nullptr;
+    s = device_ctx(&ctx);
+    if (s != LRS_OK) return s;
+
+    StatePriv* pv = new StatePriv;
+    cudaGetDevice(&pv->device);
+    pv->prec_host.assign(prec_map_host, prec_map_host + shape->heads);
+    pv->offsets_host = offs;
+
+    lrs_state st;
+    memset(&st, 0, sizeof st);
+    st.shape = *shape;
+    st.batch_stride_bytes = stride;
+    st.code_bytes = stride * shape->batch;
+    st.scale_count = nscales;
+    st.priv = pv;
+    auto cleanup = [&](cudaError_t e, const char* what) {
+        cudaFree(st.state_codes);
+        cudaFree(st.scales);
+        cudaFree(st.prec_map);
+        cudaFree(st.head_offsets);
+        delete pv;
+        return cuda_fail(e, what);
+    };
+    cudaError_t e;
+    if ((e = cudaMalloc(&st.state_codes, std::max<int64_t>(st.code_bytes, 16))) != cudaSuccess)
+        return cleanup(e, "cudaMalloc(codes)");
+    if ((e = cudaMalloc(&st.scales, std::max<int64_t>(nscales, 4) * sizeof(float))) != cudaSuccess)
+        return cleanup(e, "cudaMalloc(scales)");
+    if ((e = cudaMalloc(&st.prec_map, std::max(shape->heads, 16))) != cudaSuccess)
+        return cleanup(e, "cudaMalloc(prec_map)");
+    if ((e = cudaMalloc(&st.head_offsets, shape->heads * sizeof(int64_t))) != cudaSuccess)
+        return cleanup(e, "cudaMalloc(head_offsets)");
+    if ((e = cudaMemcpy(st.prec_map, prec_map_host, shape->heads, cudaMemcpyHostToDevice)) !=
+        cudaSuccess)
+        return cleanup(e, "cudaMemcpy(prec_map)");
+    if ((e = cudaMemcpy(st.head_offsets, offs.data(), shape->heads * sizeof(int64_t),
+                        cudaMemcpyHostToDevice)) != cudaSuccess)
+        return cleanup(e, "cudaMemcpy(head_offsets)");
+    if ((e = lrs::launch_fill_zero(layout_args(&st, ctx->err), nullptr)) != cudaSuccess)
+        return cleanup(e, "zero fill");
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cleanup(e, "zero fill");
+    *out = st;
+    return ok();
+}
+
+lrs_status lrs_state_free(lrs_state* st) {
+    if (!st || !st->priv) return ok();
+    StatePriv* pv = static_cast<StatePriv*>(st->priv);
+    int prev = -1;
+    cudaGetDevice(&prev);
+    if (prev != pv->device) cudaSetDevice(pv->device);
+    cudaDeviceSynchronize();
+    cudaFree(st->state_codes);
+    cudaFree(st->scales);
+    cudaFree(st->prec_map);
+    cudaFree(st->head_offsets);
+    cudaFree(pv->stage);
+    if (prev != pv->device && prev >= 0) cudaSetDevice(prev);
+    delete pv;
+    memset(st, 0, sizeof *st);
+    return ok();
+}
+
+lrs_status lrs_decode_step(const lrs_state* st, void* state_codes, float* scales,
+                           const uint8_t* prec_map, const float* q, const float* k,
+                           const float* v, const float* gates, const float* beta, float* out,
+                           uint64_t seed, uint64_t step, int32_t mode, void* stream) {
+    lrs_status s = check_state(st);
+    if (s != LRS_OK) return s;
+    const lrs_shape& sh = st->shape;
+    LRS_REQUIRE_PTR(state_codes);
+    LRS_REQUIRE_PTR(scales);
+    if (!prec_map) return fail(LRS_ERR_INVALID_ARG, "prec_map is NULL");
+    LRS_REQUIRE_PTR(q);
+    LRS_REQUIRE_PTR(k);
+    LRS_REQUIRE_PTR(v);
+    LRS_REQUIRE_PTR(gates);
+    LRS_REQUIRE_PTR(out);
+    if (sh.update_kind == LRS_UPDATE_DELTA) LRS_REQUIRE_PTR(beta);
+    if (mode != LRS_ROUND_RTN && mode != LRS_ROUND_SR && mode != LRS_ROUND_BDR)
+        return fail(LRS_ERR_INVALID_ARG, "mode %d", mode);
+    const int C = sh.d_v / 32, G = sh.d_k / sh.group;
+    const void* fn = lrs::find_step_kernel(C, sh.group, sh.update_kind, sh.gate_kind, mode);
+    if (!fn) return fail(LRS_ERR_UNSUPPORTED, "no compiled kernel for this shape and mode");
+    DeviceCtx* ctx = nullptr;
+    s = device_ctx(&ctx);
+    if (s != LRS_OK) return s;
+    const int ntiles = sh.batch * sh.heads;
+    if (ntiles == 0) return ok();
+
+    const int warp_smem = lrs::step_warp_smem(C, sh.group, sh.gate_kind, G);
+    constexpr int kSmemLimit = 227 * 1024;
+    int warps = step_warps_override();
+    if (warps <= 0) warps = 8;
+    warps = std::min(warps, std::max(1, kSmemLimit / warp_smem));
+    warps = std::min(warps, 8);  // the kernel is compiled for at most 256 threads
+    const int smem = warps * warp_smem;
+
+    // per kernel and device: raise the dynamic shared memory limit once, and
+    // record how many CTAs fit on an SM
+    static std::mutex mu;
+    struct Cached { const void* fn; int dev; int smem; int per_sm; };
+    static std::vector<Cached> cache;
+    int per_sm = 0;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        const StatePriv* pv = static_cast<const StatePriv*>(st->priv);
+        for (const Cached& c : cache)
+            if (c.fn == fn && c.dev == pv->device && c.smem == smem) per_sm = c.per_sm;
+        if (per_sm == 0) {
+            cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, warps * 32, smem);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+            if (per_sm < 1) return fail(LRS_ERR_UNSUPPORTED, "step kernel does not fit on an SM");
+            cache.push_back({fn, pv->device, smem, per_sm});
+        }
+    }
+    int grid = ctx->sms * per_sm;
+    grid = std::min(grid, (ntiles + warps - 1) / warps);
+
+    lrs::StepParams p;
+    p.codes = static_cast<uint8_t*>(state_codes);
+    p.scales = scales;
+    p.prec_map = prec_map;
+    p.head_offsets = st->head_offsets;
+    p.batch_stride = st->batch_stride_bytes;
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.gates = gates;
+    p.beta = beta;
+    p.out = out;
+    p.seed = seed;
+    p.step = step;
+    p.err = ctx->err;
+    p.timeout_ns = 2000000000ull;  // 2 s: far above any legitimate wait
+    p.H = sh.heads;
+    p.d_k = sh.d_k;
+    p.G = G;
+    p.ntiles = ntiles;
+    p.warp_smem = warp_smem;
+    p.inject = 0;
+    {
+        std::lock_guard<std::mutex> lk(g_inject_mu);
+        if (g_inject) {
+            p.inject = 1;
+            p.timeout_ns = g_inject_timeout_ns;
+            g_inject = false;
+        }
+    }
+    void* args[] = {&p};
+    cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(warps * 32), args, smem,
+                                     static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the step kernel");
+    return ok();
+}
+
+lrs_status lrs_decode_step_host(const lrs_state* st, const float* q_host, const float* k_host,
+                                const float* v_host, const float* gates_host,
+                                const float* beta_host, float* out_host, uint64_t seed,
+                                uint64_t step, int32_t mode, void* stream) {
+    lrs_status s = check_state(st);
+    if (s != LRS_OK) return s;
+    const lrs_shape& sh = st->shape;
+    if (!q_host || !k_host || !v_host || !gates_host || !out_host)
+        return fail(LRS_ERR_INVALID_ARG, "a host buffer is NULL");
+    const bool delta = sh.update_kind == LRS_UPDATE_DELTA;
+    if (delta && !beta_host) return fail(LRS_ERR_INVALID_ARG, "beta_host is NULL");
+    const size_t T = static_cast<size_t>(sh.batch) * sh.heads;
+    // staging: q, k [T][d_k] | v, out [T][d_v] | gates [T][d_k or 1] | beta [T]
+    auto rnd = [](size_t n) { return (n + 3) / 4 * 4; };  // keep 16-byte alignment
+    const size_t nq = rnd(T * sh.d_k), nv = rnd(T * sh.d_v);
+    const size_t ng = rnd(sh.gate_kind == LRS_GATE_PER_KEY ? T * sh.d_k : T), nb = rnd(T);
+    const size_t need = 2 * nq + 2 * nv + ng + nb;
+    StatePriv* pv = static_cast<StatePriv*>(st->priv);
+    if (pv->stage_floats < need) {
+        cudaFree(pv->stage);
+        pv->stage = nullptr;
+        pv->stage_floats = 0;
+        cudaError_t e = cudaMalloc(&pv->stage, need * sizeof(float));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(staging)");
+        pv->stage_floats = need;
+    }
+    float* dq = pv->stage;
+    float* dk = dq + nq;
+    float* dv = dk + nq;
+    float* dout = dv + nv;
+    float* dg = dout + nv;
+    float* db = dg + ng;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const cudaMemcpyKind h2d = cudaMemcpyHostToDevice;
+    cudaError_t e;
+    if ((e = cudaMemcpyAsync(dq, q_host, T * sh.d_k * 4, h2d, cs)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(dk, k_host, T * sh.d_k * 4, h2d, cs)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(dv, v_host, T * sh.d_v * 4, h2d, cs)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(dg, gates_host,
+                             (sh.gate_kind == LRS_GATE_PER_KEY ? T * sh.d_k : T) * 4, h2d, cs)) !=
+            cudaSuccess ||
+        (delta && (e = cudaMemcpyAsync(db, beta_host, T * 4, h2d, cs)) != cudaSuccess))
+        return cuda_fail(e, "host-to-device copy of the step inputs");
+    s = lrs_decode_step(st, st->state_codes, st->scales, st->prec_map, dq, dk, dv, dg,
+                        delta ? db : nullptr, dout, seed, step, mode, stream);
+    if (s != LRS_OK) return s;
+    if ((e = cudaMemcpyAsync(out_host, dout, T * sh.d_v * 4, cudaMemcpyDeviceToHost, cs)) !=
+        cudaSuccess)
+        return cuda_fail(e, "device-to-host copy of the output");
+    return ok();
+}
+
+}  // extern "C"
+
+template <class Fn>
+static lrs_status layout_op(const lrs_state* st, void* stream, Fn&& fn) {
+    lrs_status s = check_state(st);
+    if (s != LRS_OK) return s;
+    DeviceCtx* ctx = nullptr;
+    s = device_ctx(&ctx);
+    if (s != LRS_OK) return s;
+    cudaError_t e = fn(layout_args(st, ctx->err), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "layout kernel launch");
+}
+
+extern "C" {
+
+lrs_status lrs_state_import_fp32(const lrs_state* st, const float* S, void* stream) {
+    LRS_REQUIRE_PTR(S);
+    return layout_op(st, stream, [&](const lrs::LayoutArgs& a, cudaStream_t s) {
+        return lrs::launch_import_fp32(a, S, s);
+    });
+}
+
+lrs_status lrs_state_export_fp32(const lrs_state* st, float* S, void* stream) {
+    LRS_REQUIRE_PTR(S);
+    return layout_op(st, stream, [&](const lrs::LayoutArgs& a, cudaStream_t s) {
+        return lrs::launch_export_fp32(a, S, s);
+    });
+}
+
+lrs_status lrs_state_export_codes(const lrs_state* st, int8_t* codes, void* stream) {
+    LRS_REQUIRE_PTR(codes);
+    return layout_op(st, stream, [&](const lrs::LayoutArgs& a, cudaStream_t s) {
+        return lrs::launch_export_codes(a, codes, s);
+    });
+}
+
+lrs_status lrs_state_import_codes(const lrs_state* st, const int8_t* codes, const float* scales,
+                                  void* stream) {
+    LRS_REQUIRE_PTR(codes);
+    LRS_REQUIRE_PTR(scales);
+    return layout_op(st, stream, [&](const lrs::LayoutArgs& a, cudaStream_t s) {
+        return lrs::launch_import_codes(a, codes, scales, s);
+    });
+}
+
+lrs_status lrs_state_copy_raw(const lrs_state* st, void* codes_host, float* scales_host,
+                              int32_t to_host, void* stream) {
+    lrs_status s = check_state(st);
+    if (s != LRS_OK) return s;
+    if (!codes_host || !scales_host) return fail(LRS_ERR_INVALID_ARG, "a host buffer is NULL");
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (to_host) {
+        if ((e = cudaMemcpyAsync(codes_host, st->state_codes, st->code_bytes,
+                                 cudaMemcpyDeviceToHost, cs)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(scales_host, st->scales, st->scale_count * sizeof(float),
+                                 cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
+            return cuda_fail(e, "copy to host");
+    } else {
+        if ((e = cudaMemcpyAsync(st->state_codes, codes_host, st->code_bytes,
+                                 cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(st->scales, scales_host, st->scale_count * sizeof(float),
+                                 cudaMemcpyHostToDevice, cs)) != cudaSuccess)
+            return cuda_fail(e, "copy from host");
+    }
+    if ((e = cudaStreamSynchronize(cs)) != cudaSuccess) return cuda_fail(e, "synchronize");
+    return ok();
+}
+
+lrs_status lrs_fp32_decode_step(const lrs_shape* shape, float* S, const float* q, const float* k,
+                                const float* v, const float* gates, const float* beta,
+                                float* out, void* stream) {
+    if (!shape) return fail(LRS_ERR_INVALID_ARG, "shape is NULL");
+    const lrs_shape& sh = *shape;
+    if (sh.batch < 0 || sh.heads < 1 || sh.d_k < 1)
+        return fail(LRS_ERR_INVALID_ARG, "non-positive dimension");
+    if (sh.update_kind != LRS_UPDATE_GATED && sh.update_kind != LRS_UPDATE_DELTA)
+        return fail(LRS_ERR_INVALID_ARG, "update_kind %d", sh.update_kind);
+    if (sh.gate_kind != LRS_GATE_SCALAR && sh.gate_kind != LRS_GATE_PER_KEY)
+        return fail(LRS_ERR_INVALID_ARG, "gate_kind %d", sh.gate_kind);
+    if (sh.update_kind == LRS_UPDATE_DELTA && sh.gate_kind != LRS_GATE_SCALAR)
+        return fail(LRS_ERR_UNSUPPORTED, "the delta rule takes a scalar decay");
+    if (sh.d_v != 64 && sh.d_v != 128)
+        return fail(LRS_ERR_UNSUPPORTED, "d_v=%d (supported: 64, 128)", sh.d_v);
+    if (sh.d_k % 8 != 0 || sh.d_k > 1024)
+        return fail(LRS_ERR_UNSUPPORTED, "d_k=%d (a multiple of 8, at most 1024)", sh.d_k);
+    LRS_REQUIRE_PTR(S);
+    LRS_REQUIRE_PTR(q);
+    LRS_REQUIRE_PTR(k);
+    LRS_REQUIRE_PTR(v);
+    LRS_REQUIRE_PTR(gates);
+    LRS_REQUIRE_PTR(out);
+    if (sh.update_kind == LRS_UPDATE_DELTA) LRS_REQUIRE_PTR(beta);
+    cudaError_t e = lrs::launch_fp32_step(sh.batch, sh.heads, sh.d_k, sh.d_v, sh.update_kind,
+                                          sh.gate_kind, S, q, k, v, gates, beta, out,
+                                          static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "launch of the fp32 step kernel");
+}
+
+lrs_status lrs_decay_head_means(const float* decay, int64_t outer, int32_t heads, int64_t inner,
+                                double* means, void* stream) {
+    if (outer < 1 || heads < 1 || inner < 1)
+        return fail(LRS_ERR_INVALID_ARG, "outer=%lld heads=%d inner=%lld", (long long)outer, heads,
+                    (long long)inner);
+    LRS_REQUIRE_PTR(decay);
+    LRS_REQUIRE_PTR(means);
+    cudaError_t e = lrs::launch_decay_means(decay, outer, heads, inner, means,
+                                            static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "launch of the decay-mean kernel");
+}
+
+lrs_status lrs_precision_map(int32_t heads, const double* means_host, int32_t n_int8,
+                             uint8_t* prec_map_host) {
+    if (heads < 1 || !means_host || !prec_map_host || n_int8 < 0 || n_int8 > heads)
+        return fail(LRS_ERR_INVALID_ARG, "heads=%d n_int8=%d", heads, n_int8);
+    std::vector<int> order(heads);
+    for (int h = 0; h < heads; ++h) order[h] = h;
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int a, int b) { return means_host[a] > means_host[b]; });
+    for (int h = 0; h < heads; ++h) prec_map_host[h] = 4;
+    for (int n = 0; n < n_int8; ++n) prec_map_host[order[n]] = 8;
+    return ok();
+}
+
+lrs_status lrs_sync(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    DeviceCtx* ctx = nullptr;
+    lrs_status s = device_ctx(&ctx);
+    if (s != LRS_OK) return s;
+    unsigned flags = 0;
+    e = cudaMemcpy(&flags, ctx->err, sizeof flags, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "read of the device error word");
+    if (flags == 0) return ok();
+    e = cudaMemset(ctx->err, 0, sizeof flags);
+    if (e != cudaSuccess) return cuda_fail(e, "reset of the device error word");
+    if (flags & lrs::kErrTimeout)
+        return fail(LRS_ERR_DEVICE_TIMEOUT, "a step kernel timed out waiting for its copies");
+    if (flags & lrs::kErrLayout)
+        return fail(LRS_ERR_DEVICE_LAYOUT, "prec_map does not fit the state's tile layout");
+    return fail(LRS_ERR_DEVICE_RANGE, "an imported code was outside [-qmax, qmax]");
+}
+
+lrs_status lrs_debug_inject_timeout(int32_t enable, int32_t timeout_us) {
+    if (enable && timeout_us < 1) return fail(LRS_ERR_INVALID_ARG, "timeout_us=%d", timeout_us);
+    std::lock_guard<std::mutex> lk(g_inject_mu);
+    g_inject = enable != 0;
+    g_inject_timeout_ns = static_cast<uint64_t>(timeout_us) * 1000ull;
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,43 @@
+// lrs_internal.h -- declarations shared by liblrs's translation units (host side).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace lrs {
+
+// Kernel entry of one compiled step variant, or nullptr when the combination
+// (columns per lane C = d_v/32, group rows, update kind, gate kind, rounding
+// mode) is not compiled.
+const void* find_step_kernel(int C, int group, int update_kind, int gate_kind, int mode);
+const void* find_step_kernel_rtn(int C, int group, int update_kind, int gate_kind);
+const void* find_step_kernel_sr(int C, int group, int update_kind, int gate_kind);
+const void* find_step_kernel_bdr(int C, int group, int update_kind, int gate_kind);
+
+// Bytes of shared memory one warp of the step kernel uses.
+int step_warp_smem(int C, int group, int gate_kind, int G);
+
+struct LayoutArgs {
+    uint8_t* codes;
+    float* scales;
+    const uint8_t* prec_map;
+    const int64_t* head_offsets;
+    int64_t batch_stride;
+    int32_t B, H, d_k, d_v, group;
+    unsigned* err;
+};
+
+cudaError_t launch_fill_zero(const LayoutArgs& a, cudaStream_t s);
+cudaError_t launch_import_fp32(const LayoutArgs& a, const float* S, cudaStream_t s);
+cudaError_t launch_export_fp32(const LayoutArgs& a, float* S, cudaStream_t s);
+cudaError_t launch_export_codes(const LayoutArgs& a, int8_t* codes, cudaStream_t s);
+cudaError_t launch_import_codes(const LayoutArgs& a, const int8_t* codes, const float* scales,
+                                cudaStream_t s);
+cudaError_t launch_fp32_step(int B, int H, int d_k, int d_v, int update_kind, int gate_kind,
+                             float* S, const float* q, const float* k, const float* v,
+                             const float* gates, const float* beta, float* out, cudaStream_t s);
+cudaError_t launch_decay_means(const float* decay, int64_t outer, int heads, int64_t inner,
+                               double* means, cudaStream_t s);
+bool layout_kernels_support(int d_v, int group);
+
+}  // namespace lrs

@@ -5,9 +5,11 @@ method is evaluated on (GLA, Gated DeltaNet and Mamba2-SSD decode). It holds
 none of the decode step's arithmetic, and it is the one module that both the
 CUDA path's callers and the CPU oracle's callers use.
 
-All draws come from CPU ``torch.Generator`` streams seeded per
-(workload, tensor, step), so any step's inputs can be regenerated on their own.
-Tensors are float32 and C-contiguous:
+All draws come from ``torch.Generator`` streams seeded per (workload, tensor,
+step), so any step's inputs can be regenerated on their own. Draws are made on
+the device the caller names (CPU by default); a CUDA generator gives other
+numbers than a CPU one, so a comparison takes both of its sides from one
+device's draws. Tensors are float32 and C-contiguous:
 
   q, k   [B][H][d_k]       v   [B][H][d_v]
   gates  [B][H][d_k] (per-key decay) or [B][H] (scalar decay), already the
@@ -102,29 +104,30 @@ WORKLOADS = {
 }
 
 
-def _gen(w: Workload, tensor: int, t: int) -> torch.Generator:
-    g = torch.Generator(device="cpu")
+def _gen(w: Workload, tensor: int, t: int, device="cpu") -> torch.Generator:
+    g = torch.Generator(device=device)
     g.manual_seed(1_000_003 * w.seed_id + 10_007 * tensor + t)
     return g
 
 
 def _normal(shape, gen, mean=0.0, std=1.0):
-    return torch.randn(shape, generator=gen, dtype=torch.float32) * std + mean
+    return torch.randn(shape, generator=gen, dtype=torch.float32, device=gen.device) * std + mean
 
 
 def _unit_rows(x):
     return x / torch.linalg.vector_norm(x, dim=-1, keepdim=True)
 
 
-def head_log_decay_rates(w: Workload) -> torch.Tensor:
+def head_log_decay_rates(w: Workload, device="cpu") -> torch.Tensor:
     """Mamba2 per-head A_h = -exp(U(0, 2)); empty for other families."""
     if w.family != "mamba2":
-        return torch.empty(0)
-    g = _gen(w, _T_HEAD, 0)
-    return -torch.exp(torch.rand(w.heads, generator=g, dtype=torch.float32) * 2.0)
+        return torch.empty(0, device=device)
+    g = _gen(w, _T_HEAD, 0, device)
+    return -torch.exp(torch.rand(w.heads, generator=g, dtype=torch.float32, device=device) * 2.0)
 
 
-def step_inputs(w: Workload, t: int, batch_offset: int = 0, batch: Optional[int] = None):
+def step_inputs(w: Workload, t: int, batch_offset: int = 0, batch: Optional[int] = None,
+                device="cpu"):
     """Inputs of decode step t (0-based) for batch rows [batch_offset, +batch).
 
     Rows are drawn for the whole batch and sliced, so a batch shard sees the
@@ -134,23 +137,23 @@ def step_inputs(w: Workload, t: int, batch_offset: int = 0, batch: Optional[int]
     if batch is None:
         batch = B - batch_offset
     sl = slice(batch_offset, batch_offset + batch)
-    q = _normal((B, H, dk), _gen(w, _T_Q, t))
-    k = _normal((B, H, dk), _gen(w, _T_K, t))
-    v = _normal((B, H, dv), _gen(w, _T_V, t))
+    q = _normal((B, H, dk), _gen(w, _T_Q, t, device))
+    k = _normal((B, H, dk), _gen(w, _T_K, t, device))
+    v = _normal((B, H, dv), _gen(w, _T_V, t, device))
     beta = None
     if w.family == "gla":
         k = _unit_rows(k)
-        z = _normal((B, H, dk), _gen(w, _T_G, t), mean=w.gate_mu)
+        z = _normal((B, H, dk), _gen(w, _T_G, t, device), mean=w.gate_mu)
         gates = torch.exp(-torch.nn.functional.softplus(z))
     elif w.family == "gdn":
         k = _unit_rows(k)
-        gates = torch.sigmoid(_normal((B, H), _gen(w, _T_G, t), mean=w.gate_mu))
-        beta = torch.sigmoid(_normal((B, H), _gen(w, _T_BETA, t)))
+        gates = torch.sigmoid(_normal((B, H), _gen(w, _T_G, t, device), mean=w.gate_mu))
+        beta = torch.sigmoid(_normal((B, H), _gen(w, _T_BETA, t, device)))
     elif w.family == "mamba2":
         # B_t plays k, C_t plays q, x_t scaled by dt plays v; decay exp(dt*A_h).
-        dt = torch.nn.functional.softplus(_normal((B, H), _gen(w, _T_G, t), mean=w.gate_mu,
-                                                  std=0.5))
-        A = head_log_decay_rates(w)
+        dt = torch.nn.functional.softplus(_normal((B, H), _gen(w, _T_G, t, device),
+                                                  mean=w.gate_mu, std=0.5))
+        A = head_log_decay_rates(w, device)
         gates = torch.exp(dt * A[None, :])
         v = v * dt[:, :, None]
     else:
@@ -160,24 +163,25 @@ def step_inputs(w: Workload, t: int, batch_offset: int = 0, batch: Optional[int]
     return {n: (None if x is None else x.contiguous()) for n, x in out.items()}
 
 
-def initial_state(w: Workload, batch_offset: int = 0, batch: Optional[int] = None):
+def initial_state(w: Workload, batch_offset: int = 0, batch: Optional[int] = None,
+                  device="cpu"):
     """S0 [B][H][d_k][d_v]: zeros, or N(0, s0_std^2)."""
     if batch is None:
         batch = w.batch - batch_offset
     shape = (batch, w.heads, w.d_k, w.d_v)
     if w.s0_std == 0.0:
-        return torch.zeros(shape, dtype=torch.float32)
-    full = _normal((w.batch, w.heads, w.d_k, w.d_v), _gen(w, _T_S0, 0), std=w.s0_std)
+        return torch.zeros(shape, dtype=torch.float32, device=device)
+    full = _normal((w.batch, w.heads, w.d_k, w.d_v), _gen(w, _T_S0, 0, device), std=w.s0_std)
     return full[batch_offset:batch_offset + batch].contiguous()
 
 
-def decay_tensor(w: Workload, steps: Optional[int] = None):
+def decay_tensor(w: Workload, steps: Optional[int] = None, device="cpu"):
     """All decay values of the run, [steps*B][H][inner] (inner = d_k or 1),
     the input of the decay-based precision map."""
     steps = w.steps if steps is None else steps
     parts = []
     for t in range(steps):
-        g = step_inputs(w, t)["gates"]
+        g = step_inputs(w, t, device=device)["gates"]
         parts.append(g.reshape(w.batch, w.heads, -1))
     return torch.cat(parts, 0).contiguous()
 
