@@ -11,8 +11,9 @@
  *   3. output      o_j = sum_i q_i x_ij over the updated state
  *   4. new scales  per (group of key rows, value column): absmax / qmax
  *                                                      [LoReS value-axis grouping]
- *   5. requantize  round-to-nearest, stochastic rounding  [LoReS], or
- *                  Bounded Directional Rounding           [LRB/BDR]
+ *   5. requantize  x * qmax / absmax rounded to an integer: to nearest,
+ *                  stochastically [LoReS], or by Bounded Directional
+ *                  Rounding [LRB/BDR]
  */
 #include "lrs_oracle.h"
 
@@ -58,36 +59,39 @@ float orc_uniform(uint64_t r)
 /* ---------------------------------------------------------- rounding --- */
 
 /* Code for one element. x: the updated value; deq: its value before the
- * update (dequantized old state); y = x * inv; s_new: the new scale. */
-static int round_element(int mode, float x, float deq, float y, float s_new, int qmax,
+ * update (dequantized old state); inv = qmax / A; s_new: the new scale.
+ * The value to round is the exact product y = x * inv (a product of two
+ * binary32 numbers is exact in binary64); it is rounded once, to an integer. */
+static int round_element(int mode, float x, float deq, float inv, float s_new, int qmax,
                          uint64_t r)
 {
-    float c;
+    double y = (double)x * (double)inv;
+    double c;
     if (mode == ORC_ROUND_SR) {
         /* [LoReS] stochastic rounding: up with probability equal to the
-         * fractional part. */
-        float f = floorf(y);
-        float fr = y - f;
+         * fractional part, here y - floor(y) rounded once to binary32. */
+        double f = floor(y);
+        float fr = fmaf(x, inv, (float)-f);
         float u = orc_uniform(r);
-        c = (u < fr) ? f + 1.0f : f;
+        c = (u < fr) ? f + 1.0 : f;
     } else if (mode == ORC_ROUND_BDR) {
         /* [LRB/BDR]: the update is delta = x - deq; the move the stored value
          * would make is m = c0*s_new - deq. When the two point in opposite
          * directions the element is rounded toward the update instead. */
-        float c0 = rintf(y);
+        double c0 = rint(y);
         float delta = x - deq;
-        float m = c0 * s_new - deq;
+        float m = (float)c0 * s_new - deq;
         if (delta > 0.0f && m < 0.0f)
-            c = ceilf(y);
+            c = ceil(y);
         else if (delta < 0.0f && m > 0.0f)
-            c = floorf(y);
+            c = floor(y);
         else
             c = c0;
     } else {
-        c = rintf(y); /* round half to even (default rounding mode) */
+        c = rint(y); /* round half to even (default rounding mode) */
     }
-    if (c > (float)qmax) c = (float)qmax;
-    if (c < (float)-qmax) c = (float)-qmax;
+    if (c > (double)qmax) c = (double)qmax;
+    if (c < (double)-qmax) c = (double)-qmax;
     return (int)c;
 }
 
@@ -116,11 +120,10 @@ static void requantize_tile(int d_k, int d_v, int group, int qmax, int mode, con
             scales[g * d_v + j] = s_new;
             for (int i = g * group; i < (g + 1) * group; ++i) {
                 float xv = x[i * d_v + j];
-                float y = xv * inv;
                 uint64_t r = 0;
                 if (mode == ORC_ROUND_SR) r = orc_hash(seed, step, b, h, (uint32_t)i, (uint32_t)j);
                 float dv = deq ? deq[i * d_v + j] : 0.0f;
-                codes[i * d_v + j] = (int8_t)round_element(mode, xv, dv, y, s_new, qmax, r);
+                codes[i * d_v + j] = (int8_t)round_element(mode, xv, dv, inv, s_new, qmax, r);
             }
         }
     }

@@ -110,7 +110,7 @@ def _run_case(c, mode, seed=0, step=0):
 
 @pytest.mark.parametrize("name", ["hand_gla_int8_rtn_4x2.txt", "hand_gla_int8_bdr_2x2.txt",
                                   "hand_gdn_int4_rtn_2x2.txt", "hand_gla_int8_ties_2x2.txt",
-                                  "hand_clamp_int8_1x2.txt"])
+                                  "hand_clamp_int8_1x2.txt", "hand_exact_product_int8_2x2.txt"])
 def test_hand_examples_rtn(name):
     c = _load_case(name)
     codes, scales, out = _run_case(c, oracle.ROUND_RTN)
@@ -120,7 +120,8 @@ def test_hand_examples_rtn(name):
     np.testing.assert_array_equal(codes, expect)
 
 
-@pytest.mark.parametrize("name", ["hand_gla_int8_bdr_2x2.txt", "hand_clamp_int8_1x2.txt"])
+@pytest.mark.parametrize("name", ["hand_gla_int8_bdr_2x2.txt", "hand_clamp_int8_1x2.txt",
+                                  "hand_exact_product_int8_2x2.txt"])
 def test_hand_example_bdr(name):
     c = _load_case(name)
     codes, scales, out = _run_case(c, oracle.ROUND_BDR)
@@ -157,8 +158,8 @@ def test_sr_codes_clamped_to_symmetric_range():
     seed = int(fx["seed"][0])
     c = _load_case("hand_clamp_int8_1x2.txt")
     up, down = int(fx["step_up"][0]), int(fx["step_down"][0])
-    assert oracle.uniform(oracle.hash64(seed, up, 0, 0, 0, 0)) < 2.0 ** -17
-    assert oracle.uniform(oracle.hash64(seed, down, 0, 0, 0, 1)) >= 1 - 2.0 ** -17
+    assert oracle.uniform(oracle.hash64(seed, up, 0, 0, 0, 0)) < 5 * 2.0 ** -20
+    assert oracle.uniform(oracle.hash64(seed, down, 0, 0, 0, 1)) >= 1 - 5 * 2.0 ** -20
     for step in (up, down, 0):
         codes, _, _ = _run_case(c, oracle.ROUND_SR, seed=seed, step=step)
         np.testing.assert_array_equal(codes, [[127, -127]])
@@ -397,7 +398,7 @@ def test_bdr_never_moves_against_update(bits):
         sc = np.repeat(scales, group, axis=1)
         inv = np.where(sc > 0, F32(qmax) / np.where(sc > 0, np.repeat(
             np.abs(x).reshape(2, -1, group, x.shape[2]).max(axis=2), group, axis=1), 1), 0)
-        y = (x * inv.astype(F32)).astype(F32)
+        y = x.astype(np.float64) * inv.astype(F32).astype(np.float64)   # exact product
         delta = (x - deq).astype(F32)
         moved = ((codes.astype(F32) * sc).astype(F32) - deq).astype(F32)
         bounded_up = codes == np.clip(np.ceil(y), -qmax, qmax)
