@@ -110,7 +110,8 @@ def _run_case(c, mode, seed=0, step=0):
 
 @pytest.mark.parametrize("name", ["hand_gla_int8_rtn_4x2.txt", "hand_gla_int8_bdr_2x2.txt",
                                   "hand_gdn_int4_rtn_2x2.txt", "hand_gla_int8_ties_2x2.txt",
-                                  "hand_clamp_int8_1x2.txt", "hand_exact_product_int8_2x2.txt"])
+                                  "hand_clamp_int8_1x2.txt", "hand_exact_product_int8_2x2.txt",
+                                  "hand_bdr_zero_move_int8_2x2.txt"])
 def test_hand_examples_rtn(name):
     c = _load_case(name)
     codes, scales, out = _run_case(c, oracle.ROUND_RTN)
@@ -120,8 +121,11 @@ def test_hand_examples_rtn(name):
     np.testing.assert_array_equal(codes, expect)
 
 
-@pytest.mark.parametrize("name", ["hand_gla_int8_bdr_2x2.txt", "hand_clamp_int8_1x2.txt",
-                                  "hand_exact_product_int8_2x2.txt"])
+HAND_BDR = ["hand_gla_int8_bdr_2x2.txt", "hand_clamp_int8_1x2.txt",
+            "hand_exact_product_int8_2x2.txt", "hand_bdr_zero_move_int8_2x2.txt"]
+
+
+@pytest.mark.parametrize("name", HAND_BDR)
 def test_hand_example_bdr(name):
     c = _load_case(name)
     codes, scales, out = _run_case(c, oracle.ROUND_BDR)
