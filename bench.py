@@ -207,8 +207,10 @@ def config_of(w, mode, layers, n):
 # -------------------------------------------------------------------- GPU ---
 
 def state_bytes(w, prec_bits=8):
+    """Algorithmic bytes of one step: codes and scales, each read once and
+    written once."""
     G = w.d_k // w.group
-    return w.batch * w.heads * (w.d_k * w.d_v * prec_bits // 8 + G * w.d_v * 4)
+    return 2 * w.batch * w.heads * (w.d_k * w.d_v * prec_bits // 8 + G * w.d_v * 4)
 
 
 def run_gpu(args, w):
@@ -449,11 +451,14 @@ def cpu_baseline(w, mode):
     pm = I.uniform_prec_map(w).numpy()
     S0 = I.initial_state(w)[tb, th].numpy()
     codes, scales = oracle.import_fp32(S0, pm, th, group=w.group)
+    xs = []
+    for t in range(4):
+        x = I.step_inputs(w, t)
+        xs.append({k: (None if v is None else v[tb, th].numpy().reshape(n, -1))
+                   for k, v in x.items()})
     reps, el = 0, 0.0
-    t_end = time.perf_counter() + 12.0
-    while time.perf_counter() < t_end or reps == 0:
-        x = I.step_inputs(w, reps)
-        sel = {k: (None if v is None else v[tb, th].numpy().reshape(n, -1)) for k, v in x.items()}
+    while el < 12.0 or reps == 0:
+        sel = xs[reps % len(xs)]
         t0 = time.perf_counter()
         oracle.step(codes, scales, sel["q"], sel["k"], sel["v"], sel["gates"],
                     None if sel["beta"] is None else sel["beta"].reshape(-1), pm, tb, th,

@@ -85,14 +85,15 @@ typedef struct {
  * tile starts at byte head_offsets[h] of the row and has d_k*d_v*bits/8 bytes
  * (bits = prec_map[h]). Tile (b, h) starts at b*batch_stride_bytes +
  * head_offsets[h]. Inside a tile, lane t of 32 owns value columns
- * [t*d_v/32, (t+1)*d_v/32) for every key row; its codes, row-major over
- * (row, its columns), form a byte stream cut into 16-byte units, and unit u of
- * lane t sits at tile byte (u*32 + t)*16. Within each 32-bit little-endian
- * word of the stream: int8 holds 4 consecutive elements, byte n = element n;
- * int4 holds 8 consecutive elements e0..e7, byte n = e_n | e_(n+4) << 4.
- * Codes are stored in offset binary: the byte (nibble) is code + 128 (+ 8).
- * The key rows of one scale group are therefore one contiguous
- * group*d_v*bits/8-byte block of the tile.
+ * [t*C, t*C + C), C = d_v/32, for every key row. Its codes are ordered by
+ * scale group, then by column pair p (columns t*C + 2p and t*C + 2p + 1),
+ * then by key row, then by column within the pair; this byte stream is cut
+ * into 16-byte units, and unit u of lane t sits at tile byte (u*32 + t)*16.
+ * Within each 32-bit little-endian word of the stream: int8 holds 4
+ * consecutive elements, byte n = element n; int4 holds 8 consecutive
+ * elements e0..e7, byte n = e_n | e_(n+4) << 4. Codes are stored in offset
+ * binary: the byte (nibble) is code + 128 (+ 8). The key rows of one scale
+ * group are therefore one contiguous group*d_v*bits/8-byte block of the tile.
  *
  * Scale layout: fp32 [B][H][d_k/group][d_v]. A value dequantizes as
  * code * scale[b][h][i/group][j]. */
@@ -135,16 +136,18 @@ lrs_status lrs_state_free(lrs_state *st);
  *   out_j  = sum_i q_i x_ij                    (i ascending, fused)
  *   A      = max |x_ij| over each group's rows, per column; scale' = A/qmax,
  *            inv = qmax/A (both 0 when A < 2^-100); qmax = 127 or 7
- *   y      = x_ij * inv, code' = round(y) clamped to [-qmax, qmax] by
+ *   y      = x_ij * inv taken exactly (the product is not rounded first);
+ *            code' = an integer from y, clamped to [-qmax, qmax]:
  *     LRS_ROUND_RTN  nearest, ties to even
- *     LRS_ROUND_SR   floor(y) + [u < y - floor(y)], u = top 23 bits of the
+ *     LRS_ROUND_SR   floor(y) + [u < fr], fr = y - floor(y) rounded once to
+ *                    binary32, u = top 23 bits of the
  *                    hash H(seed, step, b, h, i, j) times 2^-23, where
  *                    H = m(m(m(m(seed) ^ step) ^ (b<<32|h)) ^ (i<<32|j)) and
  *                    m is the SplitMix64 output function (add 0x9E3779B97F4A7C15,
  *                    then its 64-bit mixer)
  *     LRS_ROUND_BDR  nearest, except that when the update d = x - deq and the
- *                    move m = nearest*scale' - deq have opposite signs the
- *                    code is ceil(y) (d > 0) or floor(y) (d < 0)
+ *                    move m = RN(RN(nearest*scale') - deq) have opposite signs
+ *                    the code is ceil(y) (d > 0) or floor(y) (d < 0)
  * Every operation is binary32 with round-to-nearest-even; results are
  * deterministic and independent of the launch configuration.
  *

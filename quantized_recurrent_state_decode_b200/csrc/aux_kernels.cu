@@ -2,7 +2,7 @@
 // decode step used as the uncompressed baseline, and the per-head mean decay.
 //
 // The quantizing kernels here share the step kernel's rounding and packing
-// (round_code / encode_word), so an imported state is exactly the state a step
+// (round_pair / encode_word), so an imported state is exactly the state a step
 // with x = S would produce.
 #include "lrs_internal.h"
 #include "step_kernel.cuh"
@@ -13,7 +13,7 @@ namespace {
 
 constexpr int kAuxWarps = 8;
 
-// Byte offset, inside a tile, of the 16-byte unit `u` of lane `lane`.
+// Byte offset, inside a group block, of the 16-byte unit `u` of lane `lane`.
 __device__ __forceinline__ int unit_offset(int u, int lane) { return (u * 32 + lane) * 16; }
 
 struct TileRef {
@@ -33,63 +33,51 @@ __device__ __forceinline__ TileRef tile_ref(const LayoutArgs& a, int tile) {
     return t;
 }
 
-// Quantize x[GROUP][C] (this lane's columns of one group) with round to
-// nearest into the tile's group block and scales row.
-template <int C, int GROUP, int BITS>
-__device__ void quantize_group_rtn(const float (&x)[GROUP][C], uint8_t* gcodes, float* gscales,
-                                   int lane) {
-    constexpr int EPW = 32 / BITS;
-    constexpr int UNITS = GROUP * C * BITS / 8 / 16;
-    constexpr float QMAX = BITS == 8 ? 127.0f : 7.0f;
-    float snew[C], inv[C];
+// Round x * inv (inv = 1 for given integer codes) to nearest for one column
+// pair of one group and store the pair's units (same rounding and packing as
+// the step kernel).
+template <int GROUP, int BITS>
+__device__ void encode_pair_rtn(const float2 (&x)[GROUP], float2 inv, uint8_t* gcodes, int pc,
+                                int lane) {
+    using G = PairGeo<GROUP, BITS>;
 #pragma unroll
-    for (int c = 0; c < C; ++c) {
-        float A = 0.0f;
-#pragma unroll
-        for (int r = 0; r < GROUP; ++r) A = fmaxf(A, fabsf(x[r][c]));
-        const bool zero = A < kTiny;
-        snew[c] = zero ? 0.0f : __fdiv_rn(A, QMAX);
-        inv[c] = zero ? 0.0f : __fdiv_rn(QMAX, A);
-        gscales[lane * C + c] = snew[c];
-    }
-#pragma unroll
-    for (int un = 0; un < UNITS; ++un) {
+    for (int un = 0; un < G::UNITS; ++un) {
         uint32_t ow[4];
 #pragma unroll
         for (int wi = 0; wi < 4; ++wi) {
-            float t[EPW];
+            float t[G::EPW];
 #pragma unroll
-            for (int e = 0; e < EPW; ++e) {
-                const int el = (un * 4 + wi) * EPW + e;
-                const int r = el / C, c = el % C;
-                t[e] = round_code<kRTN, BITS>(__fmul_rn(x[r][c], inv[c]), 0.f, 0.f, 0.f, 0ull, 0u,
-                                              0u);
+            for (int e = 0; e < G::EPW; e += 2) {
+                const int r = un * G::RPU + (wi * G::EPW + e) / 2;
+                const float2 tv = round_pair<kRTN, BITS>(x[r], inv, f2(0.f), f2(0.f), 0ull, 0u, 0u);
+                t[e] = tv.x;
+                t[e + 1] = tv.y;
             }
             ow[wi] = encode_word<BITS>(t);
         }
-        *reinterpret_cast<uint4*>(gcodes + unit_offset(un, lane)) =
+        *reinterpret_cast<uint4*>(gcodes + unit_offset(pc * G::UNITS + un, lane)) =
             make_uint4(ow[0], ow[1], ow[2], ow[3]);
     }
 }
 
-// Signed codes of one group block, code[r][c] for this lane's columns.
-template <int C, int GROUP, int BITS>
-__device__ void decode_group(const uint8_t* gcodes, int lane, float (&code)[GROUP][C]) {
-    constexpr int EPW = 32 / BITS;
-    constexpr int UNITS = GROUP * C * BITS / 8 / 16;
+// Signed codes of one column pair of one group block.
+template <int GROUP, int BITS>
+__device__ void decode_pair(const uint8_t* gcodes, int pc, int lane, float2 (&code)[GROUP]) {
+    using G = PairGeo<GROUP, BITS>;
+    constexpr float BIAS = Q<BITS>::kBias;
 #pragma unroll
-    for (int un = 0; un < UNITS; ++un) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(gcodes + unit_offset(un, lane));
+    for (int un = 0; un < G::UNITS; ++un) {
+        const uint4 raw =
+            *reinterpret_cast<const uint4*>(gcodes + unit_offset(pc * G::UNITS + un, lane));
         const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
         for (int wi = 0; wi < 4; ++wi) {
-            float f[EPW];
-            decode_word<BITS>(wd[wi], f);
+            float f[G::EPW];
+            decode_word_biased<BITS>(wd[wi], f);
 #pragma unroll
-            for (int e = 0; e < EPW; ++e) {
-                const int el = (un * 4 + wi) * EPW + e;
-                code[el / C][el % C] = f[e];
-            }
+            for (int e = 0; e < G::EPW; e += 2)
+                code[un * G::RPU + (wi * G::EPW + e) / 2] =
+                    make_float2(__fsub_rn(f[e], kTwo23 + BIAS), __fsub_rn(f[e + 1], kTwo23 + BIAS));
         }
     }
 }
@@ -101,74 +89,69 @@ __device__ void layout_op_tile(const LayoutArgs& a, int op, int tile, uint8_t* t
                                const float* S, float* So, int8_t* Co, const int8_t* Ci,
                                const float* Si, int lane) {
     constexpr int DV = 32 * C;
+    constexpr int P = C / 2;
     constexpr int QMAX = BITS == 8 ? 127 : 7;
     const int G = a.d_k / GROUP;
     const int64_t tile_elems = static_cast<int64_t>(a.d_k) * DV;
     for (int g = 0; g < G; ++g) {
         uint8_t* gcodes = tcodes + static_cast<int64_t>(g) * GROUP * DV * BITS / 8;
         float* gscales = a.scales + (static_cast<int64_t>(tile) * G + g) * DV;
-        const int64_t base = tile * tile_elems + static_cast<int64_t>(g) * GROUP * DV + lane * C;
-        if (op == kOpFillZero || op == kOpImportFp32 || op == kOpImportCodes) {
-            float x[GROUP][C];
+        for (int pc = 0; pc < P; ++pc) {
+            const int j = lane * C + 2 * pc;
+            const int64_t base = tile * tile_elems + static_cast<int64_t>(g) * GROUP * DV + j;
+            float2 x[GROUP];
             if (op == kOpImportFp32) {
+                float A0 = 0.0f, A1 = 0.0f;
 #pragma unroll
-                for (int r = 0; r < GROUP; ++r)
-#pragma unroll
-                    for (int c = 0; c < C; ++c) x[r][c] = S[base + r * DV + c];
-                quantize_group_rtn<C, GROUP, BITS>(x, gcodes, gscales, lane);
-            } else {
+                for (int r = 0; r < GROUP; ++r) {
+                    x[r] = make_float2(S[base + r * DV], S[base + r * DV + 1]);
+                    A0 = fmaxf(A0, fabsf(x[r].x));
+                    A1 = fmaxf(A1, fabsf(x[r].y));
+                }
+                constexpr float QF = static_cast<float>(QMAX);
+                const float2 snew = make_float2(A0 < kTiny ? 0.0f : __fdiv_rn(A0, QF),
+                                                A1 < kTiny ? 0.0f : __fdiv_rn(A1, QF));
+                const float2 inv = make_float2(A0 < kTiny ? 0.0f : __fdiv_rn(QF, A0),
+                                               A1 < kTiny ? 0.0f : __fdiv_rn(QF, A1));
+                gscales[j] = snew.x;
+                gscales[j + 1] = snew.y;
+                encode_pair_rtn<GROUP, BITS>(x, inv, gcodes, pc, lane);
+            } else if (op == kOpFillZero || op == kOpImportCodes) {
                 // zero state, or given codes: the codes are written as they are
                 // (clamped), the scales copied.
 #pragma unroll
-                for (int r = 0; r < GROUP; ++r)
+                for (int r = 0; r < GROUP; ++r) {
+                    float cv[2] = {0.0f, 0.0f};
+                    if (op == kOpImportCodes) {
 #pragma unroll
-                    for (int c = 0; c < C; ++c) {
-                        float cv = 0.0f;
-                        if (op == kOpImportCodes) {
+                        for (int c = 0; c < 2; ++c) {
                             int ci = Ci[base + r * DV + c];
                             if (ci > QMAX || ci < -QMAX) {
                                 atomicOr(a.err, kErrRange);
                                 ci = ci > QMAX ? QMAX : -QMAX;
                             }
-                            cv = static_cast<float>(ci);
+                            cv[c] = static_cast<float>(ci);
                         }
-                        x[r][c] = cv;
                     }
-                constexpr int EPW = 32 / BITS;
-                constexpr int UNITS = GROUP * C * BITS / 8 / 16;
-#pragma unroll
-                for (int un = 0; un < UNITS; ++un) {
-                    uint32_t ow[4];
-#pragma unroll
-                    for (int wi = 0; wi < 4; ++wi) {
-                        float t[EPW];
-#pragma unroll
-                        for (int e = 0; e < EPW; ++e) {
-                            const int el = (un * 4 + wi) * EPW + e;
-                            t[e] = round_code<kRTN, BITS>(x[el / C][el % C], 0.f, 0.f, 0.f, 0ull,
-                                                          0u, 0u);
-                        }
-                        ow[wi] = encode_word<BITS>(t);
-                    }
-                    *reinterpret_cast<uint4*>(gcodes + unit_offset(un, lane)) =
-                        make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    x[r] = make_float2(cv[0], cv[1]);
                 }
+                encode_pair_rtn<GROUP, BITS>(x, f2(1.0f), gcodes, pc, lane);
+                const int64_t si = (static_cast<int64_t>(tile) * G + g) * DV + j;
+                gscales[j] = op == kOpImportCodes ? Si[si] : 0.0f;
+                gscales[j + 1] = op == kOpImportCodes ? Si[si + 1] : 0.0f;
+            } else {
+                decode_pair<GROUP, BITS>(gcodes, pc, lane, x);
 #pragma unroll
-                for (int c = 0; c < C; ++c)
-                    gscales[lane * C + c] = op == kOpImportCodes ? Si[(static_cast<int64_t>(tile) * G + g) * DV + lane * C + c] : 0.0f;
+                for (int r = 0; r < GROUP; ++r) {
+                    if (op == kOpExportFp32) {
+                        So[base + r * DV] = __fmul_rn(x[r].x, gscales[j]);
+                        So[base + r * DV + 1] = __fmul_rn(x[r].y, gscales[j + 1]);
+                    } else {
+                        Co[base + r * DV] = static_cast<int8_t>(static_cast<int>(x[r].x));
+                        Co[base + r * DV + 1] = static_cast<int8_t>(static_cast<int>(x[r].y));
+                    }
+                }
             }
-        } else {
-            float code[GROUP][C];
-            decode_group<C, GROUP, BITS>(gcodes, lane, code);
-#pragma unroll
-            for (int r = 0; r < GROUP; ++r)
-#pragma unroll
-                for (int c = 0; c < C; ++c) {
-                    if (op == kOpExportFp32)
-                        So[base + r * DV + c] = __fmul_rn(code[r][c], gscales[lane * C + c]);
-                    else
-                        Co[base + r * DV + c] = static_cast<int8_t>(static_cast<int>(code[r][c]));
-                }
         }
     }
 }

@@ -80,15 +80,23 @@ std::mutex g_inject_mu;
 bool g_inject = false;
 uint64_t g_inject_timeout_ns = 0;
 
-// Launch shape of the step kernel: warps per CTA (0 = derived from shared
-// memory). LRS_STEP_WARPS overrides it for launch-shape sweeps.
+// Launch shape of the step kernel: warps per CTA and ring slots per warp
+// (0 = the defaults below). LRS_STEP_WARPS / LRS_STEP_SLOTS override them
+// for launch-shape sweeps.
+int env_int(const char* name) {
+    const char* s = getenv(name);
+    return s ? atoi(s) : 0;
+}
 int step_warps_override() {
-    static int v = [] {
-        const char* s = getenv("LRS_STEP_WARPS");
-        return s ? atoi(s) : 0;
-    }();
+    static int v = env_int("LRS_STEP_WARPS");
     return v;
 }
+int step_slots_override() {
+    static int v = env_int("LRS_STEP_SLOTS");
+    return v;
+}
+constexpr int kDefaultWarps = 12;
+constexpr int kDefaultSlots = 2;
 
 struct StatePriv {
     int device = -1;
@@ -191,11 +199,11 @@ const void* find_step_kernel(int C, int group, int update_kind, int gate_kind, i
     }
 }
 
-int step_warp_smem(int C, int group, int gate_kind, int G) {
+int step_warp_smem(int C, int group, int gate_kind, int slots) {
 #define LRS_SLOT(CC, GG)                                                                 \
     if (C == CC && group == GG)                                                          \
-        return gate_kind == kGatePerKey ? Slot<CC, GG, kGatePerKey>::warp_bytes(G)       \
-                                        : Slot<CC, GG, kGate>::warp_bytes(G);
+        return gate_kind == kGatePerKey ? Slot<CC, GG, kGatePerKey>::warp_bytes(slots)   \
+                                        : Slot<CC, GG, kGate>::warp_bytes(slots);
     LRS_SLOT(4, 16)
     LRS_SLOT(4, 32)
     LRS_SLOT(2, 16)
@@ -336,32 +344,57 @@ lrs_status lrs_decode_step(const lrs_state* st, void* state_codes, float* scales
     const int ntiles = sh.batch * sh.heads;
     if (ntiles == 0) return ok();
 
-    const int warp_smem = lrs::step_warp_smem(C, sh.group, sh.gate_kind, G);
+    // ring slots per warp: the delta rule keeps a whole tile resident; the
+    // gated forms stream a few groups ahead (at most G, so that the single v
+    // buffer is never overwritten before it is read)
+    int slots = G;
+    if (sh.update_kind != LRS_UPDATE_DELTA) {
+        slots = step_slots_override() > 0 ? step_slots_override() : kDefaultSlots;
+        slots = std::min(slots, G);
+    }
+    slots = std::max(1, std::min(slots, lrs::kMaxSlots));
+    const int warp_smem = lrs::step_warp_smem(C, sh.group, sh.gate_kind, slots);
     constexpr int kSmemLimit = 227 * 1024;
     int warps = step_warps_override();
-    if (warps <= 0) warps = 8;
+    if (warps <= 0) warps = kDefaultWarps;
     warps = std::min(warps, std::max(1, kSmemLimit / warp_smem));
-    warps = std::min(warps, 8);  // the kernel is compiled for at most 256 threads
+    warps = std::min(warps, lrs::step_max_warps(sh.group, mode));
     const int smem = warps * warp_smem;
 
-    // per kernel and device: raise the dynamic shared memory limit once, and
-    // record how many CTAs fit on an SM
+    // Per kernel and device, raise the dynamic shared memory limit once to the
+    // largest launch can ask for (the attribute belongs to the function, so it
+    // is never lowered again); per launch shape, record how many CTAs fit.
     static std::mutex mu;
-    struct Cached { const void* fn; int dev; int smem; int per_sm; };
-    static std::vector<Cached> cache;
+    struct Prepared { const void* fn; int dev; };
+    struct Occupancy { const void* fn; int dev; int smem; int threads; int per_sm; };
+    static std::vector<Prepared> prepared;
+    static std::vector<Occupancy> occupancy;
     int per_sm = 0;
     {
         std::lock_guard<std::mutex> lk(mu);
-        const StatePriv* pv = static_cast<const StatePriv*>(st->priv);
-        for (const Cached& c : cache)
-            if (c.fn == fn && c.dev == pv->device && c.smem == smem) per_sm = c.per_sm;
+        const int dev = static_cast<const StatePriv*>(st->priv)->device;
+        bool ready = false;
+        for (const Prepared& c : prepared) ready = ready || (c.fn == fn && c.dev == dev);
+        if (!ready) {
+            cudaError_t e =
+                cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                return cuda_fail(e, "cudaFuncSetAttribute");
+            }
+            prepared.push_back({fn, dev});
+        }
+        for (const Occupancy& c : occupancy)
+            if (c.fn == fn && c.dev == dev && c.smem == smem && c.threads == warps * 32)
+                per_sm = c.per_sm;
         if (per_sm == 0) {
-            cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, warps * 32, smem);
-            if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+            cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, warps * 32, smem);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+            }
             if (per_sm < 1) return fail(LRS_ERR_UNSUPPORTED, "step kernel does not fit on an SM");
-            cache.push_back({fn, pv->device, smem, per_sm});
+            occupancy.push_back({fn, dev, smem, warps * 32, per_sm});
         }
     }
     int grid = ctx->sms * per_sm;
@@ -388,6 +421,7 @@ lrs_status lrs_decode_step(const lrs_state* st, void* state_codes, float* scales
     p.G = G;
     p.ntiles = ntiles;
     p.warp_smem = warp_smem;
+    p.slots = slots;
     p.inject = 0;
     {
         std::lock_guard<std::mutex> lk(g_inject_mu);
@@ -400,7 +434,10 @@ lrs_status lrs_decode_step(const lrs_state* st, void* state_codes, float* scales
     void* args[] = {&p};
     cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(warps * 32), args, smem,
                                      static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "launch of the step kernel");
+    if (e != cudaSuccess) {
+        cudaGetLastError();  // a failed launch must not surface again in a later call
+        return cuda_fail(e, "launch of the step kernel");
+    }
     return ok();
 }
 

@@ -4,12 +4,15 @@
 // [t*C, t*C + C) (C = d_v / 32) over every key row, so every reduction the
 // step needs over the key axis -- u = k^T deq (delta rule), o = x^T q and the
 // per-(group, column) absmax -- runs inside one thread, in key order, with no
-// shuffles. The tile streams through shared memory one scale group at a time:
-// each group has its own slot and mbarrier; its codes, scales and the group's
-// q, k (and per-key gate) rows arrive by 1-D bulk copies issued by lane 0, and
-// as soon as a group is consumed its slot is refilled with the same group of
-// the warp's next tile. New codes and scales are written straight back with
-// 128-bit streaming stores, in place.
+// shuffles. A lane works through its columns one adjacent pair at a time, so
+// only one pair's updated values of one scale group are live in registers.
+//
+// The tile streams through shared memory one scale group at a time, through a
+// ring of slots per warp, each with its own mbarrier: lane 0 fills a slot with
+// 1-D bulk copies (the group's codes and scales, its q, k and per-key gate
+// rows, and v with the tile's first group) and refills it with the warp's
+// next item as soon as it is consumed. New codes and scales go back in place
+// with 128-bit streaming stores.
 //
 // Sources: "Quantizing Recurrent Language Models Is Easier Than You Think"
 // (abstract: value-axis scale grouping, mixed precision by decay, stochastic
@@ -24,7 +27,11 @@ namespace lrs {
 constexpr int kGate = 0, kGatePerKey = 1;        // matches lrs_gate_kind
 constexpr int kGated = 0, kDelta = 1;            // matches lrs_update_kind
 constexpr int kRTN = 0, kSR = 1, kBDR = 2;       // matches lrs_round_mode
-constexpr int kMaxGroups = 16;
+constexpr int kMaxSlots = 16;
+// Launch bound of a step variant in warps: 12 (at most 168 registers a thread)
+// where the live state fits, 8 (255 registers) for the wider groups and for
+// the rounding modes that carry more temporaries.
+constexpr int step_max_warps(int group, int mode) { return (mode != 0 || group > 32) ? 8 : 12; }
 constexpr float kTiny = 0x1p-100f;               // absmax below this: stored as zero
 
 struct StepParams {
@@ -44,14 +51,15 @@ struct StepParams {
     unsigned* err;
     uint64_t timeout_ns;
     int32_t H, d_k, G, ntiles;
+    int32_t slots;       // ring slots per warp, 1..min(G, 16); the delta rule needs G
     int32_t warp_smem;   // bytes of shared memory per warp
     int32_t inject;      // fault injection: issue no copies
 };
 
 // Shared-memory layout of one warp:
-//   [0, 128)            mbarriers, one per group slot
-//   [128, 128 + 4*d_v)  v of the current tile (arrives with slot 0)
-//   then G slots of SlotBytes each:
+//   [0, 128)            mbarriers, one per slot
+//   [128, 128 + 4*d_v)  v of the tile whose first group was issued last
+//   then `slots` slots of kBytes each:
 //     codes (GROUP*d_v bytes: room for int8) | scales (d_v fp32) |
 //     q, k, [gate] (GROUP fp32 each)
 template <int C, int GROUP, int GATE>
@@ -65,22 +73,69 @@ struct Slot {
     static constexpr int kBytes = kG + (GATE == kGatePerKey ? GROUP * 4 : 0);
     static constexpr int kHeader = 128 + DV * 4;
     static_assert(kBytes % 16 == 0, "slot alignment");
-    static int warp_bytes(int G) { return (kHeader + G * kBytes + 127) / 128 * 128; }
+    static int warp_bytes(int slots) { return (kHeader + slots * kBytes + 127) / 128 * 128; }
 };
 
+// ------------------------------------------------------- packed fp32 math ---
+// The two columns of a pair go through the sm_100 two-wide fp32 instructions;
+// each half is an IEEE binary32 operation rounded to nearest even. They are
+// written with an explicit .rn so that no multiply and add is ever fused into
+// one rounding behind our back (results must follow the stated roundings).
+
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+__device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
+
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return r;
+}
+
+// max(a, |b|, |c|): one three-input maximum.
+__device__ __forceinline__ float max_abs3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(fabsf(b)), "f"(fabsf(c)));
+    return r;
+}
+
+// The stored bytes of one 32-bit word as floats 2^23 + byte (offset binary),
+// in element order (int4: byte n holds elements n and n+4).
 template <int BITS>
-__device__ __forceinline__ void decode_word(uint32_t w, float (&f)[32 / BITS]) {
+__device__ __forceinline__ void decode_word_biased(uint32_t w, float (&f)[32 / BITS]) {
     if constexpr (BITS == 8) {
 #pragma unroll
-        for (int n = 0; n < 4; ++n)
-            f[n] = __fsub_rn(byte_to_biased_float(w, n), kTwo23 + 128.0f);
+        for (int n = 0; n < 4; ++n) f[n] = byte_to_biased_float(w, n);
     } else {
         const uint32_t lo = w & 0x0F0F0F0Fu;
         const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
         for (int n = 0; n < 4; ++n) {
-            f[n] = __fsub_rn(byte_to_biased_float(lo, n), kTwo23 + 8.0f);
-            f[n + 4] = __fsub_rn(byte_to_biased_float(hi, n), kTwo23 + 8.0f);
+            f[n] = byte_to_biased_float(lo, n);
+            f[n + 4] = byte_to_biased_float(hi, n);
         }
     }
 }
@@ -96,36 +151,49 @@ __device__ __forceinline__ uint32_t encode_word(const float (&t)[32 / BITS]) {
     }
 }
 
-// Rounded code of y, returned as the float 1.5*2^23 + bias + code whose low
-// byte is the stored offset-binary byte.
+template <int BITS> struct Q;
+template <> struct Q<8> { static constexpr float kMax = 127.0f, kBias = 128.0f; };
+template <> struct Q<4> { static constexpr float kMax = 7.0f, kBias = 8.0f; };
+
+// Codes of two elements (value columns j, j+1 of key row i), returned as the
+// floats 1.5*2^23 + bias + code whose low byte is the stored byte. The value
+// rounded is the exact product x*inv: one fused multiply-add rounds it
+// straight to an integer.
 template <int MODE, int BITS>
-__device__ __forceinline__ float round_code(float y, float x, float deq, float s_new,
-                                            uint64_t hkey, uint32_t i, uint32_t j) {
-    constexpr float QMAX = BITS == 8 ? 127.0f : 7.0f;
-    constexpr float BIAS = BITS == 8 ? 128.0f : 8.0f;
+__device__ __forceinline__ float2 round_pair(float2 x, float2 inv, float2 deq, float2 s_new,
+                                             uint64_t hkey, uint32_t i, uint32_t j) {
+    constexpr float QMAX = Q<BITS>::kMax, BIAS = Q<BITS>::kBias;
     if constexpr (MODE == kRTN) {
-        // |y| <= qmax (1 + 2^-24) because inv = RN(qmax/A) and |x| <= A, so
-        // the nearest integer never leaves [-qmax, qmax]: no clamp needed.
-        return __fadd_rn(y, kRound + BIAS);
+        // |x*inv| <= qmax (1 + 2^-24) since inv = RN(qmax/A) and |x| <= A:
+        // the nearest integer never leaves [-qmax, qmax], no clamp needed.
+        return fma2(x, inv, f2(kRound + BIAS));
     } else {
-        const float rn = __fsub_rn(__fadd_rn(y, kRound), kRound);  // rint(y), exact
-        float c;
+        const float2 n = add2(fma2(x, inv, f2(kRound)), f2(-kRound));  // nearest integer
+        const float2 d = fma2(x, inv, neg2(n));                          // sign of x*inv - n
+        float2 c;
         if constexpr (MODE == kSR) {
-            const float f = rn > y ? __fsub_rn(rn, 1.0f) : rn;    // floor(y)
-            const float fr = __fsub_rn(y, f);
-            const float u = element_uniform(hkey, i, j);
-            c = u < fr ? __fadd_rn(f, 1.0f) : f;
+            const float2 f = make_float2(d.x < 0.0f ? n.x - 1.0f : n.x,
+                                         d.y < 0.0f ? n.y - 1.0f : n.y);  // floor
+            const float2 fr = fma2(x, inv, neg2(f));                      // fraction, rounded once
+            const float u0 = element_uniform(hkey, i, j);
+            const float u1 = element_uniform(hkey, i, j + 1);
+            c.x = u0 < fr.x ? f.x + 1.0f : f.x;
+            c.y = u1 < fr.y ? f.y + 1.0f : f.y;
         } else {
-            const float delta = __fsub_rn(x, deq);
-            const float m = __fsub_rn(__fmul_rn(rn, s_new), deq);
-            c = rn;
-            if (delta > 0.0f && m < 0.0f)
-                c = rn < y ? __fadd_rn(rn, 1.0f) : rn;            // ceil(y)
-            else if (delta < 0.0f && m > 0.0f)
-                c = rn > y ? __fsub_rn(rn, 1.0f) : rn;            // floor(y)
+            // the update and the move; the move's product and difference are
+            // two separate roundings (scalar _rn operations are never fused)
+            const float2 delta = add2(x, neg2(deq));
+            const float2 m = make_float2(__fsub_rn(__fmul_rn(n.x, s_new.x), deq.x),
+                                         __fsub_rn(__fmul_rn(n.y, s_new.y), deq.y));
+            c = n;
+            if (delta.x > 0.0f && m.x < 0.0f) c.x = d.x > 0.0f ? n.x + 1.0f : n.x;       // ceil
+            else if (delta.x < 0.0f && m.x > 0.0f) c.x = d.x < 0.0f ? n.x - 1.0f : n.x;  // floor
+            if (delta.y > 0.0f && m.y < 0.0f) c.y = d.y > 0.0f ? n.y + 1.0f : n.y;
+            else if (delta.y < 0.0f && m.y > 0.0f) c.y = d.y < 0.0f ? n.y - 1.0f : n.y;
         }
-        c = fminf(fmaxf(c, -QMAX), QMAX);
-        return __fadd_rn(c, kRound + BIAS);
+        c.x = fminf(fmaxf(c.x, -QMAX), QMAX);
+        c.y = fminf(fmaxf(c.y, -QMAX), QMAX);
+        return add2(c, f2(kRound + BIAS));
     }
 }
 
@@ -135,141 +203,147 @@ __device__ __forceinline__ void st_cs_u4(void* p, uint32_t a, uint32_t b, uint32
                  : "memory");
 }
 
-template <int C>
-__device__ __forceinline__ void st_cs_f(float* p, const float (&s)[C]) {
-    if constexpr (C == 4) {
-        asm volatile("st.global.cs.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(s[0]), "f"(s[1]),
-                     "f"(s[2]), "f"(s[3])
-                     : "memory");
-    } else {
-        asm volatile("st.global.cs.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(s[0]), "f"(s[1])
-                     : "memory");
-    }
+__device__ __forceinline__ void st_cs_f2(float* p, float2 s) {
+    asm volatile("st.global.cs.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(s.x), "f"(s.y) : "memory");
 }
 
-template <int C>
-__device__ __forceinline__ void ld_smem_f(const float* p, float (&s)[C]) {
-    if constexpr (C == 4) {
-        const float4 t = *reinterpret_cast<const float4*>(p);
-        s[0] = t.x; s[1] = t.y; s[2] = t.z; s[3] = t.w;
-    } else {
-        const float2 t = *reinterpret_cast<const float2*>(p);
-        s[0] = t.x; s[1] = t.y;
-    }
-}
-
-// Delta rule, first pass over the tile: u_j += k_i * deq_ij for the rows of
-// one group, in key order.
-template <int C, int GROUP, int BITS>
-__device__ __forceinline__ void group_ktS(const uint8_t* __restrict__ cs,
-                                          const float* __restrict__ ss,
-                                          const float* __restrict__ ks, int lane, float (&u)[C]) {
-    constexpr int EPW = 32 / BITS;
-    constexpr int UNITS = GROUP * C * BITS / 8 / 16;
-    float sc[C];
-    ld_smem_f<C>(ss + lane * C, sc);
+// N consecutive floats of shared memory (N a multiple of 4) into registers.
+template <int N>
+__device__ __forceinline__ void ld_smem_rows(const float* p, float (&r)[N]) {
 #pragma unroll
-    for (int un = 0; un < UNITS; ++un) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(cs + (un * 32 + lane) * 16);
+    for (int i = 0; i < N / 4; ++i) {
+        const float4 t = reinterpret_cast<const float4*>(p)[i];
+        r[4 * i] = t.x; r[4 * i + 1] = t.y; r[4 * i + 2] = t.z; r[4 * i + 3] = t.w;
+    }
+}
+
+// Geometry of one lane's codes for one column pair of one scale group: a run
+// of 16-byte units, each holding EPU consecutive elements of the pair's
+// row-major (row, column) stream, i.e. RPU key rows.
+template <int GROUP, int BITS>
+struct PairGeo {
+    static constexpr int EPW = 32 / BITS;       // elements per 32-bit word
+    static constexpr int EPU = 4 * EPW;         // elements per 16-byte unit
+    static constexpr int RPU = EPU / 2;         // key rows per unit
+    static constexpr int UNITS = GROUP / RPU;   // units per pair per group
+    static_assert(RPU % 4 == 0 && GROUP % RPU == 0, "unit geometry");
+};
+
+__device__ __forceinline__ uint4 lds_unit(const uint8_t* cs, int unit, int lane) {
+    return *reinterpret_cast<const uint4*>(cs + (unit * 32 + lane) * 16);
+}
+
+// Delta rule, first pass: u += k_i * deq_i for one column pair over the rows
+// of one group, in key order.
+template <int GROUP, int BITS>
+__device__ __forceinline__ void pair_ktS(const uint8_t* __restrict__ cs, int ubase, float2 sc,
+                                         const float* __restrict__ ks, int lane, float2& u) {
+    using G = PairGeo<GROUP, BITS>;
+    constexpr float BIAS = Q<BITS>::kBias;
+#pragma unroll
+    for (int un = 0; un < G::UNITS; ++un) {
+        const uint4 raw = lds_unit(cs, ubase + un, lane);
         const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+        float kk[G::RPU];
+        ld_smem_rows<G::RPU>(ks + un * G::RPU, kk);
 #pragma unroll
         for (int wi = 0; wi < 4; ++wi) {
-            float f[EPW];
-            decode_word<BITS>(wd[wi], f);
+            float f[G::EPW];
+            decode_word_biased<BITS>(wd[wi], f);
 #pragma unroll
-            for (int e = 0; e < EPW; ++e) {
-                const int el = (un * 4 + wi) * EPW + e;
-                const int r = el / C, c = el % C;
-                const float deq = __fmul_rn(f[e], sc[c]);
-                u[c] = __fmaf_rn(ks[r], deq, u[c]);
+            for (int e = 0; e < G::EPW; e += 2) {
+                const int rl = (wi * G::EPW + e) / 2;
+                const float2 code = add2(make_float2(f[e], f[e + 1]), f2(-(kTwo23 + BIAS)));
+                u = fma2(f2(kk[rl]), mul2(code, sc), u);
             }
         }
     }
 }
 
-// One scale group of one tile: dequantize, update, accumulate the output,
-// new scales, requantize and store.
-template <int C, int GROUP, int GATE, int MODE, int BITS>
-__device__ __forceinline__ void group_step(const uint8_t* __restrict__ cs,
-                                           const float* __restrict__ ss,
-                                           const float* __restrict__ qs,
-                                           const float* __restrict__ ks,
-                                           const float* __restrict__ gs, float gscalar,
-                                           const float (&w)[C], float (&o)[C],
-                                           uint8_t* __restrict__ gcodes,
-                                           float* __restrict__ gscales, uint64_t hkey, int row0,
-                                           int lane) {
-    constexpr int EPW = 32 / BITS;
-    constexpr int UNITS = GROUP * C * BITS / 8 / 16;
-    constexpr float QMAX = BITS == 8 ? 127.0f : 7.0f;
-
-    float sc[C];
-    ld_smem_f<C>(ss + lane * C, sc);
-    float x[GROUP][C];
-    float amax[C];
-#pragma unroll
-    for (int c = 0; c < C; ++c) amax[c] = 0.0f;
+// One column pair of one scale group: dequantize, update, accumulate the
+// output, new scales, requantize and store.
+template <int GROUP, int GATE, int MODE, int BITS>
+__device__ __forceinline__ void pair_step(const uint8_t* __restrict__ cs, int ubase, float2 sc,
+                                          const float* __restrict__ qs,
+                                          const float* __restrict__ ks,
+                                          const float* __restrict__ gs, float gscalar, float2 w,
+                                          float2& o, uint8_t* __restrict__ gcodes,
+                                          float* __restrict__ gscale, uint64_t hkey, int row0,
+                                          uint32_t j0, int lane) {
+    using G = PairGeo<GROUP, BITS>;
+    constexpr float QMAX = Q<BITS>::kMax, BIAS = Q<BITS>::kBias;
+    float2 x[GROUP];
 
 #pragma unroll
-    for (int un = 0; un < UNITS; ++un) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(cs + (un * 32 + lane) * 16);
+    for (int un = 0; un < G::UNITS; ++un) {
+        const uint4 raw = lds_unit(cs, ubase + un, lane);
         const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+        float kk[G::RPU], qq[G::RPU], gg[G::RPU];
+        ld_smem_rows<G::RPU>(ks + un * G::RPU, kk);
+        ld_smem_rows<G::RPU>(qs + un * G::RPU, qq);
+        if constexpr (GATE == kGatePerKey) ld_smem_rows<G::RPU>(gs + un * G::RPU, gg);
 #pragma unroll
         for (int wi = 0; wi < 4; ++wi) {
-            float f[EPW];
-            decode_word<BITS>(wd[wi], f);
+            float f[G::EPW];
+            decode_word_biased<BITS>(wd[wi], f);
 #pragma unroll
-            for (int e = 0; e < EPW; ++e) {
-                const int el = (un * 4 + wi) * EPW + e;
-                const int r = el / C, c = el % C;
-                const float deq = __fmul_rn(f[e], sc[c]);
-                const float gi = GATE == kGatePerKey ? gs[r] : gscalar;
-                const float kw = __fmul_rn(ks[r], w[c]);
-                const float xv = __fmaf_rn(gi, deq, kw);
-                o[c] = __fmaf_rn(qs[r], xv, o[c]);
-                amax[c] = fmaxf(amax[c], fabsf(xv));
-                x[r][c] = xv;
+            for (int e = 0; e < G::EPW; e += 2) {
+                const int rl = (wi * G::EPW + e) / 2;
+                const float gi = GATE == kGatePerKey ? gg[rl] : gscalar;
+                const float2 code = add2(make_float2(f[e], f[e + 1]), f2(-(kTwo23 + BIAS)));
+                const float2 deq = mul2(code, sc);
+                const float2 kw = mul2(f2(kk[rl]), w);
+                const float2 xv = fma2(f2(gi), deq, kw);
+                o = fma2(f2(qq[rl]), xv, o);
+                x[un * G::RPU + rl] = xv;
             }
         }
     }
 
-    float snew[C], inv[C];
+    // absmax per column over the group's rows (order-free)
+    float a0 = 0.0f, a1 = 0.0f, b0 = 0.0f, b1 = 0.0f;
 #pragma unroll
-    for (int c = 0; c < C; ++c) {
-        const float A = amax[c];
-        const bool zero = A < kTiny;
-        snew[c] = zero ? 0.0f : __fdiv_rn(A, QMAX);
-        inv[c] = zero ? 0.0f : __fdiv_rn(QMAX, A);
+    for (int r = 0; r < GROUP; r += 4) {
+        a0 = max_abs3(a0, x[r].x, x[r + 1].x);
+        a1 = max_abs3(a1, x[r + 2].x, x[r + 3].x);
+        b0 = max_abs3(b0, x[r].y, x[r + 1].y);
+        b1 = max_abs3(b1, x[r + 2].y, x[r + 3].y);
     }
-    st_cs_f<C>(gscales + lane * C, snew);
+    const float A0 = fmaxf(a0, a1), A1 = fmaxf(b0, b1);
+    float2 snew, inv;
+    snew.x = A0 < kTiny ? 0.0f : __fdiv_rn(A0, QMAX);
+    inv.x = A0 < kTiny ? 0.0f : __fdiv_rn(QMAX, A0);
+    snew.y = A1 < kTiny ? 0.0f : __fdiv_rn(A1, QMAX);
+    inv.y = A1 < kTiny ? 0.0f : __fdiv_rn(QMAX, A1);
+    st_cs_f2(gscale, snew);
 
 #pragma unroll
-    for (int un = 0; un < UNITS; ++un) {
+    for (int un = 0; un < G::UNITS; ++un) {
         uint32_t ow[4];
         uint32_t wd[4] = {0u, 0u, 0u, 0u};
         if constexpr (MODE == kBDR) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(cs + (un * 32 + lane) * 16);
+            const uint4 raw = lds_unit(cs, ubase + un, lane);
             wd[0] = raw.x; wd[1] = raw.y; wd[2] = raw.z; wd[3] = raw.w;
         }
 #pragma unroll
         for (int wi = 0; wi < 4; ++wi) {
-            float f[EPW];
-            if constexpr (MODE == kBDR) decode_word<BITS>(wd[wi], f);
-            float t[EPW];
+            float f[G::EPW];
+            if constexpr (MODE == kBDR) decode_word_biased<BITS>(wd[wi], f);
+            float t[G::EPW];
 #pragma unroll
-            for (int e = 0; e < EPW; ++e) {
-                const int el = (un * 4 + wi) * EPW + e;
-                const int r = el / C, c = el % C;
-                const float y = __fmul_rn(x[r][c], inv[c]);
-                float deq = 0.0f;
-                if constexpr (MODE == kBDR) deq = __fmul_rn(f[e], sc[c]);
-                t[e] = round_code<MODE, BITS>(y, x[r][c], deq, snew[c], hkey,
-                                              static_cast<uint32_t>(row0 + r),
-                                              static_cast<uint32_t>(lane * C + c));
+            for (int e = 0; e < G::EPW; e += 2) {
+                const int r = un * G::RPU + (wi * G::EPW + e) / 2;
+                float2 deq = f2(0.0f);
+                if constexpr (MODE == kBDR)
+                    deq = mul2(add2(make_float2(f[e], f[e + 1]), f2(-(kTwo23 + BIAS))), sc);
+                const float2 tv = round_pair<MODE, BITS>(x[r], inv, deq, snew, hkey,
+                                                         static_cast<uint32_t>(row0 + r), j0);
+                t[e] = tv.x;
+                t[e + 1] = tv.y;
             }
             ow[wi] = encode_word<BITS>(t);
         }
-        st_cs_u4(gcodes + (un * 32 + lane) * 16, ow[0], ow[1], ow[2], ow[3]);
+        st_cs_u4(gcodes + ((ubase + un) * 32 + lane) * 16, ow[0], ow[1], ow[2], ow[3]);
     }
 }
 
@@ -293,192 +367,231 @@ __device__ __forceinline__ TileInfo tile_info(const StepParams& p, int tile, int
     return ti;
 }
 
+// Fill `slot` with group g of tile `tile` (lane 0 only). A tile whose layout
+// does not fit gets a bare arrival, so the slot's phase still completes.
 template <int C, int GROUP, int GATE>
-__device__ __forceinline__ void issue_slot(const StepParams& p, uint8_t* wsm, int tile, int g,
-                                           const TileInfo& ti, uint64_t pol_state,
-                                           uint64_t pol_in) {
+__device__ __forceinline__ void issue_item(const StepParams& p, uint8_t* wsm, int slot, int tile,
+                                           int g, uint64_t pol_state, uint64_t pol_in) {
     using S = Slot<C, GROUP, GATE>;
     constexpr int DV = 32 * C;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(wsm);
-    uint8_t* slot = wsm + S::kHeader + g * S::kBytes;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(wsm) + slot;
+    const TileInfo ti = tile_info(p, tile, DV);
+    if (ti.prec == 0) {
+        mbar_arrive(bar);
+        return;
+    }
+    uint8_t* sm = wsm + S::kHeader + slot * S::kBytes;
     const uint32_t cbytes = GROUP * DV * ti.prec / 8;
     uint32_t total = cbytes + DV * 4 + 2 * GROUP * 4;
     if (GATE == kGatePerKey) total += GROUP * 4;
     if (g == 0) total += DV * 4;
-    mbar_arrive_expect_tx(&bars[g], total);
-    bulk_g2s(slot, p.codes + ti.code_off + static_cast<int64_t>(g) * cbytes, cbytes, &bars[g],
+    mbar_arrive_expect_tx(bar, total);
+    bulk_g2s(sm, p.codes + ti.code_off + static_cast<int64_t>(g) * cbytes, cbytes, bar, pol_state);
+    bulk_g2s(sm + S::kScales, p.scales + (static_cast<int64_t>(tile) * p.G + g) * DV, DV * 4, bar,
              pol_state);
-    bulk_g2s(slot + S::kScales, p.scales + (static_cast<int64_t>(tile) * p.G + g) * DV, DV * 4,
-             &bars[g], pol_state);
     const int64_t rowbase = static_cast<int64_t>(tile) * p.d_k + g * GROUP;
-    bulk_g2s(slot + S::kQ, p.q + rowbase, GROUP * 4, &bars[g], pol_in);
-    bulk_g2s(slot + S::kK, p.k + rowbase, GROUP * 4, &bars[g], pol_in);
-    if (GATE == kGatePerKey) bulk_g2s(slot + S::kG, p.gates + rowbase, GROUP * 4, &bars[g], pol_in);
-    if (g == 0)
-        bulk_g2s(wsm + 128, p.v + static_cast<int64_t>(tile) * DV, DV * 4, &bars[g], pol_in);
+    bulk_g2s(sm + S::kQ, p.q + rowbase, GROUP * 4, bar, pol_in);
+    bulk_g2s(sm + S::kK, p.k + rowbase, GROUP * 4, bar, pol_in);
+    if (GATE == kGatePerKey) bulk_g2s(sm + S::kG, p.gates + rowbase, GROUP * 4, bar, pol_in);
+    if (g == 0) bulk_g2s(wsm + 128, p.v + static_cast<int64_t>(tile) * DV, DV * 4, bar, pol_in);
 }
 
+// Position in a warp's ring: item k lives in slot k % slots and completes
+// phase parity (k / slots) & 1 of that slot's mbarrier.
+struct Ring {
+    int slot = 0;
+    uint32_t par = 0;
+    __device__ __forceinline__ void advance(int slots) {
+        if (++slot == slots) {
+            slot = 0;
+            par ^= 1u;
+        }
+    }
+};
+
+// The warp's items are (tile, group) pairs in order: item k is group k % G of
+// the warp's tile k / G (tiles gw, gw + W, ...).
 template <int C, int GROUP, int UPD, int GATE, int MODE>
-__global__ void __launch_bounds__(256, 1) step_kernel(const StepParams p) {
+__global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
+    step_kernel(const StepParams p) {
     using S = Slot<C, GROUP, GATE>;
     constexpr int DV = 32 * C;
+    constexpr int P = C / 2;
     extern __shared__ __align__(128) uint8_t smem[];
     const int lane = threadIdx.x & 31;
     const int wib = threadIdx.x >> 5;
     const int nw = blockDim.x >> 5;
     const int W = gridDim.x * nw;
-    int tile = blockIdx.x * nw + wib;
+    const int gw = blockIdx.x * nw + wib;
     uint8_t* wsm = smem + wib * p.warp_smem;
     uint64_t* bars = reinterpret_cast<uint64_t*>(wsm);
     const float* v_s = reinterpret_cast<const float*>(wsm + 128);
-    const int G = p.G;
+    const int G = p.G, NS = p.slots;
+    const int ntw = gw < p.ntiles ? (p.ntiles - gw + W - 1) / W : 0;   // this warp's tiles
+    const int64_t K = static_cast<int64_t>(ntw) * G;                    // this warp's items
 
     if (lane == 0) {
-        for (int g = 0; g < G; ++g) mbar_init(&bars[g], 1);
+        for (int s = 0; s < NS; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
     }
     __syncwarp();
 
     const uint64_t pol_state = policy_evict_first();
     const uint64_t pol_in = policy_evict_first();
-    // Every slot of a tile is issued once per tile, so all slots advance their
-    // mbarrier phase together: the k-th tile issued by this warp completes
-    // phase parity k & 1 in each slot.
-    uint32_t issued = 0;    // tiles issued so far by this warp
-    uint32_t cur_par = 0;   // phase parity of the current tile's copies
-    uint32_t inflight = 0;  // slots with copies issued and not yet waited for
-    uint32_t pend_par = 0;  // per slot: parity of the phase it is waiting for
+    Ring ic, is;                 // consumer and issuer positions
+    int64_t kc = 0, ki = 0;      // items consumed, items issued
+    int it_tile = 0, it_g = 0;   // (tile of this warp, group) of item ki
 
-    auto issue_tile_slot = [&](int t, int g, const TileInfo& tinfo, uint32_t par) {
-        if (lane == 0) issue_slot<C, GROUP, GATE>(p, wsm, t, g, tinfo, pol_state, pol_in);
-        inflight |= 1u << g;
-        pend_par = (pend_par & ~(1u << g)) | (par << g);
-    };
-
-    if (tile < p.ntiles) {
-        const TileInfo ti = tile_info(p, tile, DV);
-        if (ti.prec != 0 && !p.inject) {
-            cur_par = issued & 1u;
-            for (int g = 0; g < G; ++g) issue_tile_slot(tile, g, ti, cur_par);
-            ++issued;
+    auto issue_next = [&]() {
+        if (ki < K && !p.inject) {
+            if (lane == 0)
+                issue_item<C, GROUP, GATE>(p, wsm, is.slot, gw + it_tile * W, it_g, pol_state,
+                                           pol_in);
+            ++ki;
+            is.advance(NS);
+            if (++it_g == G) {
+                it_g = 0;
+                ++it_tile;
+            }
         }
-    }
+    };
+    for (int s = 0; s < NS; ++s) issue_next();
 
     float nscal = 0.0f, nbeta = 0.0f;
-    if (tile < p.ntiles) {
-        if (GATE == kGate) nscal = __ldg(p.gates + tile);
-        if (UPD == kDelta) nbeta = __ldg(p.beta + tile);
+    if (ntw > 0) {
+        if (GATE == kGate) nscal = __ldg(p.gates + gw);
+        if (UPD == kDelta) nbeta = __ldg(p.beta + gw);
     }
 
-    for (; tile < p.ntiles; tile += W) {
-        const int next = tile + W;
+    bool ok = true;
+    for (int n = 0; n < ntw && ok; ++n) {
+        const int tile = gw + n * W;
         const TileInfo ti = tile_info(p, tile, DV);
-        const TileInfo tn = next < p.ntiles ? tile_info(p, next, DV) : TileInfo{0, 0};
-        const bool issue_next = tn.prec != 0 && !p.inject;
-        const uint32_t nxt_par = issued & 1u;
         const float gscalar = nscal, beta = nbeta;
-        if (next < p.ntiles) {
-            if (GATE == kGate) nscal = __ldg(p.gates + next);
-            if (UPD == kDelta) nbeta = __ldg(p.beta + next);
-        }
-        if (ti.prec == 0) {
-            // No copies were issued for this tile: record the mismatch, skip
-            // it, and start the next tile's copies in the free slots.
-            if (lane == 0) atomicOr(p.err, kErrLayout);
-            if (issue_next) {
-                for (int g = 0; g < G; ++g) issue_tile_slot(next, g, tn, nxt_par);
-                ++issued;
-                cur_par = nxt_par;
-            }
-            continue;
+        if (n + 1 < ntw) {
+            if (GATE == kGate) nscal = __ldg(p.gates + tile + W);
+            if (UPD == kDelta) nbeta = __ldg(p.beta + tile + W);
         }
         const uint64_t hkey = MODE == kSR ? tile_hash_key(p.seed, p.step,
                                                           static_cast<uint32_t>(tile / p.H),
                                                           static_cast<uint32_t>(tile % p.H))
                                           : 0ull;
-        bool ok = true;
-        float w[C], o[C];
-#pragma unroll
-        for (int c = 0; c < C; ++c) o[c] = 0.0f;
 
-        // ---- wait for the slots needed before the first group
-        const int first_wait = UPD == kDelta ? G : 1;
-        for (int g = 0; g < first_wait && ok; ++g) {
-            ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[g], cur_par, p.timeout_ns));
-            if (ok) inflight &= ~(1u << g);
-        }
-        if (ok) {
-            if (UPD == kDelta) {
-                float u[C];
-#pragma unroll
-                for (int c = 0; c < C; ++c) u[c] = 0.0f;
-                for (int g = 0; g < G; ++g) {
-                    const uint8_t* slot = wsm + S::kHeader + g * S::kBytes;
-                    const float* ss = reinterpret_cast<const float*>(slot + S::kScales);
-                    const float* ks = reinterpret_cast<const float*>(slot + S::kK);
-                    if (ti.prec == 8)
-                        group_ktS<C, GROUP, 8>(slot, ss, ks, lane, u);
-                    else
-                        group_ktS<C, GROUP, 4>(slot, ss, ks, lane, u);
-                }
-#pragma unroll
-                for (int c = 0; c < C; ++c) {
-                    const float t = __fmul_rn(gscalar, u[c]);
-                    const float d = __fsub_rn(v_s[lane * C + c], t);
-                    w[c] = __fmul_rn(beta, d);
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < C; ++c) w[c] = v_s[lane * C + c];
+        // the delta rule needs every group of the tile before its first one
+        {
+            Ring look = ic;
+            const int first = UPD == kDelta ? G : 1;
+            for (int g = 0; g < first && ok; ++g) {
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait_bounded(&bars[look.slot], look.par, p.timeout_ns));
+                look.advance(NS);
             }
+        }
+        if (!ok) break;
 
-            uint8_t* gcodes_tile = p.codes + ti.code_off;
-            const uint32_t cbytes = GROUP * DV * ti.prec / 8;
+        if (ti.prec == 0) {
+            // no copies were made for this tile: record the mismatch and skip it
+            if (lane == 0) atomicOr(p.err, kErrLayout);
             for (int g = 0; g < G; ++g) {
                 if (UPD != kDelta && g > 0) {
                     ok = __all_sync(0xffffffffu,
-                                    mbar_wait_bounded(&bars[g], cur_par, p.timeout_ns));
+                                    mbar_wait_bounded(&bars[ic.slot], ic.par, p.timeout_ns));
                     if (!ok) break;
-                    inflight &= ~(1u << g);
                 }
-                const uint8_t* slot = wsm + S::kHeader + g * S::kBytes;
-                const float* ss = reinterpret_cast<const float*>(slot + S::kScales);
-                const float* qs = reinterpret_cast<const float*>(slot + S::kQ);
-                const float* ks = reinterpret_cast<const float*>(slot + S::kK);
-                const float* gs = reinterpret_cast<const float*>(slot + S::kG);
-                float* gscales = p.scales + (static_cast<int64_t>(tile) * G + g) * DV;
-                uint8_t* gcodes = gcodes_tile + static_cast<int64_t>(g) * cbytes;
-                if (ti.prec == 8)
-                    group_step<C, GROUP, GATE, MODE, 8>(slot, ss, qs, ks, gs, gscalar, w, o,
-                                                        gcodes, gscales, hkey, g * GROUP, lane);
-                else
-                    group_step<C, GROUP, GATE, MODE, 4>(slot, ss, qs, ks, gs, gscalar, w, o,
-                                                        gcodes, gscales, hkey, g * GROUP, lane);
+                ++kc;
+                ic.advance(NS);
                 __syncwarp();
-                if (issue_next) {
-                    if (lane == 0) fence_proxy_async_smem();
-                    issue_tile_slot(next, g, tn, nxt_par);
-                }
+                issue_next();
             }
+            continue;
         }
-        if (!ok) {
-            // Record the timeout, then wait (bounded) for this warp's copies
-            // still in flight before leaving, so none lands after exit.
-            if (lane == 0) atomicOr(p.err, kErrTimeout);
-            for (int g = 0; g < G; ++g)
-                if (inflight & (1u << g))
-                    mbar_wait_bounded(&bars[g], (pend_par >> g) & 1u, p.timeout_ns);
-            return;
-        }
-        if (issue_next) {
-            ++issued;
-            cur_par = nxt_par;
-        }
-        float* op = p.out + static_cast<int64_t>(tile) * DV + lane * C;
-        if constexpr (C == 4) {
-            *reinterpret_cast<float4*>(op) = make_float4(o[0], o[1], o[2], o[3]);
+
+        float2 w[P], o[P];
+#pragma unroll
+        for (int pc = 0; pc < P; ++pc) o[pc] = f2(0.0f);
+        if (UPD == kDelta) {
+            float2 u[P];
+#pragma unroll
+            for (int pc = 0; pc < P; ++pc) u[pc] = f2(0.0f);
+            Ring r = ic;
+            for (int g = 0; g < G; ++g) {
+                const uint8_t* sm = wsm + S::kHeader + r.slot * S::kBytes;
+                const float* ss = reinterpret_cast<const float*>(sm + S::kScales) + lane * C;
+                const float* ks = reinterpret_cast<const float*>(sm + S::kK);
+#pragma unroll
+                for (int pc = 0; pc < P; ++pc) {
+                    const float2 sc = *reinterpret_cast<const float2*>(ss + 2 * pc);
+                    if (ti.prec == 8)
+                        pair_ktS<GROUP, 8>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, ks, lane, u[pc]);
+                    else
+                        pair_ktS<GROUP, 4>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, ks, lane, u[pc]);
+                }
+                r.advance(NS);
+            }
+#pragma unroll
+            for (int pc = 0; pc < P; ++pc) {
+                const float2 vv = *reinterpret_cast<const float2*>(v_s + lane * C + 2 * pc);
+                // w = beta (v - alpha u): three separate roundings
+                const float d0 = __fsub_rn(vv.x, __fmul_rn(gscalar, u[pc].x));
+                const float d1 = __fsub_rn(vv.y, __fmul_rn(gscalar, u[pc].y));
+                w[pc] = make_float2(__fmul_rn(beta, d0), __fmul_rn(beta, d1));
+            }
         } else {
-            *reinterpret_cast<float2*>(op) = make_float2(o[0], o[1]);
+#pragma unroll
+            for (int pc = 0; pc < P; ++pc)
+                w[pc] = *reinterpret_cast<const float2*>(v_s + lane * C + 2 * pc);
+        }
+
+        uint8_t* gcodes_tile = p.codes + ti.code_off;
+        const uint32_t cbytes = GROUP * DV * ti.prec / 8;
+        for (int g = 0; g < G; ++g) {
+            if (UPD != kDelta && g > 0) {
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait_bounded(&bars[ic.slot], ic.par, p.timeout_ns));
+                if (!ok) break;
+            }
+            const uint8_t* sm = wsm + S::kHeader + ic.slot * S::kBytes;
+            const float* ss = reinterpret_cast<const float*>(sm + S::kScales) + lane * C;
+            const float* qs = reinterpret_cast<const float*>(sm + S::kQ);
+            const float* ks = reinterpret_cast<const float*>(sm + S::kK);
+            const float* gs = reinterpret_cast<const float*>(sm + S::kG);
+            float* gscale = p.scales + (static_cast<int64_t>(tile) * G + g) * DV + lane * C;
+            uint8_t* gcodes = gcodes_tile + static_cast<int64_t>(g) * cbytes;
+#pragma unroll
+            for (int pc = 0; pc < P; ++pc) {
+                const float2 sc = *reinterpret_cast<const float2*>(ss + 2 * pc);
+                const uint32_t j0 = static_cast<uint32_t>(lane * C + 2 * pc);
+                if (ti.prec == 8)
+                    pair_step<GROUP, GATE, MODE, 8>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs, ks,
+                                                    gs, gscalar, w[pc], o[pc], gcodes,
+                                                    gscale + 2 * pc, hkey, g * GROUP, j0, lane);
+                else
+                    pair_step<GROUP, GATE, MODE, 4>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs, ks,
+                                                    gs, gscalar, w[pc], o[pc], gcodes,
+                                                    gscale + 2 * pc, hkey, g * GROUP, j0, lane);
+            }
+            ++kc;
+            ic.advance(NS);
+            __syncwarp();
+            if (lane == 0) fence_proxy_async_smem();
+            issue_next();
+        }
+        if (!ok) break;
+        float* op = p.out + static_cast<int64_t>(tile) * DV + lane * C;
+        if constexpr (P == 2) {
+            *reinterpret_cast<float4*>(op) = make_float4(o[0].x, o[0].y, o[1].x, o[1].y);
+        } else {
+            *reinterpret_cast<float2*>(op) = o[0];
+        }
+    }
+    if (!ok) {
+        // Record the timeout, then wait (bounded) for this warp's copies
+        // still in flight before leaving, so none lands after exit.
+        if (lane == 0) atomicOr(p.err, kErrTimeout);
+        Ring r = ic;
+        for (int64_t k = kc; k < ki; ++k) {
+            mbar_wait_bounded(&bars[r.slot], r.par, p.timeout_ns);
+            r.advance(NS);
         }
     }
 }

@@ -150,3 +150,72 @@ def test_fp32_state_kernel_matches_oracle():
                                      update_kind=w.update_kind, gate_kind=w.gate_kind)
             np.testing.assert_array_equal(out.cpu().numpy().reshape(n, -1), o_ref)
             np.testing.assert_array_equal(S.cpu().numpy().reshape(n, w.d_k, w.d_v), S_ref)
+
+
+HAND = ["hand_gla_int8_rtn_4x2.txt", "hand_gla_int8_bdr_2x2.txt", "hand_gdn_int4_rtn_2x2.txt",
+        "hand_gla_int8_ties_2x2.txt", "hand_clamp_int8_1x2.txt",
+        "hand_exact_product_int8_2x2.txt", "hand_bdr_zero_move_int8_2x2.txt"]
+
+
+@pytest.mark.parametrize("name", HAND)
+@pytest.mark.parametrize("mode", [I.ROUND_RTN, I.ROUND_SR, I.ROUND_BDR])
+def test_hand_fixtures_on_gpu(name, mode):
+    """The hand-derived steps, embedded in a 16-row-group, 64-column tile
+    (each fixture group in its own 16-row group, other rows and columns zero):
+    the GPU matches the oracle on the embedded problem, and the fixture's own
+    codes where it states them (RTN, BDR)."""
+    from tests.conftest import read_fixture
+    fx = read_fixture(name)
+    dk, dv, grp = (int(fx[k][0]) for k in ("d_k", "d_v", "group"))
+    bits = int(fx["bits"][0])
+    G = dk // grp
+    DK, DV = 16 * G, 64
+    rows = np.array([(i // grp) * 16 + i % grp for i in range(dk)])
+    delta = fx["update"][0] == "delta"
+    perkey = fx["gate"][0] == "per_key"
+    codes = np.zeros((1, 1, DK, DV), np.int8)
+    codes[0, 0, rows[:, None], np.arange(dv)[None, :]] = \
+        np.array([int(c) for c in fx["codes_old"]]).reshape(dk, dv)
+    scales = np.zeros((1, 1, G, DV), np.float32)
+    scales[0, 0, :, :dv] = np.array([float(c) for c in fx["scales_old"]]).reshape(G, dv)
+    emb = lambda key, n, fill=0.0: _embed(fx, key, n, rows, fill)
+    q, k = emb("q", DK), emb("k", DK)
+    v = np.zeros(DV, np.float32)
+    v[:dv] = [float(c) for c in fx["v"]]
+    gates = emb("gates", DK, 1.0) if perkey else np.array([float(fx["gates"][0])], np.float32)
+    beta = np.array([float(fx["beta"][0])], np.float32) if delta else None
+    shp = lrs.shape(1, 1, DK, DV, 16, 1 if delta else 0, 1 if perkey else 0)
+    pm = np.array([bits], np.uint8)
+    st = lrs.lrs_state_alloc(shp, pm)
+    try:
+        lrs.lrs_state_import_codes(st, torch.from_numpy(codes).cuda(),
+                                   torch.from_numpy(scales).cuda())
+        out = torch.empty(1, 1, DV, device="cuda")
+        t = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).cuda()
+        lrs.lrs_decode_step(st, st.state_codes, st.scales, st.prec_map, t(q), t(k), t(v),
+                            t(gates), t(beta), out, 7, 3, mode)
+        lrs.lrs_sync()
+        got = torch.empty(1, 1, DK, DV, dtype=torch.int8, device="cuda")
+        lrs.lrs_state_export_codes(st, got)
+        lrs.lrs_sync()
+        got = got.cpu().numpy()[0, 0]
+        rc, rs = codes[0].copy(), scales[0].copy()
+        ro = oracle.step(rc, rs, q[None], k[None], v[None], gates[None], beta, pm, [0], [0],
+                         group=16, update_kind=1 if delta else 0, gate_kind=1 if perkey else 0,
+                         mode=mode, seed=7, step=3)
+        np.testing.assert_array_equal(got, rc[0])
+        np.testing.assert_array_equal(out.cpu().numpy()[0, 0], ro[0])
+        key = {I.ROUND_RTN: "codes_rtn", I.ROUND_BDR: "codes_bdr"}.get(mode)
+        if key in fx:
+            expect = np.array([int(c) for c in fx[key]]).reshape(dk, dv)
+            np.testing.assert_array_equal(got[rows[:, None], np.arange(dv)[None, :]], expect)
+            np.testing.assert_array_equal(out.cpu().numpy()[0, 0, :dv],
+                                          np.array([float(c) for c in fx["out"]], np.float32))
+    finally:
+        lrs.lrs_state_free(st)
+
+
+def _embed(fx, key, n, rows, fill):
+    a = np.full(n, fill, np.float32)
+    a[rows] = [float(c) for c in fx[key]]
+    return a

@@ -13,16 +13,22 @@ from tests import parity as P
 pytestmark = pytest.mark.gpu
 
 
-def pack_tile_reference(codes, bits):
+def pack_tile_reference(codes, bits, group):
     """Packed bytes of one tile, written from the layout documented in lrs.h:
-    lane t owns columns [t*C, t*C+C); its codes, row-major over (row, column),
-    form a byte stream (offset binary; int4: byte n of each 32-bit word holds
-    elements n and n+4) cut into 16-byte units, unit u of lane t at (u*32+t)*16."""
+    lane t owns columns [t*C, t*C+C); its codes, ordered by scale group, column
+    pair, key row, column within the pair, form a byte stream (offset binary;
+    int4: byte n of each 32-bit word holds elements n and n+4) cut into
+    16-byte units, unit u of lane t at (u*32+t)*16."""
     d_k, d_v = codes.shape
     C = d_v // 32
     tile = np.zeros(d_k * d_v * bits // 8, np.uint8)
     for t in range(32):
-        elems = codes[:, t * C:(t + 1) * C].reshape(-1).astype(np.int64)
+        elems = []
+        for g in range(d_k // group):
+            for p in range(C // 2):
+                cols = codes[g * group:(g + 1) * group, t * C + 2 * p: t * C + 2 * p + 2]
+                elems.append(cols.reshape(-1))
+        elems = np.concatenate(elems).astype(np.int64)
         if bits == 8:
             stream = (elems + 128).astype(np.uint8)
         else:
@@ -61,7 +67,8 @@ def test_packed_layout_and_code_round_trip(d_k, d_v, group):
             for h in range(H):
                 n = d_k * d_v * int(pm[h]) // 8
                 got = raw[b * stride + offs[h]: b * stride + offs[h] + n]
-                np.testing.assert_array_equal(got, pack_tile_reference(codes[b, h], int(pm[h])))
+                np.testing.assert_array_equal(got, pack_tile_reference(codes[b, h], int(pm[h]),
+                                                                          group))
         back = torch.empty(B, H, d_k, d_v, dtype=torch.int8, device="cuda")
         lrs.lrs_state_export_codes(st, back)
         np.testing.assert_array_equal(back.cpu().numpy(), codes)
