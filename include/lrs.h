@@ -175,6 +175,37 @@ lrs_status lrs_decode_step_host(const lrs_state *st, const float *q_host, const 
                                 const float *beta_host, float *out_host, uint64_t seed,
                                 uint64_t step, int32_t mode, void *stream);
 
+/* lrs_decode_step_host without any device allocation. This entry point has no
+ * counterpart in the method's sources; it exists for callers that cannot
+ * allocate device memory at the time they step: code running while a stream
+ * is captured into a CUDA graph (where cudaMalloc is not allowed), and
+ * processes whose device memory belongs to another allocator or a fixed pool.
+ * Its scratch -- a device error word and the staging of q, k, v, gates, beta
+ * and out -- is a 32 MiB array inside the library's image, which every GPU
+ * that loads the library holds until the process exits. It calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *   - Limit: the staging must fit: 256 + 16-byte-padded sizes of q, k
+ *     ([B][H][d_k]), v, out ([B][H][d_v]), gates and beta must not exceed
+ *     32 MiB; a larger step is rejected with LRS_ERR_UNSUPPORTED and nothing
+ *     is launched. (B=256, H=32, 128x128 with per-key gates needs 20 MiB.)
+ *   - The first call on a device looks up the array's device address; make
+ *     it before any stream capture on that device.
+ *   - Every call shares the one array, which keeps the last call's contents:
+ *     calls that overlap on the GPU (other streams, other threads) race and
+ *     corrupt each other's inputs and outputs. Serialize them.
+ *   - device_error_host (may be NULL) receives, asynchronously on stream, the
+ *     device error bits of this call's kernel: 0 when none, else bit 0 = a
+ *     wait timed out, bit 1 = the precision map did not fit the layout. The
+ *     word is cleared at the start of each call; lrs_sync does not see it.
+ * Arguments otherwise as lrs_decode_step_host (the state's own buffers are
+ * stepped; host buffers pinned for asynchronous copies). */
+lrs_status lrs_decode_step_host_noalloc(const lrs_state *st, const float *q_host,
+                                        const float *k_host, const float *v_host,
+                                        const float *gates_host, const float *beta_host,
+                                        float *out_host, uint32_t *device_error_host,
+                                        uint64_t seed, uint64_t step, int32_t mode,
+                                        void *stream);
+
 /* Quantize an fp32 state S [B][H][d_k][d_v] (device) into st with
  * round-to-nearest (new scales and codes exactly as in a step with x = S). */
 lrs_status lrs_state_import_fp32(const lrs_state *st, const float *S, void *stream);

@@ -645,3 +645,14 @@ lrs_status lrs_debug_inject_timeout(int32_t enable, int32_t timeout_us) {
 }
 
 }  // extern "C"
+
+namespace lrs {
+
+// Status helpers for entry points defined in other translation units: they
+// set and clear the same thread-local message as the functions above.
+lrs_status api_fail(lrs_status s, const char* msg) { return fail(s, "%s", msg); }
+lrs_status api_cuda_fail(cudaError_t e, const char* what) { return cuda_fail(e, what); }
+lrs_status api_ok() { return ok(); }
+lrs_status api_check_state(const lrs_state* st) { return check_state(st); }
+
+}  // namespace lrs

@@ -4,6 +4,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "lrs.h"
+
 namespace lrs {
 
 // Kernel entry of one compiled step variant, or nullptr when the combination
@@ -39,5 +41,11 @@ cudaError_t launch_fp32_step(int B, int H, int d_k, int d_v, int update_kind, in
 cudaError_t launch_decay_means(const float* decay, int64_t outer, int heads, int64_t inner,
                                double* means, cudaStream_t s);
 bool layout_kernels_support(int d_v, int group);
+
+// Status helpers shared by the C-ABI translation units (lrs_api.cu).
+lrs_status api_fail(lrs_status s, const char* msg);
+lrs_status api_cuda_fail(cudaError_t e, const char* what);
+lrs_status api_ok();
+lrs_status api_check_state(const lrs_state* st);
 
 }  // namespace lrs

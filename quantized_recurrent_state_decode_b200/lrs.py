@@ -59,6 +59,8 @@ _SIGS = {
                         ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int32, _P],
     "lrs_decode_step_host": [ctypes.POINTER(lrs_state), _P, _P, _P, _P, _P, _P,
                              ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int32, _P],
+    "lrs_decode_step_host_noalloc": [ctypes.POINTER(lrs_state), _P, _P, _P, _P, _P, _P, _P,
+                                     ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int32, _P],
     "lrs_state_import_fp32": [ctypes.POINTER(lrs_state), _P, _P],
     "lrs_state_export_fp32": [ctypes.POINTER(lrs_state), _P, _P],
     "lrs_state_export_codes": [ctypes.POINTER(lrs_state), _P, _P],
@@ -172,6 +174,14 @@ def lrs_decode_step_host(st, q_host, k_host, v_host, gates_host, beta_host, out_
     _check(lib().lrs_decode_step_host(ctypes.byref(st), _ptr(q_host), _ptr(k_host),
                                       _ptr(v_host), _ptr(gates_host), _ptr(beta_host),
                                       _ptr(out_host), seed, step, mode, _stream(stream)))
+
+
+def lrs_decode_step_host_noalloc(st, q_host, k_host, v_host, gates_host, beta_host, out_host,
+                                 device_error_host, seed, step, mode, stream=None):
+    _check(lib().lrs_decode_step_host_noalloc(
+        ctypes.byref(st), _ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(gates_host),
+        _ptr(beta_host), _ptr(out_host), _ptr(device_error_host), seed, step, mode,
+        _stream(stream)))
 
 
 def lrs_state_import_fp32(st, S, stream=None):
