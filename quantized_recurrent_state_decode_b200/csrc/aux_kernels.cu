@@ -2,7 +2,7 @@
 // decode step used as the uncompressed baseline, and the per-head mean decay.
 //
 // The quantizing kernels here share the step kernel's rounding and packing
-// (round_pair / encode_word), so an imported state is exactly the state a step
+// (round_rows / encode_word), so an imported state is exactly the state a step
 // with x = S would produce.
 #include "lrs_internal.h"
 #include "step_kernel.cuh"
@@ -49,7 +49,7 @@ __device__ void encode_pair_rtn(const float2 (&x)[GROUP], float2 inv, uint8_t* g
 #pragma unroll
             for (int e = 0; e < G::EPW; e += 2) {
                 const int r = un * G::RPU + (wi * G::EPW + e) / 2;
-                const float2 tv = round_pair<kRTN, BITS>(x[r], inv, f2(0.f), f2(0.f), 0ull, 0u, 0u);
+                const float2 tv = round_rows<kRTN, BITS>(x[r], inv, f2(0.f), f2(0.f), 0ull, 0u, 0u);
                 t[e] = tv.x;
                 t[e + 1] = tv.y;
             }
@@ -109,10 +109,10 @@ __device__ void layout_op_tile(const LayoutArgs& a, int op, int tile, uint8_t* t
                     A1 = fmaxf(A1, fabsf(x[r].y));
                 }
                 constexpr float QF = static_cast<float>(QMAX);
-                const float2 snew = make_float2(A0 < kTiny ? 0.0f : __fdiv_rn(A0, QF),
-                                                A1 < kTiny ? 0.0f : __fdiv_rn(A1, QF));
-                const float2 inv = make_float2(A0 < kTiny ? 0.0f : __fdiv_rn(QF, A0),
-                                               A1 < kTiny ? 0.0f : __fdiv_rn(QF, A1));
+                const float2 snew = make_float2(A0 < kTiny ? 0.0f : div_by_qmax<QMAX>(A0),
+                                                A1 < kTiny ? 0.0f : div_by_qmax<QMAX>(A1));
+                const float2 inv = make_float2(A0 < kTiny ? 0.0f : div_rn_fast(QF, A0),
+                                               A1 < kTiny ? 0.0f : div_rn_fast(QF, A1));
                 gscales[j] = snew.x;
                 gscales[j + 1] = snew.y;
                 encode_pair_rtn<GROUP, BITS>(x, inv, gcodes, pc, lane);

@@ -77,7 +77,8 @@ struct Slot {
 };
 
 // ------------------------------------------------------- packed fp32 math ---
-// The two columns of a pair go through the sm_100 two-wide fp32 instructions;
+// Two consecutive key rows of one column go through the sm_100 two-wide fp32
+// instructions;
 // each half is an IEEE binary32 operation rounded to nearest even. They are
 // written with an explicit .rn so that no multiply and add is ever fused into
 // one rounding behind our back (results must follow the stated roundings).
@@ -155,12 +156,12 @@ template <int BITS> struct Q;
 template <> struct Q<8> { static constexpr float kMax = 127.0f, kBias = 128.0f; };
 template <> struct Q<4> { static constexpr float kMax = 7.0f, kBias = 8.0f; };
 
-// Codes of two elements (value columns j, j+1 of key row i), returned as the
-// floats 1.5*2^23 + bias + code whose low byte is the stored byte. The value
-// rounded is the exact product x*inv: one fused multiply-add rounds it
-// straight to an integer.
+// Codes of two elements (key rows i, i+1 of value column j), returned as the
+// floats 1.5*2^23 + bias + code whose low byte is the stored byte. inv,
+// s_new: the column's values in both halves. The value rounded is the exact
+// product x*inv: one fused multiply-add rounds it straight to an integer.
 template <int MODE, int BITS>
-__device__ __forceinline__ float2 round_pair(float2 x, float2 inv, float2 deq, float2 s_new,
+__device__ __forceinline__ float2 round_rows(float2 x, float2 inv, float2 deq, float2 s_new,
                                              uint64_t hkey, uint32_t i, uint32_t j) {
     constexpr float QMAX = Q<BITS>::kMax, BIAS = Q<BITS>::kBias;
     if constexpr (MODE == kRTN) {
@@ -176,7 +177,7 @@ __device__ __forceinline__ float2 round_pair(float2 x, float2 inv, float2 deq, f
                                          d.y < 0.0f ? n.y - 1.0f : n.y);  // floor
             const float2 fr = fma2(x, inv, neg2(f));                      // fraction, rounded once
             const float u0 = element_uniform(hkey, i, j);
-            const float u1 = element_uniform(hkey, i, j + 1);
+            const float u1 = element_uniform(hkey, i + 1, j);
             c.x = u0 < fr.x ? f.x + 1.0f : f.x;
             c.y = u1 < fr.y ? f.y + 1.0f : f.y;
         } else {
@@ -185,11 +186,16 @@ __device__ __forceinline__ float2 round_pair(float2 x, float2 inv, float2 deq, f
             const float2 delta = add2(x, neg2(deq));
             const float2 m = make_float2(__fsub_rn(__fmul_rn(n.x, s_new.x), deq.x),
                                          __fsub_rn(__fmul_rn(n.y, s_new.y), deq.y));
-            c = n;
-            if (delta.x > 0.0f && m.x < 0.0f) c.x = d.x > 0.0f ? n.x + 1.0f : n.x;       // ceil
-            else if (delta.x < 0.0f && m.x > 0.0f) c.x = d.x < 0.0f ? n.x - 1.0f : n.x;  // floor
-            if (delta.y > 0.0f && m.y < 0.0f) c.y = d.y > 0.0f ? n.y + 1.0f : n.y;
-            else if (delta.y < 0.0f && m.y > 0.0f) c.y = d.y < 0.0f ? n.y - 1.0f : n.y;
+            // A reversal (update and move of opposite signs) takes ceil(x*inv)
+            // when the update is positive and floor(x*inv) when it is
+            // negative; ceil = n + 1 exactly when x*inv > n, floor = n - 1
+            // exactly when x*inv < n. Written with selects, no branches.
+            const bool up0 = (delta.x > 0.0f) & (m.x < 0.0f) & (d.x > 0.0f);
+            const bool dn0 = (delta.x < 0.0f) & (m.x > 0.0f) & (d.x < 0.0f);
+            const bool up1 = (delta.y > 0.0f) & (m.y < 0.0f) & (d.y > 0.0f);
+            const bool dn1 = (delta.y < 0.0f) & (m.y > 0.0f) & (d.y < 0.0f);
+            c.x = n.x + (up0 ? 1.0f : 0.0f) - (dn0 ? 1.0f : 0.0f);
+            c.y = n.y + (up1 ? 1.0f : 0.0f) - (dn1 ? 1.0f : 0.0f);
         }
         c.x = fminf(fmaxf(c.x, -QMAX), QMAX);
         c.y = fminf(fmaxf(c.y, -QMAX), QMAX);
@@ -219,10 +225,14 @@ __device__ __forceinline__ void ld_smem_rows(const float* p, float (&r)[N]) {
 
 // Geometry of one lane's codes for one column pair of one scale group: a run
 // of 16-byte units, each holding EPU consecutive elements of the pair's
-// row-major (row, column) stream, i.e. RPU key rows.
+// row-major (row, column) stream, i.e. RPU key rows; a 32-bit word holds RPW
+// rows. The packed arithmetic works on two consecutive key rows of one
+// column: in a word, the rows (r, r+1) of column c are elements 4p + c and
+// 4p + 2 + c for row pair p of the word.
 template <int GROUP, int BITS>
 struct PairGeo {
     static constexpr int EPW = 32 / BITS;       // elements per 32-bit word
+    static constexpr int RPW = EPW / 2;         // key rows per word
     static constexpr int EPU = 4 * EPW;         // elements per 16-byte unit
     static constexpr int RPU = EPU / 2;         // key rows per unit
     static constexpr int UNITS = GROUP / RPU;   // units per pair per group
@@ -233,13 +243,14 @@ __device__ __forceinline__ uint4 lds_unit(const uint8_t* cs, int unit, int lane)
     return *reinterpret_cast<const uint4*>(cs + (unit * 32 + lane) * 16);
 }
 
-// Delta rule, first pass: u += k_i * deq_i for one column pair over the rows
-// of one group, in key order.
+// Delta rule, first pass: u_c += k_i * deq_ic for the two columns of one
+// pair over the rows of one group, in key order.
 template <int GROUP, int BITS>
 __device__ __forceinline__ void pair_ktS(const uint8_t* __restrict__ cs, int ubase, float2 sc,
                                          const float* __restrict__ ks, int lane, float2& u) {
     using G = PairGeo<GROUP, BITS>;
     constexpr float BIAS = Q<BITS>::kBias;
+    const float2 s0 = f2(sc.x), s1 = f2(sc.y);
 #pragma unroll
     for (int un = 0; un < G::UNITS; ++un) {
         const uint4 raw = lds_unit(cs, ubase + un, lane);
@@ -251,17 +262,24 @@ __device__ __forceinline__ void pair_ktS(const uint8_t* __restrict__ cs, int uba
             float f[G::EPW];
             decode_word_biased<BITS>(wd[wi], f);
 #pragma unroll
-            for (int e = 0; e < G::EPW; e += 2) {
-                const int rl = (wi * G::EPW + e) / 2;
-                const float2 code = add2(make_float2(f[e], f[e + 1]), f2(-(kTwo23 + BIAS)));
-                u = fma2(f2(kk[rl]), mul2(code, sc), u);
+            for (int rp = 0; rp < G::RPW / 2; ++rp) {
+                const int rl = wi * G::RPW + 2 * rp;
+                const float2 kr = make_float2(kk[rl], kk[rl + 1]);
+                const float2 c0 = add2(make_float2(f[4 * rp], f[4 * rp + 2]), f2(-(kTwo23 + BIAS)));
+                const float2 c1 = add2(make_float2(f[4 * rp + 1], f[4 * rp + 3]), f2(-(kTwo23 + BIAS)));
+                const float2 d0 = mul2(c0, s0), d1 = mul2(c1, s1);
+                u.x = __fmaf_rn(kr.x, d0.x, u.x);
+                u.x = __fmaf_rn(kr.y, d0.y, u.x);
+                u.y = __fmaf_rn(kr.x, d1.x, u.y);
+                u.y = __fmaf_rn(kr.y, d1.y, u.y);
             }
         }
     }
 }
 
 // One column pair of one scale group: dequantize, update, accumulate the
-// output, new scales, requantize and store.
+// output, new scales, requantize and store. x[rp][c] holds rows (2rp, 2rp+1)
+// of column c of the pair.
 template <int GROUP, int GATE, int MODE, int BITS>
 __device__ __forceinline__ void pair_step(const uint8_t* __restrict__ cs, int ubase, float2 sc,
                                           const float* __restrict__ qs,
@@ -272,7 +290,10 @@ __device__ __forceinline__ void pair_step(const uint8_t* __restrict__ cs, int ub
                                           uint32_t j0, int lane) {
     using G = PairGeo<GROUP, BITS>;
     constexpr float QMAX = Q<BITS>::kMax, BIAS = Q<BITS>::kBias;
-    float2 x[GROUP];
+    const float2 s0 = f2(sc.x), s1 = f2(sc.y);     // per-column constants as pairs
+    const float2 w0 = f2(w.x), w1 = f2(w.y);
+    const float2 gsc = f2(gscalar);
+    float2 x[GROUP / 2][2];
 
 #pragma unroll
     for (int un = 0; un < G::UNITS; ++un) {
@@ -287,15 +308,22 @@ __device__ __forceinline__ void pair_step(const uint8_t* __restrict__ cs, int ub
             float f[G::EPW];
             decode_word_biased<BITS>(wd[wi], f);
 #pragma unroll
-            for (int e = 0; e < G::EPW; e += 2) {
-                const int rl = (wi * G::EPW + e) / 2;
-                const float gi = GATE == kGatePerKey ? gg[rl] : gscalar;
-                const float2 code = add2(make_float2(f[e], f[e + 1]), f2(-(kTwo23 + BIAS)));
-                const float2 deq = mul2(code, sc);
-                const float2 kw = mul2(f2(kk[rl]), w);
-                const float2 xv = fma2(f2(gi), deq, kw);
-                o = fma2(f2(qq[rl]), xv, o);
-                x[un * G::RPU + rl] = xv;
+            for (int rp = 0; rp < G::RPW / 2; ++rp) {
+                const int rl = wi * G::RPW + 2 * rp;
+                const int r = un * G::RPU + rl;
+                const float2 kr = make_float2(kk[rl], kk[rl + 1]);
+                const float2 qr = make_float2(qq[rl], qq[rl + 1]);
+                const float2 gr = GATE == kGatePerKey ? make_float2(gg[rl], gg[rl + 1]) : gsc;
+                const float2 c0 = add2(make_float2(f[4 * rp], f[4 * rp + 2]), f2(-(kTwo23 + BIAS)));
+                const float2 c1 = add2(make_float2(f[4 * rp + 1], f[4 * rp + 3]), f2(-(kTwo23 + BIAS)));
+                const float2 x0 = fma2(gr, mul2(c0, s0), mul2(kr, w0));
+                const float2 x1 = fma2(gr, mul2(c1, s1), mul2(kr, w1));
+                o.x = __fmaf_rn(qr.x, x0.x, o.x);
+                o.x = __fmaf_rn(qr.y, x0.y, o.x);
+                o.y = __fmaf_rn(qr.x, x1.x, o.y);
+                o.y = __fmaf_rn(qr.y, x1.y, o.y);
+                x[r / 2][0] = x0;
+                x[r / 2][1] = x1;
             }
         }
     }
@@ -303,19 +331,22 @@ __device__ __forceinline__ void pair_step(const uint8_t* __restrict__ cs, int ub
     // absmax per column over the group's rows (order-free)
     float a0 = 0.0f, a1 = 0.0f, b0 = 0.0f, b1 = 0.0f;
 #pragma unroll
-    for (int r = 0; r < GROUP; r += 4) {
-        a0 = max_abs3(a0, x[r].x, x[r + 1].x);
-        a1 = max_abs3(a1, x[r + 2].x, x[r + 3].x);
-        b0 = max_abs3(b0, x[r].y, x[r + 1].y);
-        b1 = max_abs3(b1, x[r + 2].y, x[r + 3].y);
+    for (int rp = 0; rp < GROUP / 2; rp += 2) {
+        a0 = max_abs3(a0, x[rp][0].x, x[rp][0].y);
+        a1 = max_abs3(a1, x[rp + 1][0].x, x[rp + 1][0].y);
+        b0 = max_abs3(b0, x[rp][1].x, x[rp][1].y);
+        b1 = max_abs3(b1, x[rp + 1][1].x, x[rp + 1][1].y);
     }
     const float A0 = fmaxf(a0, a1), A1 = fmaxf(b0, b1);
     float2 snew, inv;
-    snew.x = A0 < kTiny ? 0.0f : __fdiv_rn(A0, QMAX);
-    inv.x = A0 < kTiny ? 0.0f : __fdiv_rn(QMAX, A0);
-    snew.y = A1 < kTiny ? 0.0f : __fdiv_rn(A1, QMAX);
-    inv.y = A1 < kTiny ? 0.0f : __fdiv_rn(QMAX, A1);
+    constexpr int QM = static_cast<int>(QMAX);
+    snew.x = A0 < kTiny ? 0.0f : div_by_qmax<QM>(A0);
+    inv.x = A0 < kTiny ? 0.0f : div_rn_fast(QMAX, A0);
+    snew.y = A1 < kTiny ? 0.0f : div_by_qmax<QM>(A1);
+    inv.y = A1 < kTiny ? 0.0f : div_rn_fast(QMAX, A1);
     st_cs_f2(gscale, snew);
+    const float2 inv0 = f2(inv.x), inv1 = f2(inv.y);
+    const float2 sn0 = f2(snew.x), sn1 = f2(snew.y);
 
 #pragma unroll
     for (int un = 0; un < G::UNITS; ++un) {
@@ -331,15 +362,20 @@ __device__ __forceinline__ void pair_step(const uint8_t* __restrict__ cs, int ub
             if constexpr (MODE == kBDR) decode_word_biased<BITS>(wd[wi], f);
             float t[G::EPW];
 #pragma unroll
-            for (int e = 0; e < G::EPW; e += 2) {
-                const int r = un * G::RPU + (wi * G::EPW + e) / 2;
-                float2 deq = f2(0.0f);
-                if constexpr (MODE == kBDR)
-                    deq = mul2(add2(make_float2(f[e], f[e + 1]), f2(-(kTwo23 + BIAS))), sc);
-                const float2 tv = round_pair<MODE, BITS>(x[r], inv, deq, snew, hkey,
-                                                         static_cast<uint32_t>(row0 + r), j0);
-                t[e] = tv.x;
-                t[e + 1] = tv.y;
+            for (int rp = 0; rp < G::RPW / 2; ++rp) {
+                const int r = un * G::RPU + wi * G::RPW + 2 * rp;
+                float2 dq0 = f2(0.0f), dq1 = f2(0.0f);
+                if constexpr (MODE == kBDR) {
+                    dq0 = mul2(add2(make_float2(f[4 * rp], f[4 * rp + 2]), f2(-(kTwo23 + BIAS))), s0);
+                    dq1 = mul2(add2(make_float2(f[4 * rp + 1], f[4 * rp + 3]), f2(-(kTwo23 + BIAS))), s1);
+                }
+                const uint32_t i = static_cast<uint32_t>(row0 + r);
+                const float2 t0 = round_rows<MODE, BITS>(x[r / 2][0], inv0, dq0, sn0, hkey, i, j0);
+                const float2 t1 = round_rows<MODE, BITS>(x[r / 2][1], inv1, dq1, sn1, hkey, i, j0 + 1);
+                t[4 * rp] = t0.x;
+                t[4 * rp + 2] = t0.y;
+                t[4 * rp + 1] = t1.x;
+                t[4 * rp + 3] = t1.y;
             }
             ow[wi] = encode_word<BITS>(t);
         }
