@@ -141,15 +141,42 @@ __device__ __forceinline__ void decode_word_biased(uint32_t w, float (&f)[32 / B
     }
 }
 
+// Pack the stored bytes (nibbles) of 4 (8) rounded codes into one word. The
+// bit pattern of each rounded value t is K + u, K = bits(1.5 * 2^23), u the
+// stored byte (nibble), so the word is sum(bits(t_n) << shift_n) minus
+// K * sum(1 << shift_n), all modulo 2^32: integer multiply-adds, which run on
+// the fused-multiply-add pipe beside the byte permutes of the decode.
 template <int BITS>
 __device__ __forceinline__ uint32_t encode_word(const float (&t)[32 / BITS]) {
+    constexpr uint32_t K = 0x4B400000u;
+    uint32_t r;
     if constexpr (BITS == 8) {
-        return pack_low_bytes(t[0], t[1], t[2], t[3]);
+        constexpr uint32_t KS = K * 0x01010101u;
+        asm("{\n\t.reg .u32 a;\n\t"
+            "mad.lo.u32 a, %2, 256, %1;\n\t"
+            "mad.lo.u32 a, %3, 65536, a;\n\t"
+            "mad.lo.u32 a, %4, 16777216, a;\n\t"
+            "sub.u32 %0, a, %5;\n\t}"
+            : "=r"(r)
+            : "r"(__float_as_uint(t[0])), "r"(__float_as_uint(t[1])), "r"(__float_as_uint(t[2])),
+              "r"(__float_as_uint(t[3])), "r"(KS));
     } else {
-        const uint32_t lo = pack_low_bytes(t[0], t[1], t[2], t[3]);
-        const uint32_t hi = pack_low_bytes(t[4], t[5], t[6], t[7]);
-        return lo | (hi << 4);
+        constexpr uint32_t KS = K * 0x11111111u;
+        asm("{\n\t.reg .u32 a;\n\t"
+            "mad.lo.u32 a, %2, 16, %1;\n\t"
+            "mad.lo.u32 a, %3, 256, a;\n\t"
+            "mad.lo.u32 a, %4, 4096, a;\n\t"
+            "mad.lo.u32 a, %5, 65536, a;\n\t"
+            "mad.lo.u32 a, %6, 1048576, a;\n\t"
+            "mad.lo.u32 a, %7, 16777216, a;\n\t"
+            "mad.lo.u32 a, %8, 268435456, a;\n\t"
+            "sub.u32 %0, a, %9;\n\t}"
+            : "=r"(r)
+            : "r"(__float_as_uint(t[0])), "r"(__float_as_uint(t[4])), "r"(__float_as_uint(t[1])),
+              "r"(__float_as_uint(t[5])), "r"(__float_as_uint(t[2])), "r"(__float_as_uint(t[6])),
+              "r"(__float_as_uint(t[3])), "r"(__float_as_uint(t[7])), "r"(KS));
     }
+    return r;
 }
 
 template <int BITS> struct Q;
@@ -383,46 +410,63 @@ __device__ __forceinline__ void pair_step(const uint8_t* __restrict__ cs, int ub
     }
 }
 
-// Layout of tile `tile`: byte offset of its codes and its precision, or
-// prec = 0 when prec_map does not fit the offsets.
-struct TileInfo {
+// A warp's walk over its tiles gw, gw + W, ...: the tile's batch row and
+// head are advanced incrementally (no division per tile), and its layout
+// read from the precision map and head offsets: the byte offset of its codes
+// and its precision, or prec = 0 when prec_map does not fit the offsets.
+struct TileCursor {
+    int tile, b, h;
+    int db, dh;          // W / H and W % H
     int64_t code_off;
     int prec;
+
+    __device__ __forceinline__ void init(const StepParams& p, int first, int W) {
+        tile = first;
+        b = first / p.H;
+        h = first - b * p.H;
+        db = W / p.H;
+        dh = W - db * p.H;
+    }
+    __device__ __forceinline__ void advance(const StepParams& p, int W) {
+        tile += W;
+        b += db;
+        h += dh;
+        if (h >= p.H) {
+            h -= p.H;
+            ++b;
+        }
+    }
+    __device__ __forceinline__ void load(const StepParams& p, int dv) {
+        const int pr = __ldg(p.prec_map + h);
+        const int64_t off = __ldg(p.head_offsets + h);
+        const int64_t end = (h + 1 < p.H) ? __ldg(p.head_offsets + h + 1) : p.batch_stride;
+        const int64_t bytes = static_cast<int64_t>(p.d_k) * dv * pr / 8;
+        prec = ((pr == 4 || pr == 8) && off >= 0 && off + bytes <= end) ? pr : 0;
+        code_off = static_cast<int64_t>(b) * p.batch_stride + off;
+    }
 };
 
-__device__ __forceinline__ TileInfo tile_info(const StepParams& p, int tile, int dv) {
-    const int h = tile % p.H;
-    const int b = tile / p.H;
-    const int prec = __ldg(p.prec_map + h);
-    const int64_t off = __ldg(p.head_offsets + h);
-    const int64_t end = (h + 1 < p.H) ? __ldg(p.head_offsets + h + 1) : p.batch_stride;
-    const int64_t bytes = static_cast<int64_t>(p.d_k) * dv * prec / 8;
-    TileInfo ti;
-    ti.prec = ((prec == 4 || prec == 8) && off >= 0 && off + bytes <= end) ? prec : 0;
-    ti.code_off = static_cast<int64_t>(b) * p.batch_stride + off;
-    return ti;
-}
-
-// Fill `slot` with group g of tile `tile` (lane 0 only). A tile whose layout
-// does not fit gets a bare arrival, so the slot's phase still completes.
+// Fill `slot` with group g of the cursor's tile (lane 0 only). A tile whose
+// layout does not fit gets a bare arrival, so the slot's phase still completes.
 template <int C, int GROUP, int GATE>
-__device__ __forceinline__ void issue_item(const StepParams& p, uint8_t* wsm, int slot, int tile,
-                                           int g, uint64_t pol_state, uint64_t pol_in) {
+__device__ __forceinline__ void issue_item(const StepParams& p, uint8_t* wsm, int slot,
+                                           const TileCursor& tc, int g, uint64_t pol_state,
+                                           uint64_t pol_in) {
     using S = Slot<C, GROUP, GATE>;
     constexpr int DV = 32 * C;
     uint64_t* bar = reinterpret_cast<uint64_t*>(wsm) + slot;
-    const TileInfo ti = tile_info(p, tile, DV);
-    if (ti.prec == 0) {
+    if (tc.prec == 0) {
         mbar_arrive(bar);
         return;
     }
+    const int tile = tc.tile;
     uint8_t* sm = wsm + S::kHeader + slot * S::kBytes;
-    const uint32_t cbytes = GROUP * DV * ti.prec / 8;
+    const uint32_t cbytes = GROUP * DV * tc.prec / 8;
     uint32_t total = cbytes + DV * 4 + 2 * GROUP * 4;
     if (GATE == kGatePerKey) total += GROUP * 4;
     if (g == 0) total += DV * 4;
     mbar_arrive_expect_tx(bar, total);
-    bulk_g2s(sm, p.codes + ti.code_off + static_cast<int64_t>(g) * cbytes, cbytes, bar, pol_state);
+    bulk_g2s(sm, p.codes + tc.code_off + static_cast<int64_t>(g) * cbytes, cbytes, bar, pol_state);
     bulk_g2s(sm + S::kScales, p.scales + (static_cast<int64_t>(tile) * p.G + g) * DV, DV * 4, bar,
              pol_state);
     const int64_t rowbase = static_cast<int64_t>(tile) * p.d_k + g * GROUP;
@@ -476,18 +520,20 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
     const uint64_t pol_in = policy_evict_first();
     Ring ic, is;                 // consumer and issuer positions
     int64_t kc = 0, ki = 0;      // items consumed, items issued
-    int it_tile = 0, it_g = 0;   // (tile of this warp, group) of item ki
+    int it_g = 0;                // group of item ki
+    TileCursor itc;              // tile of item ki
+    itc.init(p, gw, W);
+    if (K > 0) itc.load(p, DV);
 
     auto issue_next = [&]() {
         if (ki < K && !p.inject) {
-            if (lane == 0)
-                issue_item<C, GROUP, GATE>(p, wsm, is.slot, gw + it_tile * W, it_g, pol_state,
-                                           pol_in);
+            if (lane == 0) issue_item<C, GROUP, GATE>(p, wsm, is.slot, itc, it_g, pol_state, pol_in);
             ++ki;
             is.advance(NS);
             if (++it_g == G) {
                 it_g = 0;
-                ++it_tile;
+                itc.advance(p, W);
+                if (ki < K) itc.load(p, DV);
             }
         }
     };
@@ -500,17 +546,19 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
     }
 
     bool ok = true;
-    for (int n = 0; n < ntw && ok; ++n) {
-        const int tile = gw + n * W;
-        const TileInfo ti = tile_info(p, tile, DV);
+    TileCursor ti;               // the consumer's tile
+    ti.init(p, gw, W);
+    for (int n = 0; n < ntw && ok; ++n, ti.advance(p, W)) {
+        const int tile = ti.tile;
+        ti.load(p, DV);
         const float gscalar = nscal, beta = nbeta;
         if (n + 1 < ntw) {
             if (GATE == kGate) nscal = __ldg(p.gates + tile + W);
             if (UPD == kDelta) nbeta = __ldg(p.beta + tile + W);
         }
         const uint64_t hkey = MODE == kSR ? tile_hash_key(p.seed, p.step,
-                                                          static_cast<uint32_t>(tile / p.H),
-                                                          static_cast<uint32_t>(tile % p.H))
+                                                          static_cast<uint32_t>(ti.b),
+                                                          static_cast<uint32_t>(ti.h))
                                           : 0ull;
 
         // the delta rule needs every group of the tile before its first one
