@@ -141,7 +141,7 @@ def run_reference(args, w):
 
     nthreads = oracle.default_threads()
     mode = MODES[args.mode] if args.mode else w.mode
-    pm = I.uniform_prec_map(w).numpy()
+    pm = oracle_precision_map(w)
     # calibrate: time per tile with all threads
     ntiles_all = w.batch * w.heads
     rng = np.random.default_rng(0)
@@ -192,6 +192,16 @@ def run_reference(args, w):
     print(json.dumps(line))
 
 
+def oracle_precision_map(w):
+    import oracle
+    from quantized_recurrent_state_decode_b200 import inputs as I
+    pm = I.uniform_prec_map(w)
+    if pm is not None:
+        return pm.numpy()
+    decay = I.decay_tensor(w, steps=min(w.steps, 16))
+    return oracle.precision_map(oracle.decay_means(decay.numpy()), I.n_int8_heads(w))
+
+
 def config_of(w, mode, layers, n):
     from quantized_recurrent_state_decode_b200 import inputs as I
     prec = {"int8": "int8", "int4": "int4", "mixed": "mixed int8/int4"}[w.precision]
@@ -206,11 +216,30 @@ def config_of(w, mode, layers, n):
 
 # -------------------------------------------------------------------- GPU ---
 
-def state_bytes(w, prec_bits=8):
+def precision_map(w, lrs, dev):
+    """Per-head precision: uniform for int8/int4 workloads; for mixed ones,
+    the library's mean decay per head over the first steps' gates, ranked."""
+    import numpy as np
+    import torch
+    from quantized_recurrent_state_decode_b200 import inputs as I
+    pm = I.uniform_prec_map(w)
+    if pm is not None:
+        return pm.numpy()
+    decay = I.decay_tensor(w, steps=min(w.steps, 16), device=dev)
+    outer, H, inner = decay.shape
+    means = torch.zeros(H, dtype=torch.float64, device=dev)
+    lrs.lrs_decay_head_means(decay, outer, H, inner, means)
+    torch.cuda.synchronize()
+    return lrs.lrs_precision_map(means.cpu().numpy(), I.n_int8_heads(w))
+
+
+def state_bytes(w, pm=None):
     """Algorithmic bytes of one step: codes and scales, each read once and
-    written once."""
+    written once (per-head code widths from the precision map)."""
     G = w.d_k // w.group
-    return 2 * w.batch * w.heads * (w.d_k * w.d_v * prec_bits // 8 + G * w.d_v * 4)
+    bits = [8] * w.heads if pm is None else [int(b) for b in pm]
+    per_row = sum(w.d_k * w.d_v * b // 8 + G * w.d_v * 4 for b in bits)
+    return 2 * w.batch * per_row
 
 
 def run_gpu(args, w):
@@ -238,7 +267,7 @@ def run_gpu(args, w):
     wg = w.with_batch(w.batch * world)
     off, nb = batch_slice(wg.batch, rank, world)
     wl = w.with_batch(nb)
-    pm = I.uniform_prec_map(w).numpy()
+    pm = precision_map(w, lrs, dev)
     shp = lrs.shape(nb, w.heads, w.d_k, w.d_v, w.group, w.update_kind, w.gate_kind)
     L = args.layers
     states = [lrs.lrs_state_alloc(shp, pm) for _ in range(L)]
@@ -297,7 +326,7 @@ def run_gpu(args, w):
         sampler.stop()
 
     steps_per_s = world * args.steps / (ms_max / 1e3)
-    bytes_step = state_bytes(wl)
+    bytes_step = state_bytes(wl, pm)
     launch_s = ms / 1e3 / args.steps
     achieved = bytes_step / launch_s / 1e9
     peak, peak_kind = measured_peaks()
@@ -333,7 +362,7 @@ def run_gpu(args, w):
     extras = {}
     if not args.no_extras and rank == 0:
         with torch.cuda.stream(stream):
-            extras = run_extras(args, w, wl, states, xs, out, seed, stream, L, NI, mode, dev)
+            extras = run_extras(args, w, wl, states, xs, out, seed, stream, L, NI, mode, dev, pm)
 
     for st in states:
         lrs.lrs_state_free(st)
@@ -354,7 +383,9 @@ def run_gpu(args, w):
                      "frac": achieved / peak, "peak_kind": peak_kind + " (hbm_gbs, burst copy)",
                      "traffic": profiled_traffic(),
                      "algorithmic_bytes_per_launch": bytes_step,
-                     "kernel": "lrs::step_kernel<4,32,gated,per_key,%s>" % (
+                     "kernel": "lrs::step_kernel<C=%d,group=%d,%s,%s,%s>" % (
+                         w.d_v // 32, w.group, "delta" if w.update_kind else "gated",
+                         "per_key" if w.gate_kind else "scalar",
                          {0: "rtn", 1: "sr", 2: "bdr"}[mode])},
         "e2e": {"value": world * e2e_steps / (e2e_ms / 1e3), "unit": "steps/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
@@ -379,7 +410,7 @@ def _capture_on(stream, n, pick, lrs, out, seed, mode):
     return g
 
 
-def run_extras(args, w, wl, states, xs, out, seed, stream, L, NI, mode, dev):
+def run_extras(args, w, wl, states, xs, out, seed, stream, L, NI, mode, dev, pm):
     """Other rounding modes on the same state, and the fp32-state kernel on the
     same inputs (rank 0 only, not part of the headline number)."""
     import torch
@@ -403,7 +434,7 @@ def run_extras(args, w, wl, states, xs, out, seed, stream, L, NI, mode, dev):
         torch.cuda.synchronize()
         ms = e0.elapsed_time(e1) / n
         res["mode_" + name] = {"ms_per_step": ms, "steps_per_s": 1e3 / ms,
-                               "state_gbs": state_bytes(wl) / (ms / 1e3) / 1e9}
+                               "state_gbs": state_bytes(wl, pm) / (ms / 1e3) / 1e9}
         del g
     lrs.lrs_sync()
     # fp32 state kernel: 4 rotated fp32 states
@@ -448,7 +479,7 @@ def cpu_baseline(w, mode):
     tiles = np.sort(rng.choice(ntiles_all, size=n, replace=False))
     tb = (tiles // w.heads).astype(np.int32)
     th = (tiles % w.heads).astype(np.int32)
-    pm = I.uniform_prec_map(w).numpy()
+    pm = oracle_precision_map(w)
     S0 = I.initial_state(w)[tb, th].numpy()
     codes, scales = oracle.import_fp32(S0, pm, th, group=w.group)
     xs = []
@@ -481,6 +512,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--mode", default=None, choices=sorted(MODES))
     ap.add_argument("--layers", type=int, default=4)
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     args = ap.parse_args()
@@ -488,6 +520,8 @@ def main():
         ap.error("--warmup must be at least 3")
     from quantized_recurrent_state_decode_b200 import inputs as I
     w = I.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.with_batch(args.batch)
     if args.impl == "reference":
         if int(os.environ.get("RANK", "0")) != 0:
             return

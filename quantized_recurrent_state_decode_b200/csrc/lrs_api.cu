@@ -199,11 +199,12 @@ const void* find_step_kernel(int C, int group, int update_kind, int gate_kind, i
     }
 }
 
-int step_warp_smem(int C, int group, int gate_kind, int slots) {
-#define LRS_SLOT(CC, GG)                                                                 \
-    if (C == CC && group == GG)                                                          \
-        return gate_kind == kGatePerKey ? Slot<CC, GG, kGatePerKey>::warp_bytes(slots)   \
-                                        : Slot<CC, GG, kGate>::warp_bytes(slots);
+int step_warp_smem(int C, int group, int gate_kind, int slots, int mode) {
+    const bool xs = stage_x(mode);
+#define LRS_SLOT(CC, GG)                                                                    \
+    if (C == CC && group == GG)                                                             \
+        return gate_kind == kGatePerKey ? Slot<CC, GG, kGatePerKey>::warp_bytes(slots, xs)  \
+                                        : Slot<CC, GG, kGate>::warp_bytes(slots, xs);
     LRS_SLOT(4, 16)
     LRS_SLOT(4, 32)
     LRS_SLOT(2, 16)
@@ -353,7 +354,7 @@ lrs_status lrs_decode_step(const lrs_state* st, void* state_codes, float* scales
         slots = std::min(slots, G);
     }
     slots = std::max(1, std::min(slots, lrs::kMaxSlots));
-    const int warp_smem = lrs::step_warp_smem(C, sh.group, sh.gate_kind, slots);
+    const int warp_smem = lrs::step_warp_smem(C, sh.group, sh.gate_kind, slots, mode);
     constexpr int kSmemLimit = 227 * 1024;
     int warps = step_warps_override();
     if (warps <= 0) warps = kDefaultWarps;

@@ -16,8 +16,9 @@ const void* find_step_kernel_rtn(int C, int group, int update_kind, int gate_kin
 const void* find_step_kernel_sr(int C, int group, int update_kind, int gate_kind);
 const void* find_step_kernel_bdr(int C, int group, int update_kind, int gate_kind);
 
-// Bytes of shared memory one warp of the step kernel uses with `slots` ring slots.
-int step_warp_smem(int C, int group, int gate_kind, int slots);
+// Bytes of shared memory one warp of the step kernel uses with `slots` ring
+// slots in rounding mode `mode`.
+int step_warp_smem(int C, int group, int gate_kind, int slots, int mode);
 
 struct LayoutArgs {
     uint8_t* codes;

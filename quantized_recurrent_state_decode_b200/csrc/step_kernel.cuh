@@ -31,7 +31,7 @@ constexpr int kMaxSlots = 16;
 // Launch bound of a step variant in warps: 12 (at most 168 registers a thread)
 // where the live state fits, 8 (255 registers) for the wider groups and for
 // the rounding modes that carry more temporaries.
-constexpr int step_max_warps(int group, int mode) { return (mode != 0 || group > 32) ? 8 : 12; }
+__host__ __device__ constexpr int step_max_warps(int group, int mode) { return (mode != 0 || group > 32) ? 8 : 12; }
 constexpr float kTiny = 0x1p-100f;               // absmax below this: stored as zero
 
 struct StepParams {
@@ -73,8 +73,14 @@ struct Slot {
     static constexpr int kBytes = kG + (GATE == kGatePerKey ? GROUP * 4 : 0);
     static constexpr int kHeader = 128 + DV * 4;
     static_assert(kBytes % 16 == 0, "slot alignment");
-    static int warp_bytes(int slots) { return (kHeader + slots * kBytes + 127) / 128 * 128; }
+    static constexpr int kXsBytes = GROUP * 256;   // x staging (SR, BDR): 16 B per row pair and lane
+    static int warp_bytes(int slots, bool xs) {
+        return (kHeader + slots * kBytes + (xs ? kXsBytes : 0) + 127) / 128 * 128;
+    }
 };
+
+// Modes that stage the group's updated values in shared memory.
+__host__ __device__ constexpr bool stage_x(int mode) { return mode != 0; }
 
 // ------------------------------------------------------- packed fp32 math ---
 // Two consecutive key rows of one column go through the sm_100 two-wide fp32
@@ -446,6 +452,108 @@ struct TileCursor {
     }
 };
 
+// The same step for modes whose per-element rounding is long (SR, BDR): the
+// group's updated values are staged in the warp's shared-memory x buffer
+// instead of registers, so both phases are short loops over 16-byte units and
+// the kernel's code stays small enough for the instruction cache. xs holds
+// (x[r][c0], x[r+1][c0], x[r][c1], x[r+1][c1]) per row pair r and lane.
+template <int GROUP, int GATE, int MODE, int BITS>
+__device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int ubase, float2 sc,
+                                             const float* __restrict__ qs,
+                                             const float* __restrict__ ks,
+                                             const float* __restrict__ gs, float gscalar,
+                                             float2 w, float2& o, uint8_t* __restrict__ gcodes,
+                                             float* __restrict__ gscale, uint64_t hkey, int row0,
+                                             uint32_t j0, int lane, float4* __restrict__ xs) {
+    using G = PairGeo<GROUP, BITS>;
+    constexpr float QMAX = Q<BITS>::kMax, BIAS = Q<BITS>::kBias;
+    constexpr int RPUH = G::RPU / 2;              // row pairs per unit
+    const float2 s0 = f2(sc.x), s1 = f2(sc.y);
+    const float2 w0 = f2(w.x), w1 = f2(w.y);
+    const float2 gsc = f2(gscalar);
+    float a0 = 0.0f, b0 = 0.0f;
+
+#pragma unroll 1
+    for (int un = 0; un < G::UNITS; ++un) {
+        const uint4 raw = lds_unit(cs, ubase + un, lane);
+        const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+        float kk[G::RPU], qq[G::RPU], gg[G::RPU];
+        ld_smem_rows<G::RPU>(ks + un * G::RPU, kk);
+        ld_smem_rows<G::RPU>(qs + un * G::RPU, qq);
+        if constexpr (GATE == kGatePerKey) ld_smem_rows<G::RPU>(gs + un * G::RPU, gg);
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+            float f[G::EPW];
+            decode_word_biased<BITS>(wd[wi], f);
+#pragma unroll
+            for (int rp = 0; rp < G::RPW / 2; ++rp) {
+                const int rl = wi * G::RPW + 2 * rp;
+                const float2 kr = make_float2(kk[rl], kk[rl + 1]);
+                const float2 qr = make_float2(qq[rl], qq[rl + 1]);
+                const float2 gr = GATE == kGatePerKey ? make_float2(gg[rl], gg[rl + 1]) : gsc;
+                const float2 c0 = add2(make_float2(f[4 * rp], f[4 * rp + 2]), f2(-(kTwo23 + BIAS)));
+                const float2 c1 = add2(make_float2(f[4 * rp + 1], f[4 * rp + 3]), f2(-(kTwo23 + BIAS)));
+                const float2 x0 = fma2(gr, mul2(c0, s0), mul2(kr, w0));
+                const float2 x1 = fma2(gr, mul2(c1, s1), mul2(kr, w1));
+                o.x = __fmaf_rn(qr.x, x0.x, o.x);
+                o.x = __fmaf_rn(qr.y, x0.y, o.x);
+                o.y = __fmaf_rn(qr.x, x1.x, o.y);
+                o.y = __fmaf_rn(qr.y, x1.y, o.y);
+                a0 = max_abs3(a0, x0.x, x0.y);
+                b0 = max_abs3(b0, x1.x, x1.y);
+                xs[(un * RPUH + rl / 2) * 32 + lane] = make_float4(x0.x, x0.y, x1.x, x1.y);
+            }
+        }
+    }
+
+    float2 snew, inv;
+    constexpr int QM = static_cast<int>(QMAX);
+    snew.x = a0 < kTiny ? 0.0f : div_by_qmax<QM>(a0);
+    inv.x = a0 < kTiny ? 0.0f : div_rn_fast(QMAX, a0);
+    snew.y = b0 < kTiny ? 0.0f : div_by_qmax<QM>(b0);
+    inv.y = b0 < kTiny ? 0.0f : div_rn_fast(QMAX, b0);
+    st_cs_f2(gscale, snew);
+    const float2 inv0 = f2(inv.x), inv1 = f2(inv.y);
+    const float2 sn0 = f2(snew.x), sn1 = f2(snew.y);
+
+#pragma unroll 1
+    for (int un = 0; un < G::UNITS; ++un) {
+        uint32_t ow[4];
+        uint32_t wd[4] = {0u, 0u, 0u, 0u};
+        if constexpr (MODE == kBDR) {
+            const uint4 raw = lds_unit(cs, ubase + un, lane);
+            wd[0] = raw.x; wd[1] = raw.y; wd[2] = raw.z; wd[3] = raw.w;
+        }
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+            float f[G::EPW];
+            if constexpr (MODE == kBDR) decode_word_biased<BITS>(wd[wi], f);
+            float t[G::EPW];
+#pragma unroll
+            for (int rp = 0; rp < G::RPW / 2; ++rp) {
+                const int rl = wi * G::RPW + 2 * rp;
+                const float4 xv = xs[(un * RPUH + rl / 2) * 32 + lane];
+                float2 dq0 = f2(0.0f), dq1 = f2(0.0f);
+                if constexpr (MODE == kBDR) {
+                    dq0 = mul2(add2(make_float2(f[4 * rp], f[4 * rp + 2]), f2(-(kTwo23 + BIAS))), s0);
+                    dq1 = mul2(add2(make_float2(f[4 * rp + 1], f[4 * rp + 3]), f2(-(kTwo23 + BIAS))), s1);
+                }
+                const uint32_t i = static_cast<uint32_t>(row0 + un * G::RPU + rl);
+                const float2 t0 = round_rows<MODE, BITS>(make_float2(xv.x, xv.y), inv0, dq0, sn0,
+                                                         hkey, i, j0);
+                const float2 t1 = round_rows<MODE, BITS>(make_float2(xv.z, xv.w), inv1, dq1, sn1,
+                                                         hkey, i, j0 + 1);
+                t[4 * rp] = t0.x;
+                t[4 * rp + 2] = t0.y;
+                t[4 * rp + 1] = t1.x;
+                t[4 * rp + 3] = t1.y;
+            }
+            ow[wi] = encode_word<BITS>(t);
+        }
+        st_cs_u4(gcodes + ((ubase + un) * 32 + lane) * 16, ow[0], ow[1], ow[2], ow[3]);
+    }
+}
+
 // Fill `slot` with group g of the cursor's tile (lane 0 only). A tile whose
 // layout does not fit gets a bare arrival, so the slot's phase still completes.
 template <int C, int GROUP, int GATE>
@@ -507,6 +615,7 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(wsm);
     const float* v_s = reinterpret_cast<const float*>(wsm + 128);
     const int G = p.G, NS = p.slots;
+    float4* xs = reinterpret_cast<float4*>(wsm + S::kHeader + NS * S::kBytes);   // SR, BDR
     const int ntw = gw < p.ntiles ? (p.ntiles - gw + W - 1) / W : 0;   // this warp's tiles
     const int64_t K = static_cast<int64_t>(ntw) * G;                    // this warp's items
 
@@ -561,23 +670,15 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
                                                           static_cast<uint32_t>(ti.h))
                                           : 0ull;
 
-        // the delta rule needs every group of the tile before its first one
-        {
-            Ring look = ic;
-            const int first = UPD == kDelta ? G : 1;
-            for (int g = 0; g < first && ok; ++g) {
-                ok = __all_sync(0xffffffffu,
-                                mbar_wait_bounded(&bars[look.slot], look.par, p.timeout_ns));
-                look.advance(NS);
-            }
-        }
+        // the tile's first group
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[ic.slot], ic.par, p.timeout_ns));
         if (!ok) break;
 
         if (ti.prec == 0) {
             // no copies were made for this tile: record the mismatch and skip it
             if (lane == 0) atomicOr(p.err, kErrLayout);
             for (int g = 0; g < G; ++g) {
-                if (UPD != kDelta && g > 0) {
+                if (g > 0) {
                     ok = __all_sync(0xffffffffu,
                                     mbar_wait_bounded(&bars[ic.slot], ic.par, p.timeout_ns));
                     if (!ok) break;
@@ -597,19 +698,32 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
             float2 u[P];
 #pragma unroll
             for (int pc = 0; pc < P; ++pc) u[pc] = f2(0.0f);
+            // the first pass takes the groups as they arrive (the ring holds
+            // the whole tile), the second pass finds them all resident
             Ring r = ic;
-            for (int g = 0; g < G; ++g) {
+            for (int g = 0; g < G && ok; ++g) {
+                if (g > 0)
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait_bounded(&bars[r.slot], r.par, p.timeout_ns));
+                if (!ok) break;
                 const uint8_t* sm = wsm + S::kHeader + r.slot * S::kBytes;
                 const float* ss = reinterpret_cast<const float*>(sm + S::kScales) + lane * C;
                 const float* ks = reinterpret_cast<const float*>(sm + S::kK);
-#pragma unroll
+                float2 up = u[0], uq = u[P - 1];
+#pragma unroll 1
                 for (int pc = 0; pc < P; ++pc) {
                     const float2 sc = *reinterpret_cast<const float2*>(ss + 2 * pc);
                     if (ti.prec == 8)
-                        pair_ktS<GROUP, 8>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, ks, lane, u[pc]);
+                        pair_ktS<GROUP, 8>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, ks, lane, up);
                     else
-                        pair_ktS<GROUP, 4>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, ks, lane, u[pc]);
+                        pair_ktS<GROUP, 4>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, ks, lane, up);
+                    if constexpr (P == 2) {
+                        const float2 t = up;
+                        up = uq; uq = t;
+                    }
                 }
+                u[0] = up;
+                u[P - 1] = P == 2 ? uq : up;
                 r.advance(NS);
             }
 #pragma unroll
@@ -626,6 +740,7 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
                 w[pc] = *reinterpret_cast<const float2*>(v_s + lane * C + 2 * pc);
         }
 
+        if (!ok) break;
         uint8_t* gcodes_tile = p.codes + ti.code_off;
         const uint32_t cbytes = GROUP * DV * ti.prec / 8;
         for (int g = 0; g < G; ++g) {
@@ -641,19 +756,41 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
             const float* gs = reinterpret_cast<const float*>(sm + S::kG);
             float* gscale = p.scales + (static_cast<int64_t>(tile) * G + g) * DV + lane * C;
             uint8_t* gcodes = gcodes_tile + static_cast<int64_t>(g) * cbytes;
-#pragma unroll
+            // The column pairs run one after the other through one copy of the
+            // (large) pair code; the pairs' w and o rotate through (wp, op).
+            float2 wp = w[0], op = o[0], wq = w[P - 1], oq = o[P - 1];
+#pragma unroll 1
             for (int pc = 0; pc < P; ++pc) {
                 const float2 sc = *reinterpret_cast<const float2*>(ss + 2 * pc);
                 const uint32_t j0 = static_cast<uint32_t>(lane * C + 2 * pc);
-                if (ti.prec == 8)
-                    pair_step<GROUP, GATE, MODE, 8>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs, ks,
-                                                    gs, gscalar, w[pc], o[pc], gcodes,
-                                                    gscale + 2 * pc, hkey, g * GROUP, j0, lane);
-                else
-                    pair_step<GROUP, GATE, MODE, 4>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs, ks,
-                                                    gs, gscalar, w[pc], o[pc], gcodes,
-                                                    gscale + 2 * pc, hkey, g * GROUP, j0, lane);
+                if constexpr (stage_x(MODE)) {
+                    if (ti.prec == 8)
+                        pair_step_xs<GROUP, GATE, MODE, 8>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs,
+                                                           ks, gs, gscalar, wp, op, gcodes,
+                                                           gscale + 2 * pc, hkey, g * GROUP, j0,
+                                                           lane, xs);
+                    else
+                        pair_step_xs<GROUP, GATE, MODE, 4>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs,
+                                                           ks, gs, gscalar, wp, op, gcodes,
+                                                           gscale + 2 * pc, hkey, g * GROUP, j0,
+                                                           lane, xs);
+                } else {
+                    if (ti.prec == 8)
+                        pair_step<GROUP, GATE, MODE, 8>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs, ks,
+                                                        gs, gscalar, wp, op, gcodes,
+                                                        gscale + 2 * pc, hkey, g * GROUP, j0, lane);
+                    else
+                        pair_step<GROUP, GATE, MODE, 4>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs, ks,
+                                                        gs, gscalar, wp, op, gcodes,
+                                                        gscale + 2 * pc, hkey, g * GROUP, j0, lane);
+                }
+                if constexpr (P == 2) {
+                    const float2 tw = wp, to = op;
+                    wp = wq; op = oq; wq = tw; oq = to;
+                }
             }
+            o[0] = op;
+            o[P - 1] = P == 2 ? oq : op;
             ++kc;
             ic.advance(NS);
             __syncwarp();
