@@ -49,7 +49,8 @@ __device__ void encode_pair_rtn(const float2 (&x)[GROUP], float2 inv, uint8_t* g
 #pragma unroll
             for (int e = 0; e < G::EPW; e += 2) {
                 const int r = un * G::RPU + (wi * G::EPW + e) / 2;
-                const float2 tv = round_rows<kRTN, BITS>(x[r], inv, f2(0.f), f2(0.f), 0ull, 0u, 0u);
+                const float2 kb = make_float2(word_bias<BITS>(e), word_bias<BITS>(e + 1));
+                const float2 tv = round_rows<kRTN, BITS>(x[r], inv, f2(0.f), f2(0.f), kb, 0ull, 0u, 0u);
                 t[e] = tv.x;
                 t[e + 1] = tv.y;
             }

@@ -147,27 +147,45 @@ __device__ __forceinline__ void decode_word_biased(uint32_t w, float (&f)[32 / B
     }
 }
 
-// Pack the stored bytes (nibbles) of 4 (8) rounded codes into one word. The
-// bit pattern of each rounded value t is K + u, K = bits(1.5 * 2^23), u the
-// stored byte (nibble), so the word is sum(bits(t_n) << shift_n) minus
-// K * sum(1 << shift_n), all modulo 2^32: integer multiply-adds, which run on
-// the fused-multiply-add pipe beside the byte permutes of the decode.
+// Rounded codes leave the rounding as floats 2^23 + B_n + code, whose bit
+// patterns are 0x4B000000 + B_n + code (B_n + code in [1, 2^23)), with the
+// stored byte (nibble) in the low bits. word_bias<BITS>(n) is 2^23 + B_n for
+// element n of a 32-bit word. Packing (encode_word) adds the patterns
+// shifted to their positions modulo 2^32; only the unshifted pattern (and,
+// for int4, the one shifted by 4) keeps any of 0x4B000000. B_n is the
+// offset-binary bias (128, 8) except at two positions whose extra amounts
+// cancel those leftovers: int8 elements 2 and 3 take 384 and 308 (adding
+// 1 and 180 to the top byte: 0x4B + 1 + 180 = 256), int4 elements 6 and 3
+// (nibbles 5 and 6) take 24 and 12 (adding 1 and 4 to nibble 6, against
+// 0x4B + 0xB0 from the two low patterns). Every B_n is even, so rounding
+// 2^23 + B_n + y to nearest-even breaks a tie of y the same way as rint.
+template <int BITS>
+__host__ __device__ constexpr float word_bias(int n) {
+    if constexpr (BITS == 8) {
+        return kTwo23 + (n == 2 ? 384.0f : n == 3 ? 308.0f : 128.0f);
+    } else {
+        return kTwo23 + (n == 3 ? 12.0f : n == 6 ? 24.0f : 8.0f);
+    }
+}
+
+// Pack the stored bytes (nibbles) of 4 (8) rounded codes into one word with
+// integer multiply-adds on their bit patterns, modulo 2^32: a pattern
+// shifted left by 8 (4) bits or more keeps only its low bits, and the high
+// bits that remain cancel by the choice of word_bias (see above). The
+// multiply-adds run on the fused-multiply-add pipe beside the byte permutes
+// of the decode.
 template <int BITS>
 __device__ __forceinline__ uint32_t encode_word(const float (&t)[32 / BITS]) {
-    constexpr uint32_t K = 0x4B400000u;
     uint32_t r;
     if constexpr (BITS == 8) {
-        constexpr uint32_t KS = K * 0x01010101u;
         asm("{\n\t.reg .u32 a;\n\t"
             "mad.lo.u32 a, %2, 256, %1;\n\t"
             "mad.lo.u32 a, %3, 65536, a;\n\t"
-            "mad.lo.u32 a, %4, 16777216, a;\n\t"
-            "sub.u32 %0, a, %5;\n\t}"
+            "mad.lo.u32 %0, %4, 16777216, a;\n\t}"
             : "=r"(r)
             : "r"(__float_as_uint(t[0])), "r"(__float_as_uint(t[1])), "r"(__float_as_uint(t[2])),
-              "r"(__float_as_uint(t[3])), "r"(KS));
+              "r"(__float_as_uint(t[3])));
     } else {
-        constexpr uint32_t KS = K * 0x11111111u;
         asm("{\n\t.reg .u32 a;\n\t"
             "mad.lo.u32 a, %2, 16, %1;\n\t"
             "mad.lo.u32 a, %3, 256, a;\n\t"
@@ -175,12 +193,11 @@ __device__ __forceinline__ uint32_t encode_word(const float (&t)[32 / BITS]) {
             "mad.lo.u32 a, %5, 65536, a;\n\t"
             "mad.lo.u32 a, %6, 1048576, a;\n\t"
             "mad.lo.u32 a, %7, 16777216, a;\n\t"
-            "mad.lo.u32 a, %8, 268435456, a;\n\t"
-            "sub.u32 %0, a, %9;\n\t}"
+            "mad.lo.u32 %0, %8, 268435456, a;\n\t}"
             : "=r"(r)
             : "r"(__float_as_uint(t[0])), "r"(__float_as_uint(t[4])), "r"(__float_as_uint(t[1])),
               "r"(__float_as_uint(t[5])), "r"(__float_as_uint(t[2])), "r"(__float_as_uint(t[6])),
-              "r"(__float_as_uint(t[3])), "r"(__float_as_uint(t[7])), "r"(KS));
+              "r"(__float_as_uint(t[3])), "r"(__float_as_uint(t[7])));
     }
     return r;
 }
@@ -189,18 +206,46 @@ template <int BITS> struct Q;
 template <> struct Q<8> { static constexpr float kMax = 127.0f, kBias = 128.0f; };
 template <> struct Q<4> { static constexpr float kMax = 7.0f, kBias = 8.0f; };
 
+// New scales and their inverses for two columns of one group, from their
+// absmax A: s' = RN(A/qmax), inv = RN(qmax/A), both 0 where A is below kTiny.
+// The same remainder-corrected divisions as div_by_qmax and div_rn_fast
+// (lrs_device.cuh), each step done for both columns in one two-wide
+// instruction; above 2^100 the inverse falls back to IEEE division.
+template <int BITS>
+__device__ __forceinline__ void new_scales(float A0, float A1, float2& snew, float2& inv) {
+    constexpr float QMAX = Q<BITS>::kMax;
+    constexpr float Y = 1.0f / QMAX;                 // RN(1/qmax)
+    const float2 A = make_float2(A0, A1);
+    const float2 nA = neg2(A);
+    // s' = A/qmax with the constant reciprocal
+    const float2 q0 = mul2(A, f2(Y));
+    const float2 s = fma2(fma2(q0, f2(-QMAX), A), f2(Y), q0);
+    // inv = qmax/A with the refined hardware reciprocal
+    float2 y0;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y0.x) : "f"(A0));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y0.y) : "f"(A1));
+    const float2 y = fma2(fma2(nA, y0, f2(1.0f)), y0, y0);
+    const float2 p0 = mul2(f2(QMAX), y);
+    float2 iv = fma2(fma2(p0, nA, f2(QMAX)), y, p0);
+    if (A0 > 0x1p100f) iv.x = __fdiv_rn(QMAX, A0);
+    if (A1 > 0x1p100f) iv.y = __fdiv_rn(QMAX, A1);
+    snew = make_float2(A0 < kTiny ? 0.0f : s.x, A1 < kTiny ? 0.0f : s.y);
+    inv = make_float2(A0 < kTiny ? 0.0f : iv.x, A1 < kTiny ? 0.0f : iv.y);
+}
+
 // Codes of two elements (key rows i, i+1 of value column j), returned as the
-// floats 1.5*2^23 + bias + code whose low byte is the stored byte. inv,
-// s_new: the column's values in both halves. The value rounded is the exact
-// product x*inv: one fused multiply-add rounds it straight to an integer.
+// floats kb + code (kb: word_bias of the two elements' word positions) whose
+// low bits are the stored byte (nibble). inv, s_new: the column's values in
+// both halves. The value rounded is the exact product x*inv: one fused
+// multiply-add rounds it straight to an integer.
 template <int MODE, int BITS>
 __device__ __forceinline__ float2 round_rows(float2 x, float2 inv, float2 deq, float2 s_new,
-                                             uint64_t hkey, uint32_t i, uint32_t j) {
-    constexpr float QMAX = Q<BITS>::kMax, BIAS = Q<BITS>::kBias;
+                                             float2 kb, uint64_t hkey, uint32_t i, uint32_t j) {
+    constexpr float QMAX = Q<BITS>::kMax;
     if constexpr (MODE == kRTN) {
         // |x*inv| <= qmax (1 + 2^-24) since inv = RN(qmax/A) and |x| <= A:
         // the nearest integer never leaves [-qmax, qmax], no clamp needed.
-        return fma2(x, inv, f2(kRound + BIAS));
+        return fma2(x, inv, kb);
     } else {
         const float2 n = add2(fma2(x, inv, f2(kRound)), f2(-kRound));  // nearest integer
         const float2 d = fma2(x, inv, neg2(n));                          // sign of x*inv - n
@@ -232,7 +277,7 @@ __device__ __forceinline__ float2 round_rows(float2 x, float2 inv, float2 deq, f
         }
         c.x = fminf(fmaxf(c.x, -QMAX), QMAX);
         c.y = fminf(fmaxf(c.y, -QMAX), QMAX);
-        return add2(c, f2(kRound + BIAS));
+        return add2(c, kb);
     }
 }
 
@@ -322,7 +367,7 @@ __device__ __forceinline__ void pair_step(const uint8_t* __restrict__ cs, int ub
                                           float* __restrict__ gscale, uint64_t hkey, int row0,
                                           uint32_t j0, int lane) {
     using G = PairGeo<GROUP, BITS>;
-    constexpr float QMAX = Q<BITS>::kMax, BIAS = Q<BITS>::kBias;
+    constexpr float BIAS = Q<BITS>::kBias;
     const float2 s0 = f2(sc.x), s1 = f2(sc.y);     // per-column constants as pairs
     const float2 w0 = f2(w.x), w1 = f2(w.y);
     const float2 gsc = f2(gscalar);
@@ -372,11 +417,7 @@ __device__ __forceinline__ void pair_step(const uint8_t* __restrict__ cs, int ub
     }
     const float A0 = fmaxf(a0, a1), A1 = fmaxf(b0, b1);
     float2 snew, inv;
-    constexpr int QM = static_cast<int>(QMAX);
-    snew.x = A0 < kTiny ? 0.0f : div_by_qmax<QM>(A0);
-    inv.x = A0 < kTiny ? 0.0f : div_rn_fast(QMAX, A0);
-    snew.y = A1 < kTiny ? 0.0f : div_by_qmax<QM>(A1);
-    inv.y = A1 < kTiny ? 0.0f : div_rn_fast(QMAX, A1);
+    new_scales<BITS>(A0, A1, snew, inv);
     st_cs_f2(gscale, snew);
     const float2 inv0 = f2(inv.x), inv1 = f2(inv.y);
     const float2 sn0 = f2(snew.x), sn1 = f2(snew.y);
@@ -403,8 +444,11 @@ __device__ __forceinline__ void pair_step(const uint8_t* __restrict__ cs, int ub
                     dq1 = mul2(add2(make_float2(f[4 * rp + 1], f[4 * rp + 3]), f2(-(kTwo23 + BIAS))), s1);
                 }
                 const uint32_t i = static_cast<uint32_t>(row0 + r);
-                const float2 t0 = round_rows<MODE, BITS>(x[r / 2][0], inv0, dq0, sn0, hkey, i, j0);
-                const float2 t1 = round_rows<MODE, BITS>(x[r / 2][1], inv1, dq1, sn1, hkey, i, j0 + 1);
+                const float2 kb0 = make_float2(word_bias<BITS>(4 * rp), word_bias<BITS>(4 * rp + 2));
+                const float2 kb1 = make_float2(word_bias<BITS>(4 * rp + 1), word_bias<BITS>(4 * rp + 3));
+                const float2 t0 = round_rows<MODE, BITS>(x[r / 2][0], inv0, dq0, sn0, kb0, hkey, i, j0);
+                const float2 t1 = round_rows<MODE, BITS>(x[r / 2][1], inv1, dq1, sn1, kb1, hkey, i,
+                                                         j0 + 1);
                 t[4 * rp] = t0.x;
                 t[4 * rp + 2] = t0.y;
                 t[4 * rp + 1] = t1.x;
@@ -466,7 +510,7 @@ __device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int
                                              float* __restrict__ gscale, uint64_t hkey, int row0,
                                              uint32_t j0, int lane, float4* __restrict__ xs) {
     using G = PairGeo<GROUP, BITS>;
-    constexpr float QMAX = Q<BITS>::kMax, BIAS = Q<BITS>::kBias;
+    constexpr float BIAS = Q<BITS>::kBias;
     constexpr int RPUH = G::RPU / 2;              // row pairs per unit
     const float2 s0 = f2(sc.x), s1 = f2(sc.y);
     const float2 w0 = f2(w.x), w1 = f2(w.y);
@@ -507,11 +551,7 @@ __device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int
     }
 
     float2 snew, inv;
-    constexpr int QM = static_cast<int>(QMAX);
-    snew.x = a0 < kTiny ? 0.0f : div_by_qmax<QM>(a0);
-    inv.x = a0 < kTiny ? 0.0f : div_rn_fast(QMAX, a0);
-    snew.y = b0 < kTiny ? 0.0f : div_by_qmax<QM>(b0);
-    inv.y = b0 < kTiny ? 0.0f : div_rn_fast(QMAX, b0);
+    new_scales<BITS>(a0, b0, snew, inv);
     st_cs_f2(gscale, snew);
     const float2 inv0 = f2(inv.x), inv1 = f2(inv.y);
     const float2 sn0 = f2(snew.x), sn1 = f2(snew.y);
@@ -539,10 +579,12 @@ __device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int
                     dq1 = mul2(add2(make_float2(f[4 * rp + 1], f[4 * rp + 3]), f2(-(kTwo23 + BIAS))), s1);
                 }
                 const uint32_t i = static_cast<uint32_t>(row0 + un * G::RPU + rl);
+                const float2 kb0 = make_float2(word_bias<BITS>(4 * rp), word_bias<BITS>(4 * rp + 2));
+                const float2 kb1 = make_float2(word_bias<BITS>(4 * rp + 1), word_bias<BITS>(4 * rp + 3));
                 const float2 t0 = round_rows<MODE, BITS>(make_float2(xv.x, xv.y), inv0, dq0, sn0,
-                                                         hkey, i, j0);
+                                                         kb0, hkey, i, j0);
                 const float2 t1 = round_rows<MODE, BITS>(make_float2(xv.z, xv.w), inv1, dq1, sn1,
-                                                         hkey, i, j0 + 1);
+                                                         kb1, hkey, i, j0 + 1);
                 t[4 * rp] = t0.x;
                 t[4 * rp + 2] = t0.y;
                 t[4 * rp + 1] = t1.x;
