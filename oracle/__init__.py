@@ -37,6 +37,13 @@ def lib():
         L.orc_step.argtypes = [i32, P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P,
                                P, u64, u64, i32]
         L.orc_step.restype = i32
+        L.orc_chunk_step.argtypes = [i32, P, P, i32, i32, i32, i32, i32, i32, P, P, P, i32, P, P,
+                                     P, P, P, P, u64, u64, i32]
+        L.orc_chunk_step.restype = i32
+        L.orc_bf16_rne.argtypes = [ctypes.c_float]
+        L.orc_bf16_rne.restype = ctypes.c_uint16
+        L.orc_bf16_rne_array.argtypes = [i64, P, P]
+        L.orc_bf16_rne_array.restype = None
         L.orc_fp32_step.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P, P, i32]
         L.orc_fp32_step.restype = i32
         L.orc_import.argtypes = [i32, P, i32, i32, i32, P, P, P, P]
@@ -99,6 +106,45 @@ def step(codes, scales, q, k, v, gates, beta, prec_map, tile_b, tile_h, *, group
     if rc != 0:
         raise ValueError("orc_step rejected its arguments (%d)" % rc)
     return out
+
+
+def chunk_step(codes, scales, q, k, v, gates, beta, prec_map, tile_b, tile_h, *, group,
+               update_kind, gate_kind, mode, seed=0, step=0, nthreads=1):
+    """T tokens per tile applied to the fp32 state, one requantization at the end.
+
+    q, k [T][n][d_k]; v [T][n][d_v]; gates [T][n][d_k] or [T][n]; beta [T][n]
+    or None; codes/scales as in step(), updated in place. Returns out f32
+    [T][n][d_v].
+    """
+    n, d_k, d_v = codes.shape
+    assert codes.dtype == np.int8 and scales.dtype == np.float32
+    q, k, v, gates, beta = map(_f32, (q, k, v, gates, beta))
+    T = q.shape[0]
+    assert q.shape == (T, n, d_k) and k.shape == (T, n, d_k) and v.shape == (T, n, d_v)
+    prec_map = np.ascontiguousarray(prec_map, dtype=np.uint8)
+    tile_b = np.ascontiguousarray(tile_b, dtype=np.int32)
+    tile_h = np.ascontiguousarray(tile_h, dtype=np.int32)
+    out = np.zeros((T, n, d_v), np.float32)
+    rc = lib().orc_chunk_step(n, _p(tile_b), _p(tile_h), d_k, d_v, group, update_kind,
+                              gate_kind, mode, _p(prec_map), _p(codes), _p(scales), T, _p(q),
+                              _p(k), _p(v), _p(gates), _p(beta), _p(out), seed, step, nthreads)
+    if rc != 0:
+        raise ValueError("orc_chunk_step rejected its arguments (%d)" % rc)
+    return out
+
+
+def bf16_rne(x):
+    """float32 array -> uint16 bfloat16 patterns, nearest with ties to even."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.zeros(x.shape, np.uint16)
+    lib().orc_bf16_rne_array(x.size, _p(x), _p(out))
+    return out
+
+
+def bf16_to_f32(u):
+    """uint16 bfloat16 patterns -> the float32 values they denote (exact)."""
+    u = np.ascontiguousarray(u, dtype=np.uint16)
+    return (u.astype(np.uint32) << 16).view(np.float32)
 
 
 def fp32_step(S, q, k, v, gates, beta, *, update_kind, gate_kind, nthreads=1):

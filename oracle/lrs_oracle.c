@@ -186,6 +186,7 @@ static int qmax_of(uint8_t bits)
 
 typedef struct {
     int ntiles, d_k, d_v, group, update_kind, gate_kind, mode, nthreads, tid;
+    int T; /* tokens per call (chunked update); 1 for a decode step */
     const int32_t *tile_b, *tile_h;
     const uint8_t *prec_map;
     int8_t *codes;
@@ -209,6 +210,37 @@ static void *worker(void *arg)
         return (void *)1;
     }
     size_t gate_len = (W->gate_kind == ORC_GATE_PER_KEY) ? (size_t)d_k : 1;
+    if (W->T > 1) {
+        float *cur = (float *)malloc(n * sizeof(float));
+        if (!cur) {
+            free(deq); free(x); free(w);
+            return (void *)1;
+        }
+        size_t NT = (size_t)W->ntiles;
+        for (int t = W->tid; t < W->ntiles; t += W->nthreads) {
+            int8_t *c = W->codes + (size_t)t * n;
+            float *s = W->scales + (size_t)t * G * d_v;
+            int qmax = qmax_of(W->prec_map[W->tile_h[t]]);
+            for (int i = 0; i < d_k; ++i)
+                for (int j = 0; j < d_v; ++j)
+                    deq[i * d_v + j] = (float)c[i * d_v + j] * s[(i / W->group) * d_v + j];
+            memcpy(cur, deq, n * sizeof(float));
+            /* the tokens in order, each an update of the fp32 state and its output */
+            for (int tok = 0; tok < W->T; ++tok) {
+                size_t row = (size_t)tok * NT + (size_t)t;
+                update_tile(d_k, d_v, W->update_kind, W->gate_kind, cur, W->q + row * d_k,
+                            W->k + row * d_k, W->v + row * d_v, W->gates + row * gate_len,
+                            W->beta ? W->beta[row] : 0.0f, w, x, W->out + row * d_v);
+                memcpy(cur, x, n * sizeof(float));
+            }
+            /* one requantization at the chunk's end; BDR compares with the
+             * state at the chunk's start */
+            requantize_tile(d_k, d_v, W->group, qmax, W->mode, cur, deq, c, s, W->seed, W->step,
+                            (uint32_t)W->tile_b[t], (uint32_t)W->tile_h[t]);
+        }
+        free(cur); free(deq); free(x); free(w);
+        return NULL;
+    }
     for (int t = W->tid; t < W->ntiles; t += W->nthreads) {
         const float *q = W->q + (size_t)t * d_k;
         const float *k = W->k + (size_t)t * d_k;
@@ -295,6 +327,63 @@ int orc_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int d_k, 
     W.q = q; W.k = k; W.v = v; W.gates = gates; W.beta = beta; W.out = out;
     W.seed = seed; W.step = step; W.quantized = 1;
     return run_tiles(&W, nthreads);
+}
+
+int orc_chunk_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int d_k, int d_v,
+                   int group, int update_kind, int gate_kind, int mode, const uint8_t *prec_map,
+                   int8_t *codes, float *scales, int T, const float *q, const float *k,
+                   const float *v, const float *gates, const float *beta, float *out,
+                   uint64_t seed, uint64_t step, int nthreads)
+{
+    if (T < 1) return -1;
+    if (T == 1)
+        return orc_step(ntiles, tile_b, tile_h, d_k, d_v, group, update_kind, gate_kind, mode,
+                        prec_map, codes, scales, q, k, v, gates, beta, out, seed, step, nthreads);
+    if (ntiles < 0 || check_shape(d_k, d_v, group, update_kind, gate_kind) != 0) return -1;
+    if (mode != ORC_ROUND_RTN && mode != ORC_ROUND_SR && mode != ORC_ROUND_BDR) return -1;
+    if (ntiles == 0) return 0;
+    if (!tile_b || !tile_h || !prec_map || !codes || !scales || !q || !k || !v || !gates || !out)
+        return -1;
+    if (update_kind == ORC_UPDATE_DELTA && !beta) return -1;
+    for (int t = 0; t < ntiles; ++t)
+        if (tile_h[t] < 0 || qmax_of(prec_map[tile_h[t]]) < 0) return -1;
+    work_t W;
+    memset(&W, 0, sizeof W);
+    W.ntiles = ntiles; W.d_k = d_k; W.d_v = d_v; W.group = group;
+    W.update_kind = update_kind; W.gate_kind = gate_kind; W.mode = mode; W.T = T;
+    W.tile_b = tile_b; W.tile_h = tile_h; W.prec_map = prec_map;
+    W.codes = codes; W.scales = scales;
+    W.q = q; W.k = k; W.v = v; W.gates = gates; W.beta = beta; W.out = out;
+    W.seed = seed; W.step = step; W.quantized = 1;
+    return run_tiles(&W, nthreads);
+}
+
+uint16_t orc_bf16_rne(float x)
+{
+    uint32_t u;
+    memcpy(&u, &x, sizeof u);
+    uint32_t sign = u & 0x80000000u;
+    if (isnan(x)) return (uint16_t)((sign >> 16) | 0x7FC0u);
+    /* |x| lies between the bfloat16 values with patterns lo (the upper half
+     * of x's pattern, i.e. x truncated toward zero) and lo + 1 (the next one
+     * away from zero; past the largest finite value that is infinity). The
+     * dropped half of the pattern says where: below 0x8000 nearer lo, above
+     * nearer lo + 1, equal a tie, which goes to the even pattern. */
+    uint32_t lo = u >> 16;
+    uint32_t rest = u & 0xFFFFu;
+    uint32_t r;
+    if (rest < 0x8000u)
+        r = lo;
+    else if (rest > 0x8000u)
+        r = lo + 1;
+    else
+        r = (lo & 1u) ? lo + 1 : lo;
+    return (uint16_t)r;
+}
+
+void orc_bf16_rne_array(int64_t n, const float *x, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_bf16_rne(x[i]);
 }
 
 int orc_fp32_step(int ntiles, int d_k, int d_v, int update_kind, int gate_kind, float *S,

@@ -84,6 +84,24 @@ void orc_decay_means(int64_t outer, int heads, int64_t inner, const float *decay
  * lower head index) get 8-bit codes, the rest 4-bit. */
 int orc_precision_map(int heads, const double *means, int n_int8, uint8_t *prec_map);
 
+/* Multi-token (chunked) update: the T tokens of each tile are applied one
+ * after the other to the fp32 state, starting from the dequantized state, with
+ * one output per token; the state is requantized once, after the last token.
+ * Token t's inputs are those of a decode step, stacked on a leading token axis:
+ * q, k [T][ntiles][d_k]; v, out [T][ntiles][d_v]; gates [T][ntiles][d_k] or
+ * [T][ntiles]; beta [T][ntiles]. With T = 1 this is orc_step. */
+int orc_chunk_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h,
+                   int d_k, int d_v, int group, int update_kind, int gate_kind, int mode,
+                   const uint8_t *prec_map, int8_t *codes, float *scales, int T,
+                   const float *q, const float *k, const float *v, const float *gates,
+                   const float *beta, float *out, uint64_t seed, uint64_t step, int nthreads);
+
+/* bfloat16 (the upper half of binary32: sign, 8 exponent bits, 7 fraction
+ * bits) nearest to x, ties to the even fraction; NaN becomes a quiet NaN of the
+ * same sign. Returns the 16-bit pattern. */
+uint16_t orc_bf16_rne(float x);
+void orc_bf16_rne_array(int64_t n, const float *x, uint16_t *out);
+
 #ifdef __cplusplus
 }
 #endif
