@@ -437,6 +437,39 @@ def run_extras(args, w, wl, states, xs, out, seed, stream, L, NI, mode, dev, pm)
                                "state_gbs": state_bytes(wl, pm) / (ms / 1e3) / 1e9}
         del g
     lrs.lrs_sync()
+    # the same step with bfloat16 q, k, v and out
+    xb = [{k: (v.to(torch.bfloat16) if k in ("q", "k", "v") else v) for k, v in x.items()}
+          for x in xs]
+    outb = torch.empty(out.shape, dtype=torch.bfloat16, device=dev)
+
+    def step_bf16(i):
+        st, x = states[i % L], xb[i % NI]
+        lrs.lrs_decode_step_bf16(st, st.state_codes, st.scales, st.prec_map, x["q"], x["k"],
+                                 x["v"], x["gates"], x["beta"], outb, seed, i, mode, stream)
+    for i in range(8):
+        step_bf16(i)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            step_bf16(i)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    io_f32 = sum(v.numel() * 4 for v in xs[0].values() if v is not None) + out.numel() * 4
+    io_b = sum(v.numel() * v.element_size() for v in xb[0].values() if v is not None) + \
+        outb.numel() * 2
+    res["io_bf16"] = {"ms_per_step": ms, "steps_per_s": 1e3 / ms,
+                      "state_gbs": state_bytes(wl, pm) / (ms / 1e3) / 1e9,
+                      "io_bytes_per_step": io_b, "io_bytes_per_step_f32": io_f32,
+                      "api": "lrs_decode_step_bf16"}
+    del g
+    lrs.lrs_sync()
+    res["chunk"] = run_chunk_extra(w, wl, states, seed, stream, L, mode, dev, pm)
     # fp32 state kernel: 4 rotated fp32 states
     shp = lrs.shape(wl.batch, w.heads, w.d_k, w.d_v, w.group, w.update_kind, w.gate_kind)
     Ls = 4
@@ -465,6 +498,70 @@ def run_extras(args, w, wl, states, xs, out, seed, stream, L, NI, mode, dev, pm)
                                 "state_gbs": fb / (ms / 1e3) / 1e9, "bytes_per_step": fb}
     del g, Ss
     return res
+
+
+FP32_LANES_PER_SM = 128      # fp32 fused multiply-add lanes per SM (sm_100)
+
+
+def run_chunk_extra(w, wl, states, seed, stream, L, mode, dev, pm, T=16, n=32):
+    """The multi-token update (T tokens per tile, one requantization) on the
+    same states: time per chunk, and its fp32 arithmetic against the fp32 FMA
+    peak at the SM clock limit (the chunk is bound by arithmetic, not HBM)."""
+    import torch
+    from quantized_recurrent_state_decode_b200 import inputs as I
+    from quantized_recurrent_state_decode_b200 import lrs
+    if w.d_k not in (64, 128) or w.d_v not in (64, 128):
+        return None
+    xc = I.chunk_inputs(wl, 0, T, device=dev)
+    out = torch.empty(T, wl.batch, w.heads, w.d_v, device=dev)
+
+    def launch(i):
+        st = states[i % L]
+        lrs.lrs_chunk_step(st, st.state_codes, st.scales, st.prec_map, T, xc["q"], xc["k"],
+                           xc["v"], xc["gates"], xc["beta"], out, seed, i, mode, stream)
+    for i in range(4):
+        launch(i)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            launch(i)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    del g
+    lrs.lrs_sync()
+    elems = wl.batch * w.heads * w.d_k * w.d_v
+    flops_el = 7 if w.update_kind == 1 else 5       # k*w, g*x + kw, q*x (+ k*x for u)
+    flops = elems * T * flops_el
+    props = torch.cuda.get_device_properties(dev)
+    clk = _sm_max_mhz()
+    peak = props.multi_processor_count * FP32_LANES_PER_SM * 2 * clk * 1e6 / 1e12 if clk else None
+    achieved = flops / (ms / 1e3) / 1e12
+    io = sum(v.numel() * 4 for v in xc.values() if v is not None) + out.numel() * 4
+    return {"tokens_per_chunk": T, "ms_per_chunk": ms,
+            "tile_tokens_per_s": wl.batch * w.heads * T / (ms / 1e3),
+            "api": "lrs_chunk_step",
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak if peak else None,
+                         "peak_kind": "fp32 FMA lanes x 2 x SMs x max SM clock (%s MHz)" % clk,
+                         "flops_per_element_token": flops_el},
+            "state_bytes": state_bytes(wl, pm),
+            "io_bytes_per_chunk": io}
+
+
+def _sm_max_mhz():
+    try:
+        out = subprocess.run(["nvidia-smi", "--query-gpu=clocks.max.sm", "--format=csv,noheader,"
+                              "nounits", "-i", os.environ.get("LOCAL_RANK", "0")],
+                             capture_output=True, text=True, timeout=20).stdout
+        return float(out.strip().splitlines()[0])
+    except Exception:
+        return None
 
 
 def cpu_baseline(w, mode):

@@ -48,7 +48,7 @@
 extern "C" {
 #endif
 
-#define LRS_VERSION 1
+#define LRS_VERSION 2
 
 typedef enum {
     LRS_OK = 0,
@@ -163,6 +163,44 @@ lrs_status lrs_decode_step(const lrs_state *st, void *state_codes, float *scales
                            const uint8_t *prec_map, const float *q, const float *k,
                            const float *v, const float *gates, const float *beta, float *out,
                            uint64_t seed, uint64_t step, int32_t mode, void *stream);
+
+/* The step with bfloat16 q, k, v and out, as a model layer in bfloat16 feeds
+ * and consumes it (the state, gates and beta are as in lrs_decode_step). The
+ * method's sources fix no input precision; this variant reads each bfloat16
+ * input as the float32 it denotes (exactly), runs the same fp32 step, and
+ * writes each output element as the bfloat16 nearest to the fp32 o_j (ties to
+ * even). q, k: [B][H][d_k], v, out: [B][H][d_v], bfloat16 bit patterns
+ * (sign, 8 exponent bits, 7 fraction bits), device memory, 16-byte aligned.
+ * Everything else -- layout, ownership, errors, asynchrony -- as
+ * lrs_decode_step. */
+lrs_status lrs_decode_step_bf16(const lrs_state *st, void *state_codes, float *scales,
+                                const uint8_t *prec_map, const uint16_t *q, const uint16_t *k,
+                                const uint16_t *v, const float *gates, const float *beta,
+                                uint16_t *out, uint64_t seed, uint64_t step, int32_t mode,
+                                void *stream);
+
+/* Multi-token (chunked) update: T tokens applied to every tile in order, one
+ * requantization at the end. The method's sources describe only the decode
+ * step, where the state is requantized after every update; for the tokens
+ * that precede decode (a prefill chunk, the tokens of a speculative-decoding
+ * verification) this entry point keeps the fp32 state on chip across the T
+ * updates and requantizes once, so repeated requantization happens once per
+ * chunk. Per tile: S = dequantized state; for t = 0..T-1 in order, the same
+ * update and output as lrs_decode_step with token t's inputs (S <- x,
+ * out[t] = x^T q_t); then new scales and codes from S by `mode` -- for BDR the
+ * update is S - (dequantized state at the chunk's start), for SR the counters
+ * are (seed, step). T = 1 gives exactly lrs_decode_step.
+ *   q, k: [T][B][H][d_k]; v, out: [T][B][H][d_v]; gates: [T][B][H][d_k]
+ *   (per-key) or [T][B][H] (scalar); beta: [T][B][H] (delta rule, else NULL):
+ *   token t's block is laid out exactly as one lrs_decode_step's inputs.
+ *   All device memory, fp32, 16-byte aligned.
+ *   Supported: d_k and d_v in {64, 128} (group as for the state); other
+ *   shapes return LRS_ERR_UNSUPPORTED. T = 0 is a no-op.
+ * Ownership, errors and asynchrony as lrs_decode_step. */
+lrs_status lrs_chunk_step(const lrs_state *st, void *state_codes, float *scales,
+                          const uint8_t *prec_map, int32_t T, const float *q, const float *k,
+                          const float *v, const float *gates, const float *beta, float *out,
+                          uint64_t seed, uint64_t step, int32_t mode, void *stream);
 
 /* The same step with HOST inputs and output: copies q, k, v, gates, beta
  * from host memory into device staging buffers owned by the state (allocated

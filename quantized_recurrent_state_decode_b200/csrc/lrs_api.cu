@@ -190,7 +190,16 @@ lrs::LayoutArgs layout_args(const lrs_state* st, unsigned* err) {
 
 namespace lrs {
 
-const void* find_step_kernel(int C, int group, int update_kind, int gate_kind, int mode) {
+const void* find_step_kernel(int C, int group, int update_kind, int gate_kind, int mode, int io) {
+    if (io == kStepIoBF16) {
+        switch (mode) {
+            case kRTN: return find_step_kernel_rtn_bf16(C, group, update_kind, gate_kind);
+            case kSR: return find_step_kernel_sr_bf16(C, group, update_kind, gate_kind);
+            case kBDR: return find_step_kernel_bdr_bf16(C, group, update_kind, gate_kind);
+            default: return nullptr;
+        }
+    }
+    if (io != kStepIoF32) return nullptr;
     switch (mode) {
         case kRTN: return find_step_kernel_rtn(C, group, update_kind, gate_kind);
         case kSR: return find_step_kernel_sr(C, group, update_kind, gate_kind);
@@ -199,18 +208,25 @@ const void* find_step_kernel(int C, int group, int update_kind, int gate_kind, i
     }
 }
 
-int step_warp_smem(int C, int group, int gate_kind, int slots, int mode) {
+int step_warp_smem(int C, int group, int gate_kind, int slots, int mode, int io, int d_k) {
     const bool xs = stage_x(mode);
-#define LRS_SLOT(CC, GG)                                                                    \
-    if (C == CC && group == GG)                                                             \
-        return gate_kind == kGatePerKey ? Slot<CC, GG, kGatePerKey>::warp_bytes(slots, xs)  \
-                                        : Slot<CC, GG, kGate>::warp_bytes(slots, xs);
+#define LRS_SLOT_IO(CC, GG, IO)                                                              \
+    return gate_kind == kGatePerKey ? Slot<CC, GG, kGatePerKey, IO>::warp_bytes(slots, xs, d_k) \
+                                    : Slot<CC, GG, kGate, IO>::warp_bytes(slots, xs, d_k);
+#define LRS_SLOT(CC, GG)                                                                     \
+    if (C == CC && group == GG) {                                                            \
+        if (io == kStepIoBF16) {                                                             \
+            LRS_SLOT_IO(CC, GG, kIoBF16)                                                     \
+        }                                                                                    \
+        LRS_SLOT_IO(CC, GG, kIoF32)                                                          \
+    }
     LRS_SLOT(4, 16)
     LRS_SLOT(4, 32)
     LRS_SLOT(2, 16)
     LRS_SLOT(2, 32)
     LRS_SLOT(2, 64)
 #undef LRS_SLOT
+#undef LRS_SLOT_IO
     return -1;
 }
 
@@ -318,10 +334,14 @@ lrs_status lrs_state_free(lrs_state* st) {
     return ok();
 }
 
-lrs_status lrs_decode_step(const lrs_state* st, void* state_codes, float* scales,
-                           const uint8_t* prec_map, const float* q, const float* k,
-                           const float* v, const float* gates, const float* beta, float* out,
-                           uint64_t seed, uint64_t step, int32_t mode, void* stream) {
+}  // extern "C"
+
+// The step with q, k, v and out of element type io (lrs::StepIo).
+static lrs_status decode_step_io(const lrs_state* st, void* state_codes, float* scales,
+                                 const uint8_t* prec_map, const void* q, const void* k,
+                                 const void* v, const float* gates, const float* beta, void* out,
+                                 uint64_t seed, uint64_t step, int32_t mode, int io,
+                                 void* stream) {
     lrs_status s = check_state(st);
     if (s != LRS_OK) return s;
     const lrs_shape& sh = st->shape;
@@ -337,7 +357,7 @@ lrs_status lrs_decode_step(const lrs_state* st, void* state_codes, float* scales
     if (mode != LRS_ROUND_RTN && mode != LRS_ROUND_SR && mode != LRS_ROUND_BDR)
         return fail(LRS_ERR_INVALID_ARG, "mode %d", mode);
     const int C = sh.d_v / 32, G = sh.d_k / sh.group;
-    const void* fn = lrs::find_step_kernel(C, sh.group, sh.update_kind, sh.gate_kind, mode);
+    const void* fn = lrs::find_step_kernel(C, sh.group, sh.update_kind, sh.gate_kind, mode, io);
     if (!fn) return fail(LRS_ERR_UNSUPPORTED, "no compiled kernel for this shape and mode");
     DeviceCtx* ctx = nullptr;
     s = device_ctx(&ctx);
@@ -354,7 +374,7 @@ lrs_status lrs_decode_step(const lrs_state* st, void* state_codes, float* scales
         slots = std::min(slots, G);
     }
     slots = std::max(1, std::min(slots, lrs::kMaxSlots));
-    const int warp_smem = lrs::step_warp_smem(C, sh.group, sh.gate_kind, slots, mode);
+    const int warp_smem = lrs::step_warp_smem(C, sh.group, sh.gate_kind, slots, mode, io, sh.d_k);
     constexpr int kSmemLimit = 227 * 1024;
     int warps = step_warps_override();
     if (warps <= 0) warps = kDefaultWarps;
@@ -440,6 +460,25 @@ lrs_status lrs_decode_step(const lrs_state* st, void* state_codes, float* scales
         return cuda_fail(e, "launch of the step kernel");
     }
     return ok();
+}
+
+extern "C" {
+
+lrs_status lrs_decode_step(const lrs_state* st, void* state_codes, float* scales,
+                           const uint8_t* prec_map, const float* q, const float* k,
+                           const float* v, const float* gates, const float* beta, float* out,
+                           uint64_t seed, uint64_t step, int32_t mode, void* stream) {
+    return decode_step_io(st, state_codes, scales, prec_map, q, k, v, gates, beta, out, seed,
+                          step, mode, lrs::kStepIoF32, stream);
+}
+
+lrs_status lrs_decode_step_bf16(const lrs_state* st, void* state_codes, float* scales,
+                                const uint8_t* prec_map, const uint16_t* q, const uint16_t* k,
+                                const uint16_t* v, const float* gates, const float* beta,
+                                uint16_t* out, uint64_t seed, uint64_t step, int32_t mode,
+                                void* stream) {
+    return decode_step_io(st, state_codes, scales, prec_map, q, k, v, gates, beta, out, seed,
+                          step, mode, lrs::kStepIoBF16, stream);
 }
 
 lrs_status lrs_decode_step_host(const lrs_state* st, const float* q_host, const float* k_host,
@@ -651,6 +690,23 @@ namespace lrs {
 
 // Status helpers for entry points defined in other translation units: they
 // set and clear the same thread-local message as the functions above.
+lrs_status device_error_word(unsigned** err, int* sms) {
+    DeviceCtx* ctx = nullptr;
+    lrs_status s = device_ctx(&ctx);
+    if (s != LRS_OK) return s;
+    *err = ctx->err;
+    *sms = ctx->sms;
+    return LRS_OK;
+}
+
+bool take_injected_timeout(uint64_t* timeout_ns) {
+    std::lock_guard<std::mutex> lk(g_inject_mu);
+    if (!g_inject) return false;
+    g_inject = false;
+    *timeout_ns = g_inject_timeout_ns;
+    return true;
+}
+
 lrs_status api_fail(lrs_status s, const char* msg) { return fail(s, "%s", msg); }
 lrs_status api_cuda_fail(cudaError_t e, const char* what) { return cuda_fail(e, what); }
 lrs_status api_ok() { return ok(); }

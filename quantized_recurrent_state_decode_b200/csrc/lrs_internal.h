@@ -8,17 +8,34 @@
 
 namespace lrs {
 
+// Element type of q, k, v and out.
+enum StepIo { kStepIoF32 = 0, kStepIoBF16 = 1 };
+
 // Kernel entry of one compiled step variant, or nullptr when the combination
 // (columns per lane C = d_v/32, group rows, update kind, gate kind, rounding
-// mode) is not compiled.
-const void* find_step_kernel(int C, int group, int update_kind, int gate_kind, int mode);
+// mode, I/O element type) is not compiled.
+const void* find_step_kernel(int C, int group, int update_kind, int gate_kind, int mode,
+                             int io = kStepIoF32);
 const void* find_step_kernel_rtn(int C, int group, int update_kind, int gate_kind);
 const void* find_step_kernel_sr(int C, int group, int update_kind, int gate_kind);
 const void* find_step_kernel_bdr(int C, int group, int update_kind, int gate_kind);
+const void* find_step_kernel_rtn_bf16(int C, int group, int update_kind, int gate_kind);
+const void* find_step_kernel_sr_bf16(int C, int group, int update_kind, int gate_kind);
+const void* find_step_kernel_bdr_bf16(int C, int group, int update_kind, int gate_kind);
 
 // Bytes of shared memory one warp of the step kernel uses with `slots` ring
-// slots in rounding mode `mode`.
-int step_warp_smem(int C, int group, int gate_kind, int slots, int mode);
+// slots in rounding mode `mode` with I/O element type `io` and d_k key rows.
+int step_warp_smem(int C, int group, int gate_kind, int slots, int mode, int io, int d_k);
+
+// The chunked-update kernel for one shape and rounding mode, with the bytes
+// of shared memory it takes per CTA ({nullptr, 0} when not compiled).
+struct ChunkKernel {
+    const void* fn;
+    int smem;
+};
+ChunkKernel find_chunk_kernel_rtn(int d_k, int d_v, int group, int update_kind, int gate_kind);
+ChunkKernel find_chunk_kernel_sr(int d_k, int d_v, int group, int update_kind, int gate_kind);
+ChunkKernel find_chunk_kernel_bdr(int d_k, int d_v, int group, int update_kind, int gate_kind);
 
 struct LayoutArgs {
     uint8_t* codes;
@@ -42,6 +59,13 @@ cudaError_t launch_fp32_step(int B, int H, int d_k, int d_v, int update_kind, in
 cudaError_t launch_decay_means(const float* decay, int64_t outer, int heads, int64_t inner,
                                double* means, cudaStream_t s);
 bool layout_kernels_support(int d_v, int group);
+
+// The current device's error word (read and cleared by lrs_sync) and SM count.
+lrs_status device_error_word(unsigned** err, int* sms);
+
+// Consumes an armed lrs_debug_inject_timeout: returns true (and the wait limit
+// to use) for the one launch that must issue no copies.
+bool take_injected_timeout(uint64_t* timeout_ns);
 
 // Status helpers shared by the C-ABI translation units (lrs_api.cu).
 lrs_status api_fail(lrs_status s, const char* msg);

@@ -27,6 +27,7 @@ namespace lrs {
 constexpr int kGate = 0, kGatePerKey = 1;        // matches lrs_gate_kind
 constexpr int kGated = 0, kDelta = 1;            // matches lrs_update_kind
 constexpr int kRTN = 0, kSR = 1, kBDR = 2;       // matches lrs_round_mode
+constexpr int kIoF32 = 0, kIoBF16 = 1;           // element type of q, k, v and out
 constexpr int kMaxSlots = 16;
 // Launch bound of a step variant in warps: 12 (at most 168 registers a thread)
 // where the live state fits, 8 (255 registers) for the wider groups and for
@@ -40,12 +41,12 @@ struct StepParams {
     const uint8_t* prec_map;
     const int64_t* head_offsets;
     int64_t batch_stride;
-    const float* q;
-    const float* k;
-    const float* v;
+    const void* q;       // fp32 or bfloat16 (the variant's IO)
+    const void* k;
+    const void* v;
     const float* gates;
     const float* beta;
-    float* out;
+    void* out;           // fp32 or bfloat16
     uint64_t seed;
     uint64_t step;
     unsigned* err;
@@ -56,26 +57,37 @@ struct StepParams {
     int32_t inject;      // fault injection: issue no copies
 };
 
-// Shared-memory layout of one warp:
-//   [0, 128)            mbarriers, one per slot
-//   [128, 128 + 4*d_v)  v of the tile whose first group was issued last
-//   then `slots` slots of kBytes each:
-//     codes (GROUP*d_v bytes: room for int8) | scales (d_v fp32) |
-//     q, k, [gate] (GROUP fp32 each)
-template <int C, int GROUP, int GATE>
+// Shared-memory layout of one warp (ES = bytes of a q, k, v element):
+//   [0, 128)          mbarriers, one per slot
+//   two tile-input buffers of tile_in_bytes(d_k) each, used by the warp's
+//   tiles in turn (tile n in buffer n & 1):
+//     q, k (d_k elements each) | [gate] (d_k fp32) | v (d_v elements)
+//   then `slots` slots of kBytes each, one scale group per item:
+//     codes (GROUP*d_v bytes: room for int8) | scales (d_v fp32)
+//   then, for SR and BDR, the x staging buffer.
+// A tile's inputs come with its first group, in one bulk copy per array.
+template <int C, int GROUP, int GATE, int IO = kIoF32>
 struct Slot {
     static constexpr int DV = 32 * C;
+    static constexpr int ES = IO == kIoBF16 ? 2 : 4;
     static constexpr int kCodes = GROUP * DV;                     // int8 capacity
     static constexpr int kScales = kCodes;
-    static constexpr int kQ = kScales + DV * 4;
-    static constexpr int kK = kQ + GROUP * 4;
-    static constexpr int kG = kK + GROUP * 4;
-    static constexpr int kBytes = kG + (GATE == kGatePerKey ? GROUP * 4 : 0);
-    static constexpr int kHeader = 128 + DV * 4;
+    static constexpr int kBytes = kScales + DV * 4;
     static_assert(kBytes % 16 == 0, "slot alignment");
     static constexpr int kXsBytes = GROUP * 256;   // x staging (SR, BDR): 16 B per row pair and lane
-    static int warp_bytes(int slots, bool xs) {
-        return (kHeader + slots * kBytes + (xs ? kXsBytes : 0) + 127) / 128 * 128;
+    // offsets inside a tile-input buffer
+    __host__ __device__ static int in_k(int d_k) { return d_k * ES; }
+    __host__ __device__ static int in_g(int d_k) { return 2 * d_k * ES; }
+    __host__ __device__ static int in_v(int d_k) {
+        return 2 * d_k * ES + (GATE == kGatePerKey ? d_k * 4 : 0);
+    }
+    __host__ __device__ static int tile_in_payload(int d_k) { return in_v(d_k) + DV * ES; }
+    __host__ __device__ static int tile_in_bytes(int d_k) {
+        return (tile_in_payload(d_k) + 15) / 16 * 16;
+    }
+    __host__ __device__ static int header(int d_k) { return 128 + 2 * tile_in_bytes(d_k); }
+    static int warp_bytes(int slots, bool xs, int d_k) {
+        return (header(d_k) + slots * kBytes + (xs ? kXsBytes : 0) + 127) / 128 * 128;
     }
 };
 
@@ -301,6 +313,51 @@ __device__ __forceinline__ void ld_smem_rows(const float* p, float (&r)[N]) {
     }
 }
 
+// bfloat16 pattern(s) -> float (exact: the pattern is the upper half of the
+// binary32 pattern).
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Rows [row0, row0 + N) of a q or k array in shared memory (element type IO),
+// as floats. row0 and N multiples of 8.
+template <int IO, int N>
+__device__ __forceinline__ void ld_rows(const uint8_t* base, int row0, float (&r)[N]) {
+    if constexpr (IO == kIoF32) {
+        ld_smem_rows<N>(reinterpret_cast<const float*>(base) + row0, r);
+    } else {
+        const uint4* p = reinterpret_cast<const uint4*>(base + row0 * 2);
+#pragma unroll
+        for (int i = 0; i < N / 8; ++i) {
+            const uint4 t = p[i];
+            const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                r[8 * i + 2 * e] = bf16_lo(w[e]);
+                r[8 * i + 2 * e + 1] = bf16_hi(w[e]);
+            }
+        }
+    }
+}
+
+// Two floats as the bfloat16 patterns nearest to them (ties to even), x in
+// the low half of the word.
+__device__ __forceinline__ uint32_t bf16x2_rn(float2 v) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(v.y), "f"(v.x));
+    return r;
+}
+
+// Elements idx, idx + 1 (idx even) of a v array in shared memory.
+template <int IO>
+__device__ __forceinline__ float2 ld_pair(const uint8_t* base, int idx) {
+    if constexpr (IO == kIoF32) {
+        return *reinterpret_cast<const float2*>(base + idx * 4);
+    } else {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(base + idx * 2);
+        return make_float2(bf16_lo(w), bf16_hi(w));
+    }
+}
+
 // Geometry of one lane's codes for one column pair of one scale group: a run
 // of 16-byte units, each holding EPU consecutive elements of the pair's
 // row-major (row, column) stream, i.e. RPU key rows; a 32-bit word holds RPW
@@ -323,9 +380,9 @@ __device__ __forceinline__ uint4 lds_unit(const uint8_t* cs, int unit, int lane)
 
 // Delta rule, first pass: u_c += k_i * deq_ic for the two columns of one
 // pair over the rows of one group, in key order.
-template <int GROUP, int BITS>
+template <int GROUP, int BITS, int IO>
 __device__ __forceinline__ void pair_ktS(const uint8_t* __restrict__ cs, int ubase, float2 sc,
-                                         const float* __restrict__ ks, int lane, float2& u) {
+                                         const uint8_t* __restrict__ ks, int lane, float2& u) {
     using G = PairGeo<GROUP, BITS>;
     constexpr float BIAS = Q<BITS>::kBias;
     const float2 s0 = f2(sc.x), s1 = f2(sc.y);
@@ -334,7 +391,7 @@ __device__ __forceinline__ void pair_ktS(const uint8_t* __restrict__ cs, int uba
         const uint4 raw = lds_unit(cs, ubase + un, lane);
         const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
         float kk[G::RPU];
-        ld_smem_rows<G::RPU>(ks + un * G::RPU, kk);
+        ld_rows<IO, G::RPU>(ks, un * G::RPU, kk);
 #pragma unroll
         for (int wi = 0; wi < 4; ++wi) {
             float f[G::EPW];
@@ -358,10 +415,10 @@ __device__ __forceinline__ void pair_ktS(const uint8_t* __restrict__ cs, int uba
 // One column pair of one scale group: dequantize, update, accumulate the
 // output, new scales, requantize and store. x[rp][c] holds rows (2rp, 2rp+1)
 // of column c of the pair.
-template <int GROUP, int GATE, int MODE, int BITS>
+template <int GROUP, int GATE, int MODE, int BITS, int IO>
 __device__ __forceinline__ void pair_step(const uint8_t* __restrict__ cs, int ubase, float2 sc,
-                                          const float* __restrict__ qs,
-                                          const float* __restrict__ ks,
+                                          const uint8_t* __restrict__ qs,
+                                          const uint8_t* __restrict__ ks,
                                           const float* __restrict__ gs, float gscalar, float2 w,
                                           float2& o, uint8_t* __restrict__ gcodes,
                                           float* __restrict__ gscale, uint64_t hkey, int row0,
@@ -378,8 +435,8 @@ __device__ __forceinline__ void pair_step(const uint8_t* __restrict__ cs, int ub
         const uint4 raw = lds_unit(cs, ubase + un, lane);
         const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
         float kk[G::RPU], qq[G::RPU], gg[G::RPU];
-        ld_smem_rows<G::RPU>(ks + un * G::RPU, kk);
-        ld_smem_rows<G::RPU>(qs + un * G::RPU, qq);
+        ld_rows<IO, G::RPU>(ks, un * G::RPU, kk);
+        ld_rows<IO, G::RPU>(qs, un * G::RPU, qq);
         if constexpr (GATE == kGatePerKey) ld_smem_rows<G::RPU>(gs + un * G::RPU, gg);
 #pragma unroll
         for (int wi = 0; wi < 4; ++wi) {
@@ -501,10 +558,10 @@ struct TileCursor {
 // instead of registers, so both phases are short loops over 16-byte units and
 // the kernel's code stays small enough for the instruction cache. xs holds
 // (x[r][c0], x[r+1][c0], x[r][c1], x[r+1][c1]) per row pair r and lane.
-template <int GROUP, int GATE, int MODE, int BITS>
+template <int GROUP, int GATE, int MODE, int BITS, int IO>
 __device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int ubase, float2 sc,
-                                             const float* __restrict__ qs,
-                                             const float* __restrict__ ks,
+                                             const uint8_t* __restrict__ qs,
+                                             const uint8_t* __restrict__ ks,
                                              const float* __restrict__ gs, float gscalar,
                                              float2 w, float2& o, uint8_t* __restrict__ gcodes,
                                              float* __restrict__ gscale, uint64_t hkey, int row0,
@@ -522,8 +579,8 @@ __device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int
         const uint4 raw = lds_unit(cs, ubase + un, lane);
         const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
         float kk[G::RPU], qq[G::RPU], gg[G::RPU];
-        ld_smem_rows<G::RPU>(ks + un * G::RPU, kk);
-        ld_smem_rows<G::RPU>(qs + un * G::RPU, qq);
+        ld_rows<IO, G::RPU>(ks, un * G::RPU, kk);
+        ld_rows<IO, G::RPU>(qs, un * G::RPU, qq);
         if constexpr (GATE == kGatePerKey) ld_smem_rows<G::RPU>(gs + un * G::RPU, gg);
 #pragma unroll
         for (int wi = 0; wi < 4; ++wi) {
@@ -596,34 +653,42 @@ __device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int
     }
 }
 
-// Fill `slot` with group g of the cursor's tile (lane 0 only). A tile whose
-// layout does not fit gets a bare arrival, so the slot's phase still completes.
-template <int C, int GROUP, int GATE>
+// Fill `slot` with group g of the cursor's tile (lane 0 only); with the
+// first group, also the tile's inputs into `tin`. A tile whose layout does not
+// fit gets a bare arrival, so the slot's phase still completes.
+template <int C, int GROUP, int GATE, int IO>
 __device__ __forceinline__ void issue_item(const StepParams& p, uint8_t* wsm, int slot,
-                                           const TileCursor& tc, int g, uint64_t pol_state,
-                                           uint64_t pol_in) {
-    using S = Slot<C, GROUP, GATE>;
+                                           const TileCursor& tc, int g, uint8_t* tin,
+                                           uint64_t pol_state, uint64_t pol_in) {
+    using S = Slot<C, GROUP, GATE, IO>;
     constexpr int DV = 32 * C;
+    constexpr int ES = S::ES;
     uint64_t* bar = reinterpret_cast<uint64_t*>(wsm) + slot;
     if (tc.prec == 0) {
         mbar_arrive(bar);
         return;
     }
     const int tile = tc.tile;
-    uint8_t* sm = wsm + S::kHeader + slot * S::kBytes;
+    const int dk = p.d_k;
+    uint8_t* sm = wsm + S::header(dk) + slot * S::kBytes;
     const uint32_t cbytes = GROUP * DV * tc.prec / 8;
-    uint32_t total = cbytes + DV * 4 + 2 * GROUP * 4;
-    if (GATE == kGatePerKey) total += GROUP * 4;
-    if (g == 0) total += DV * 4;
+    uint32_t total = cbytes + DV * 4;
+    if (g == 0) total += S::tile_in_payload(dk);
     mbar_arrive_expect_tx(bar, total);
     bulk_g2s(sm, p.codes + tc.code_off + static_cast<int64_t>(g) * cbytes, cbytes, bar, pol_state);
     bulk_g2s(sm + S::kScales, p.scales + (static_cast<int64_t>(tile) * p.G + g) * DV, DV * 4, bar,
              pol_state);
-    const int64_t rowbase = static_cast<int64_t>(tile) * p.d_k + g * GROUP;
-    bulk_g2s(sm + S::kQ, p.q + rowbase, GROUP * 4, bar, pol_in);
-    bulk_g2s(sm + S::kK, p.k + rowbase, GROUP * 4, bar, pol_in);
-    if (GATE == kGatePerKey) bulk_g2s(sm + S::kG, p.gates + rowbase, GROUP * 4, bar, pol_in);
-    if (g == 0) bulk_g2s(wsm + 128, p.v + static_cast<int64_t>(tile) * DV, DV * 4, bar, pol_in);
+    if (g == 0) {
+        const int64_t rowbase = static_cast<int64_t>(tile) * dk;
+        bulk_g2s(tin, static_cast<const uint8_t*>(p.q) + rowbase * ES, dk * ES, bar, pol_in);
+        bulk_g2s(tin + S::in_k(dk), static_cast<const uint8_t*>(p.k) + rowbase * ES, dk * ES, bar,
+                 pol_in);
+        if (GATE == kGatePerKey)
+            bulk_g2s(tin + S::in_g(dk), p.gates + rowbase, dk * 4, bar, pol_in);
+        bulk_g2s(tin + S::in_v(dk),
+                 static_cast<const uint8_t*>(p.v) + static_cast<int64_t>(tile) * DV * ES, DV * ES,
+                 bar, pol_in);
+    }
 }
 
 // Position in a warp's ring: item k lives in slot k % slots and completes
@@ -641,10 +706,10 @@ struct Ring {
 
 // The warp's items are (tile, group) pairs in order: item k is group k % G of
 // the warp's tile k / G (tiles gw, gw + W, ...).
-template <int C, int GROUP, int UPD, int GATE, int MODE>
+template <int C, int GROUP, int UPD, int GATE, int MODE, int IO>
 __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
     step_kernel(const StepParams p) {
-    using S = Slot<C, GROUP, GATE>;
+    using S = Slot<C, GROUP, GATE, IO>;
     constexpr int DV = 32 * C;
     constexpr int P = C / 2;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -655,9 +720,10 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
     const int gw = blockIdx.x * nw + wib;
     uint8_t* wsm = smem + wib * p.warp_smem;
     uint64_t* bars = reinterpret_cast<uint64_t*>(wsm);
-    const float* v_s = reinterpret_cast<const float*>(wsm + 128);
     const int G = p.G, NS = p.slots;
-    float4* xs = reinterpret_cast<float4*>(wsm + S::kHeader + NS * S::kBytes);   // SR, BDR
+    const int hdr = S::header(p.d_k), tib = S::tile_in_bytes(p.d_k);
+    const int in_k = S::in_k(p.d_k), in_g = S::in_g(p.d_k), in_v = S::in_v(p.d_k);
+    float4* xs = reinterpret_cast<float4*>(wsm + hdr + NS * S::kBytes);   // SR, BDR
     const int ntw = gw < p.ntiles ? (p.ntiles - gw + W - 1) / W : 0;   // this warp's tiles
     const int64_t K = static_cast<int64_t>(ntw) * G;                    // this warp's items
 
@@ -672,17 +738,21 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
     Ring ic, is;                 // consumer and issuer positions
     int64_t kc = 0, ki = 0;      // items consumed, items issued
     int it_g = 0;                // group of item ki
+    int it_n = 0;                // warp-local tile number of item ki
     TileCursor itc;              // tile of item ki
     itc.init(p, gw, W);
     if (K > 0) itc.load(p, DV);
 
     auto issue_next = [&]() {
         if (ki < K && !p.inject) {
-            if (lane == 0) issue_item<C, GROUP, GATE>(p, wsm, is.slot, itc, it_g, pol_state, pol_in);
+            if (lane == 0)
+                issue_item<C, GROUP, GATE, IO>(p, wsm, is.slot, itc, it_g,
+                                               wsm + 128 + (it_n & 1) * tib, pol_state, pol_in);
             ++ki;
             is.advance(NS);
             if (++it_g == G) {
                 it_g = 0;
+                ++it_n;
                 itc.advance(p, W);
                 if (ki < K) itc.load(p, DV);
             }
@@ -702,6 +772,7 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
     for (int n = 0; n < ntw && ok; ++n, ti.advance(p, W)) {
         const int tile = ti.tile;
         ti.load(p, DV);
+        const uint8_t* tin = wsm + 128 + (n & 1) * tib;   // this tile's q, k, gates, v
         const float gscalar = nscal, beta = nbeta;
         if (n + 1 < ntw) {
             if (GATE == kGate) nscal = __ldg(p.gates + tile + W);
@@ -748,17 +819,17 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
                     ok = __all_sync(0xffffffffu,
                                     mbar_wait_bounded(&bars[r.slot], r.par, p.timeout_ns));
                 if (!ok) break;
-                const uint8_t* sm = wsm + S::kHeader + r.slot * S::kBytes;
+                const uint8_t* sm = wsm + hdr + r.slot * S::kBytes;
                 const float* ss = reinterpret_cast<const float*>(sm + S::kScales) + lane * C;
-                const float* ks = reinterpret_cast<const float*>(sm + S::kK);
+                const uint8_t* ks = tin + in_k + g * GROUP * S::ES;
                 float2 up = u[0], uq = u[P - 1];
 #pragma unroll 1
                 for (int pc = 0; pc < P; ++pc) {
                     const float2 sc = *reinterpret_cast<const float2*>(ss + 2 * pc);
                     if (ti.prec == 8)
-                        pair_ktS<GROUP, 8>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, ks, lane, up);
+                        pair_ktS<GROUP, 8, IO>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, ks, lane, up);
                     else
-                        pair_ktS<GROUP, 4>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, ks, lane, up);
+                        pair_ktS<GROUP, 4, IO>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, ks, lane, up);
                     if constexpr (P == 2) {
                         const float2 t = up;
                         up = uq; uq = t;
@@ -770,7 +841,7 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
             }
 #pragma unroll
             for (int pc = 0; pc < P; ++pc) {
-                const float2 vv = *reinterpret_cast<const float2*>(v_s + lane * C + 2 * pc);
+                const float2 vv = ld_pair<IO>(tin + in_v, lane * C + 2 * pc);
                 // w = beta (v - alpha u): three separate roundings
                 const float d0 = __fsub_rn(vv.x, __fmul_rn(gscalar, u[pc].x));
                 const float d1 = __fsub_rn(vv.y, __fmul_rn(gscalar, u[pc].y));
@@ -779,7 +850,7 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
         } else {
 #pragma unroll
             for (int pc = 0; pc < P; ++pc)
-                w[pc] = *reinterpret_cast<const float2*>(v_s + lane * C + 2 * pc);
+                w[pc] = ld_pair<IO>(tin + in_v, lane * C + 2 * pc);
         }
 
         if (!ok) break;
@@ -791,11 +862,11 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
                                 mbar_wait_bounded(&bars[ic.slot], ic.par, p.timeout_ns));
                 if (!ok) break;
             }
-            const uint8_t* sm = wsm + S::kHeader + ic.slot * S::kBytes;
+            const uint8_t* sm = wsm + hdr + ic.slot * S::kBytes;
             const float* ss = reinterpret_cast<const float*>(sm + S::kScales) + lane * C;
-            const float* qs = reinterpret_cast<const float*>(sm + S::kQ);
-            const float* ks = reinterpret_cast<const float*>(sm + S::kK);
-            const float* gs = reinterpret_cast<const float*>(sm + S::kG);
+            const uint8_t* qs = tin + g * GROUP * S::ES;
+            const uint8_t* ks = tin + in_k + g * GROUP * S::ES;
+            const float* gs = reinterpret_cast<const float*>(tin + in_g) + g * GROUP;
             float* gscale = p.scales + (static_cast<int64_t>(tile) * G + g) * DV + lane * C;
             uint8_t* gcodes = gcodes_tile + static_cast<int64_t>(g) * cbytes;
             // The column pairs run one after the other through one copy of the
@@ -807,22 +878,22 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
                 const uint32_t j0 = static_cast<uint32_t>(lane * C + 2 * pc);
                 if constexpr (stage_x(MODE)) {
                     if (ti.prec == 8)
-                        pair_step_xs<GROUP, GATE, MODE, 8>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs,
+                        pair_step_xs<GROUP, GATE, MODE, 8, IO>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs,
                                                            ks, gs, gscalar, wp, op, gcodes,
                                                            gscale + 2 * pc, hkey, g * GROUP, j0,
                                                            lane, xs);
                     else
-                        pair_step_xs<GROUP, GATE, MODE, 4>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs,
+                        pair_step_xs<GROUP, GATE, MODE, 4, IO>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs,
                                                            ks, gs, gscalar, wp, op, gcodes,
                                                            gscale + 2 * pc, hkey, g * GROUP, j0,
                                                            lane, xs);
                 } else {
                     if (ti.prec == 8)
-                        pair_step<GROUP, GATE, MODE, 8>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs, ks,
+                        pair_step<GROUP, GATE, MODE, 8, IO>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs, ks,
                                                         gs, gscalar, wp, op, gcodes,
                                                         gscale + 2 * pc, hkey, g * GROUP, j0, lane);
                     else
-                        pair_step<GROUP, GATE, MODE, 4>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs, ks,
+                        pair_step<GROUP, GATE, MODE, 4, IO>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs, ks,
                                                         gs, gscalar, wp, op, gcodes,
                                                         gscale + 2 * pc, hkey, g * GROUP, j0, lane);
                 }
@@ -840,11 +911,23 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
             issue_next();
         }
         if (!ok) break;
-        float* op = p.out + static_cast<int64_t>(tile) * DV + lane * C;
-        if constexpr (P == 2) {
-            *reinterpret_cast<float4*>(op) = make_float4(o[0].x, o[0].y, o[1].x, o[1].y);
+        const int64_t oi = static_cast<int64_t>(tile) * DV + lane * C;
+        if constexpr (IO == kIoF32) {
+            float* op = static_cast<float*>(p.out) + oi;
+            if constexpr (P == 2) {
+                *reinterpret_cast<float4*>(op) = make_float4(o[0].x, o[0].y, o[1].x, o[1].y);
+            } else {
+                *reinterpret_cast<float2*>(op) = o[0];
+            }
         } else {
-            *reinterpret_cast<float2*>(op) = o[0];
+            // nearest bfloat16, ties to even
+            uint16_t* op = static_cast<uint16_t*>(p.out) + oi;
+            const uint32_t w0 = bf16x2_rn(o[0]);
+            if constexpr (P == 2) {
+                *reinterpret_cast<uint2*>(op) = make_uint2(w0, bf16x2_rn(o[1]));
+            } else {
+                *reinterpret_cast<uint32_t*>(op) = w0;
+            }
         }
     }
     if (!ok) {

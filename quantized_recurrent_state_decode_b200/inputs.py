@@ -163,6 +163,16 @@ def step_inputs(w: Workload, t: int, batch_offset: int = 0, batch: Optional[int]
     return {n: (None if x is None else x.contiguous()) for n, x in out.items()}
 
 
+def chunk_inputs(w: Workload, t0: int, T: int, batch_offset: int = 0,
+                 batch: Optional[int] = None, device="cpu"):
+    """The inputs of steps t0 .. t0 + T - 1 stacked on a leading token axis:
+    q, k [T][B][H][d_k], v [T][B][H][d_v], gates [T][B][H][d_k] or [T][B][H],
+    beta [T][B][H] or None (a chunk of T tokens)."""
+    xs = [step_inputs(w, t, batch_offset, batch, device=device) for t in range(t0, t0 + T)]
+    return {n: (None if xs[0][n] is None else torch.stack([x[n] for x in xs]).contiguous())
+            for n in xs[0]}
+
+
 def initial_state(w: Workload, batch_offset: int = 0, batch: Optional[int] = None,
                   device="cpu"):
     """S0 [B][H][d_k][d_v]: zeros, or N(0, s0_std^2)."""

@@ -57,6 +57,10 @@ _SIGS = {
     "lrs_state_free": [ctypes.POINTER(lrs_state)],
     "lrs_decode_step": [ctypes.POINTER(lrs_state), _P, _P, _P, _P, _P, _P, _P, _P, _P,
                         ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int32, _P],
+    "lrs_decode_step_bf16": [ctypes.POINTER(lrs_state), _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                             ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int32, _P],
+    "lrs_chunk_step": [ctypes.POINTER(lrs_state), _P, _P, _P, ctypes.c_int32, _P, _P, _P, _P, _P,
+                       _P, ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int32, _P],
     "lrs_decode_step_host": [ctypes.POINTER(lrs_state), _P, _P, _P, _P, _P, _P,
                              ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int32, _P],
     "lrs_decode_step_host_noalloc": [ctypes.POINTER(lrs_state), _P, _P, _P, _P, _P, _P, _P,
@@ -167,6 +171,22 @@ def lrs_decode_step(st, state_codes, scales, prec_map, q, k, v, gates, beta, out
     _check(lib().lrs_decode_step(ctypes.byref(st), _ptr(state_codes), _ptr(scales),
                                  _ptr(prec_map), _ptr(q), _ptr(k), _ptr(v), _ptr(gates),
                                  _ptr(beta), _ptr(out), seed, step, mode, _stream(stream)))
+
+
+def lrs_decode_step_bf16(st, state_codes, scales, prec_map, q, k, v, gates, beta, out, seed,
+                         step, mode, stream=None):
+    """q, k, v, out: bfloat16 device buffers (torch.bfloat16 tensors or addresses)."""
+    _check(lib().lrs_decode_step_bf16(ctypes.byref(st), _ptr(state_codes), _ptr(scales),
+                                      _ptr(prec_map), _ptr(q), _ptr(k), _ptr(v), _ptr(gates),
+                                      _ptr(beta), _ptr(out), seed, step, mode, _stream(stream)))
+
+
+def lrs_chunk_step(st, state_codes, scales, prec_map, T, q, k, v, gates, beta, out, seed, step,
+                   mode, stream=None):
+    """T tokens per tile, one requantization at the end; inputs [T][B][H][...]."""
+    _check(lib().lrs_chunk_step(ctypes.byref(st), _ptr(state_codes), _ptr(scales), _ptr(prec_map),
+                                T, _ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(beta), _ptr(out),
+                                seed, step, mode, _stream(stream)))
 
 
 def lrs_decode_step_host(st, q_host, k_host, v_host, gates_host, beta_host, out_host, seed, step,

@@ -66,8 +66,9 @@ def sample_tiles(w, pm, n_b=8, n_h=8):
 class Pair:
     """A GPU state and the oracle's copy of selected tiles."""
 
-    def __init__(self, w, pm, tiles=None, mode=None, device="cuda"):
+    def __init__(self, w, pm, tiles=None, mode=None, device="cuda", io="f32"):
         self.w, self.pm, self.device = w, np.asarray(pm, np.uint8), device
+        self.io = io
         self.mode = w.mode if mode is None else mode
         self.shape = make_shape(w)
         self.st = lrs.lrs_state_alloc(self.shape, self.pm)
@@ -83,7 +84,8 @@ class Pair:
         self.th_t = torch.as_tensor(th, dtype=torch.long, device=device)
         self.G = w.d_k // w.group
         self.prec_dev = torch.as_tensor(self.pm, device=device)
-        self.out = torch.empty(w.batch, w.heads, w.d_v, device=device)
+        self.out = torch.empty(w.batch, w.heads, w.d_v, device=device,
+                               dtype=torch.bfloat16 if io == "bf16" else torch.float32)
 
     def free(self):
         lrs.lrs_state_free(self.st)
@@ -109,9 +111,18 @@ class Pair:
         """One step on both sides; returns (gpu_out, oracle_out) for the tiles."""
         w = self.w
         beta = x["beta"]
-        lrs.lrs_decode_step(self.st, self.st.state_codes, self.st.scales, self.st.prec_map,
-                            x["q"], x["k"], x["v"], x["gates"], beta, self.out, seed, t,
-                            self.mode)
+        if self.io == "bf16":
+            # the inputs a bfloat16 model layer would pass: the seeded fp32
+            # inputs rounded to bfloat16; the oracle gets the values they denote
+            qkv = {n: x[n].to(torch.bfloat16) for n in ("q", "k", "v")}
+            lrs.lrs_decode_step_bf16(self.st, self.st.state_codes, self.st.scales,
+                                     self.st.prec_map, qkv["q"], qkv["k"], qkv["v"], x["gates"],
+                                     beta, self.out, seed, t, self.mode)
+            x = dict(x, **{n: qkv[n].float() for n in qkv})
+        else:
+            lrs.lrs_decode_step(self.st, self.st.state_codes, self.st.scales, self.st.prec_map,
+                                x["q"], x["k"], x["v"], x["gates"], beta, self.out, seed, t,
+                                self.mode)
         sel = lambda a: None if a is None else a[self.tb_t, self.th_t].cpu().numpy()
         gates = sel(x["gates"])
         o_ref = oracle.step(self.codes, self.scales, sel(x["q"]), sel(x["k"]), sel(x["v"]),
@@ -119,9 +130,14 @@ class Pair:
                             group=w.group, update_kind=w.update_kind, gate_kind=w.gate_kind,
                             mode=self.mode, seed=seed, step=t,
                             nthreads=oracle.default_threads())
-        o_gpu = self.out[self.tb_t, self.th_t].cpu().numpy()
+        o_gpu = self.out[self.tb_t, self.th_t]
         lrs.lrs_sync()
-        return o_gpu, o_ref
+        if self.io == "bf16":
+            # bfloat16 outputs compared as bit patterns with the oracle's
+            # nearest-even rounding of its fp32 output
+            o_gpu = o_gpu.view(torch.int16).cpu().numpy().view(np.uint16)
+            return o_gpu, oracle.bf16_rne(o_ref)
+        return o_gpu.cpu().numpy(), o_ref
 
     def compare_state(self, where=""):
         check_codes(self.gpu_codes(), self.codes, where)
@@ -164,13 +180,22 @@ def check_out(gpu, ref, where=""):
         where, err / scale)
 
 
-def run_parity(w, steps, tiles=None, mode=None, check_every=None, device="cuda", stats=None):
+def check_out_bf16(gpu, ref, where=""):
+    """bfloat16 outputs: the same bit patterns (the fp32 o before the final
+    rounding is exact, so its nearest bfloat16 is too)."""
+    bad = np.count_nonzero(gpu != ref)
+    assert bad == 0, "%s: %d of %d bfloat16 outputs differ, first at %s" % (
+        where, bad, gpu.size, np.argwhere(gpu != ref)[:4].tolist())
+
+
+def run_parity(w, steps, tiles=None, mode=None, check_every=None, device="cuda", stats=None,
+               io="f32"):
     """Free-running parity over `steps` steps; full state compared at
     step 0 (import), 1, 2, steps//2 and steps (or every step if check_every=1)."""
     pm = prec_map_for(w, device=device)
     if tiles == "sample":
         tiles = sample_tiles(w, pm)
-    pair = Pair(w, pm, tiles=tiles, mode=mode, device=device)
+    pair = Pair(w, pm, tiles=tiles, mode=mode, device=device, io=io)
     try:
         pair.init(I.initial_state(w, device=device))
         pair.compare_state("import")
@@ -180,7 +205,10 @@ def run_parity(w, steps, tiles=None, mode=None, check_every=None, device="cuda",
         for t in range(steps):
             x = I.step_inputs(w, t, device=device)
             o_gpu, o_ref = pair.step(x, t, seed)
-            check_out(o_gpu, o_ref, "%s step %d" % (w.name, t))
+            if io == "bf16":
+                check_out_bf16(o_gpu, o_ref, "%s step %d" % (w.name, t))
+            else:
+                check_out(o_gpu, o_ref, "%s step %d" % (w.name, t))
             exact_out += int(np.array_equal(o_gpu, o_ref))
             if check_every == 1 or (t + 1) in checkpoints:
                 pair.compare_state("%s after step %d" % (w.name, t + 1))

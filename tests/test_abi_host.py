@@ -39,7 +39,7 @@ def test_exports_every_declared_function():
 
 
 def test_version_and_status_names():
-    assert lrs.lrs_version() == 1
+    assert lrs.lrs_version() == 2
     assert lrs.lrs_status_string(lrs.LRS_ERR_DEVICE_TIMEOUT) == "LRS_ERR_DEVICE_TIMEOUT"
     assert lrs.lrs_status_string(99) == "LRS_ERR_UNKNOWN"
 
