@@ -34,6 +34,7 @@ METRIC = "quantized-state decode steps/s and state GB/s (% of HBM peak), B=256 3
 DEFAULT_WORKLOAD = "gla_rtn_int8_b256h32_128"
 MODES = {"rtn": 0, "sr": 1, "bdr": 2}
 KERNEL_SOURCES = ["quantized_recurrent_state_decode_b200/csrc/step_kernel.cuh",
+                  "quantized_recurrent_state_decode_b200/csrc/step_instances.cuh",
                   "quantized_recurrent_state_decode_b200/csrc/lrs_device.cuh",
                   "quantized_recurrent_state_decode_b200/csrc/step_rtn.cu"]
 PROFILE = os.path.join(ROOT, "profiles", "step_kernel_gla_rtn_int8_b256h32.md")

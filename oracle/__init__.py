@@ -40,6 +40,10 @@ def lib():
         L.orc_chunk_step.argtypes = [i32, P, P, i32, i32, i32, i32, i32, i32, P, P, P, i32, P, P,
                                      P, P, P, P, u64, u64, i32]
         L.orc_chunk_step.restype = i32
+        L.orc_step_pg.argtypes = L.orc_step.argtypes
+        L.orc_step_pg.restype = i32
+        L.orc_chunk_step_pg.argtypes = L.orc_chunk_step.argtypes
+        L.orc_chunk_step_pg.restype = i32
         L.orc_bf16_rne.argtypes = [ctypes.c_float]
         L.orc_bf16_rne.restype = ctypes.c_uint16
         L.orc_bf16_rne_array.argtypes = [i64, P, P]
@@ -48,6 +52,8 @@ def lib():
         L.orc_fp32_step.restype = i32
         L.orc_import.argtypes = [i32, P, i32, i32, i32, P, P, P, P]
         L.orc_import.restype = i32
+        L.orc_import_pg.argtypes = L.orc_import.argtypes
+        L.orc_import_pg.restype = i32
         L.orc_dequant.argtypes = [i32, i32, i32, i32, P, P, P]
         L.orc_dequant.restype = i32
         L.orc_decay_means.argtypes = [i64, i32, i64, P, P]
@@ -67,6 +73,16 @@ def _p(a):
 
 def _f32(a):
     return None if a is None else np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _per_group(prec_map, d_k, group, per_head_fn, per_group_fn):
+    """prec_map [H] selects the per-head entry point, [H][d_k/group] the
+    per-(head, group) one."""
+    if prec_map.ndim == 1:
+        return per_head_fn
+    if prec_map.ndim != 2 or prec_map.shape[1] != d_k // group:
+        raise ValueError("prec_map must be [H] or [H][d_k/group]")
+    return per_group_fn
 
 
 def splitmix64(z):
@@ -100,7 +116,8 @@ def step(codes, scales, q, k, v, gates, beta, prec_map, tile_b, tile_h, *, group
     tile_b = np.ascontiguousarray(tile_b, dtype=np.int32)
     tile_h = np.ascontiguousarray(tile_h, dtype=np.int32)
     out = np.zeros((n, d_v), np.float32)
-    rc = lib().orc_step(n, _p(tile_b), _p(tile_h), d_k, d_v, group, update_kind, gate_kind, mode,
+    fn = _per_group(prec_map, d_k, group, lib().orc_step, lib().orc_step_pg)
+    rc = fn(n, _p(tile_b), _p(tile_h), d_k, d_v, group, update_kind, gate_kind, mode,
                         _p(prec_map), _p(codes), _p(scales), _p(q), _p(k), _p(v), _p(gates),
                         _p(beta), _p(out), seed, step, nthreads)
     if rc != 0:
@@ -125,7 +142,8 @@ def chunk_step(codes, scales, q, k, v, gates, beta, prec_map, tile_b, tile_h, *,
     tile_b = np.ascontiguousarray(tile_b, dtype=np.int32)
     tile_h = np.ascontiguousarray(tile_h, dtype=np.int32)
     out = np.zeros((T, n, d_v), np.float32)
-    rc = lib().orc_chunk_step(n, _p(tile_b), _p(tile_h), d_k, d_v, group, update_kind,
+    fn = _per_group(prec_map, d_k, group, lib().orc_chunk_step, lib().orc_chunk_step_pg)
+    rc = fn(n, _p(tile_b), _p(tile_h), d_k, d_v, group, update_kind,
                               gate_kind, mode, _p(prec_map), _p(codes), _p(scales), T, _p(q),
                               _p(k), _p(v), _p(gates), _p(beta), _p(out), seed, step, nthreads)
     if rc != 0:
@@ -168,7 +186,8 @@ def import_fp32(S0, prec_map, tile_h, *, group):
     tile_h = np.ascontiguousarray(tile_h, dtype=np.int32)
     codes = np.zeros((n, d_k, d_v), np.int8)
     scales = np.zeros((n, d_k // group, d_v), np.float32)
-    rc = lib().orc_import(n, _p(tile_h), d_k, d_v, group, _p(prec_map), _p(S0), _p(codes),
+    fn = _per_group(prec_map, d_k, group, lib().orc_import, lib().orc_import_pg)
+    rc = fn(n, _p(tile_h), d_k, d_v, group, _p(prec_map), _p(S0), _p(codes),
                           _p(scales))
     if rc != 0:
         raise ValueError("orc_import rejected its arguments (%d)" % rc)

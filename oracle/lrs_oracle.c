@@ -97,12 +97,13 @@ static int round_element(int mode, float x, float deq, float inv, float s_new, i
 
 /* Steps 4 and 5 for one tile: new scales from x, then codes. deq may be NULL
  * for RTN (import). */
-static void requantize_tile(int d_k, int d_v, int group, int qmax, int mode, const float *x,
+static void requantize_tile(int d_k, int d_v, int group, const int *qmaxs, int mode, const float *x,
                             const float *deq, int8_t *codes, float *scales, uint64_t seed,
                             uint64_t step, uint32_t b, uint32_t h)
 {
     int G = d_k / group;
     for (int g = 0; g < G; ++g) {
+        int qmax = qmaxs[g];
         for (int j = 0; j < d_v; ++j) {
             float A = 0.0f;
             for (int i = g * group; i < (g + 1) * group; ++i) {
@@ -182,11 +183,25 @@ static int qmax_of(uint8_t bits)
     return bits == 8 ? 127 : (bits == 4 ? 7 : -1);
 }
 
+/* qmax of each scale group of head h: prec_map holds one width per head
+ * (prec_groups == 1) or one per (head, group) in [H][G] order (prec_groups ==
+ * G). Returns -1 if a width is neither 4 nor 8. */
+static int head_qmaxs(const uint8_t *prec_map, int prec_groups, int G, int h, int *qmaxs)
+{
+    for (int g = 0; g < G; ++g) {
+        uint8_t bits = prec_groups > 1 ? prec_map[(size_t)h * G + g] : prec_map[h];
+        qmaxs[g] = qmax_of(bits);
+        if (qmaxs[g] < 0) return -1;
+    }
+    return 0;
+}
+
 /* ---------------------------------------------------- tile-parallel loop --- */
 
 typedef struct {
     int ntiles, d_k, d_v, group, update_kind, gate_kind, mode, nthreads, tid;
     int T; /* tokens per call (chunked update); 1 for a decode step */
+    int prec_groups; /* 1: prec_map [H]; G: prec_map [H][G] */
     const int32_t *tile_b, *tile_h;
     const uint8_t *prec_map;
     int8_t *codes;
@@ -205,22 +220,23 @@ static void *worker(void *arg)
     float *deq = (float *)malloc(n * sizeof(float));
     float *x = (float *)malloc(n * sizeof(float));
     float *w = (float *)malloc((size_t)d_v * sizeof(float));
-    if (!deq || !x || !w) {
-        free(deq); free(x); free(w);
+    int *qm = (int *)malloc((size_t)G * sizeof(int));
+    if (!deq || !x || !w || !qm) {
+        free(deq); free(x); free(w); free(qm);
         return (void *)1;
     }
     size_t gate_len = (W->gate_kind == ORC_GATE_PER_KEY) ? (size_t)d_k : 1;
     if (W->T > 1) {
         float *cur = (float *)malloc(n * sizeof(float));
         if (!cur) {
-            free(deq); free(x); free(w);
+            free(deq); free(x); free(w); free(qm);
             return (void *)1;
         }
         size_t NT = (size_t)W->ntiles;
         for (int t = W->tid; t < W->ntiles; t += W->nthreads) {
             int8_t *c = W->codes + (size_t)t * n;
             float *s = W->scales + (size_t)t * G * d_v;
-            int qmax = qmax_of(W->prec_map[W->tile_h[t]]);
+            head_qmaxs(W->prec_map, W->prec_groups, G, W->tile_h[t], qm);
             for (int i = 0; i < d_k; ++i)
                 for (int j = 0; j < d_v; ++j)
                     deq[i * d_v + j] = (float)c[i * d_v + j] * s[(i / W->group) * d_v + j];
@@ -235,10 +251,10 @@ static void *worker(void *arg)
             }
             /* one requantization at the chunk's end; BDR compares with the
              * state at the chunk's start */
-            requantize_tile(d_k, d_v, W->group, qmax, W->mode, cur, deq, c, s, W->seed, W->step,
+            requantize_tile(d_k, d_v, W->group, qm, W->mode, cur, deq, c, s, W->seed, W->step,
                             (uint32_t)W->tile_b[t], (uint32_t)W->tile_h[t]);
         }
-        free(cur); free(deq); free(x); free(w);
+        free(cur); free(deq); free(x); free(w); free(qm);
         return NULL;
     }
     for (int t = W->tid; t < W->ntiles; t += W->nthreads) {
@@ -251,7 +267,7 @@ static void *worker(void *arg)
         if (W->quantized) {
             int8_t *c = W->codes + (size_t)t * n;
             float *s = W->scales + (size_t)t * G * d_v;
-            int qmax = qmax_of(W->prec_map[W->tile_h[t]]);
+            head_qmaxs(W->prec_map, W->prec_groups, G, W->tile_h[t], qm);
             /* 1. dequantize with the value-axis group scales */
             for (int i = 0; i < d_k; ++i)
                 for (int j = 0; j < d_v; ++j)
@@ -259,7 +275,7 @@ static void *worker(void *arg)
             /* 2-3. update and output */
             update_tile(d_k, d_v, W->update_kind, W->gate_kind, deq, q, k, v, gate, beta, w, x, out);
             /* 4-5. new scales and codes */
-            requantize_tile(d_k, d_v, W->group, qmax, W->mode, x, deq, c, s, W->seed, W->step,
+            requantize_tile(d_k, d_v, W->group, qm, W->mode, x, deq, c, s, W->seed, W->step,
                             (uint32_t)W->tile_b[t], (uint32_t)W->tile_h[t]);
         } else {
             float *S = W->S + (size_t)t * n;
@@ -267,7 +283,7 @@ static void *worker(void *arg)
             memcpy(S, x, n * sizeof(float));
         }
     }
-    free(deq); free(x); free(w);
+    free(deq); free(x); free(w); free(qm);
     return NULL;
 }
 
@@ -304,29 +320,68 @@ static int run_tiles(work_t *proto, int nthreads)
 
 /* ------------------------------------------------------------ public --- */
 
-int orc_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int d_k, int d_v,
-             int group, int update_kind, int gate_kind, int mode, const uint8_t *prec_map,
-             int8_t *codes, float *scales, const float *q, const float *k, const float *v,
-             const float *gates, const float *beta, float *out, uint64_t seed, uint64_t step,
-             int nthreads)
+/* Validation shared by the quantized entry points: every tile's head has
+ * valid widths in prec_map (per head, or per (head, group)). */
+static int check_prec(int ntiles, const int32_t *tile_h, const uint8_t *prec_map, int prec_groups,
+                      int G)
 {
+    int *qm = (int *)malloc((size_t)G * sizeof(int));
+    if (!qm) return -2;
+    int rc = 0;
+    for (int t = 0; t < ntiles && rc == 0; ++t)
+        if (tile_h[t] < 0 || head_qmaxs(prec_map, prec_groups, G, tile_h[t], qm) != 0) rc = -1;
+    free(qm);
+    return rc;
+}
+
+static int step_impl(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int d_k, int d_v,
+                     int group, int update_kind, int gate_kind, int mode, const uint8_t *prec_map,
+                     int prec_groups, int8_t *codes, float *scales, int T, const float *q,
+                     const float *k, const float *v, const float *gates, const float *beta,
+                     float *out, uint64_t seed, uint64_t step, int nthreads)
+{
+    if (T < 1) return -1;
     if (ntiles < 0 || check_shape(d_k, d_v, group, update_kind, gate_kind) != 0) return -1;
     if (mode != ORC_ROUND_RTN && mode != ORC_ROUND_SR && mode != ORC_ROUND_BDR) return -1;
     if (ntiles == 0) return 0;
     if (!tile_b || !tile_h || !prec_map || !codes || !scales || !q || !k || !v || !gates || !out)
         return -1;
     if (update_kind == ORC_UPDATE_DELTA && !beta) return -1;
-    for (int t = 0; t < ntiles; ++t)
-        if (tile_h[t] < 0 || qmax_of(prec_map[tile_h[t]]) < 0) return -1;
+    int rc = check_prec(ntiles, tile_h, prec_map, prec_groups, d_k / group);
+    if (rc != 0) return rc;
     work_t W;
     memset(&W, 0, sizeof W);
     W.ntiles = ntiles; W.d_k = d_k; W.d_v = d_v; W.group = group;
-    W.update_kind = update_kind; W.gate_kind = gate_kind; W.mode = mode;
+    W.update_kind = update_kind; W.gate_kind = gate_kind; W.mode = mode; W.T = T;
+    W.prec_groups = prec_groups;
     W.tile_b = tile_b; W.tile_h = tile_h; W.prec_map = prec_map;
     W.codes = codes; W.scales = scales;
     W.q = q; W.k = k; W.v = v; W.gates = gates; W.beta = beta; W.out = out;
     W.seed = seed; W.step = step; W.quantized = 1;
     return run_tiles(&W, nthreads);
+}
+
+int orc_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int d_k, int d_v,
+             int group, int update_kind, int gate_kind, int mode, const uint8_t *prec_map,
+             int8_t *codes, float *scales, const float *q, const float *k, const float *v,
+             const float *gates, const float *beta, float *out, uint64_t seed, uint64_t step,
+             int nthreads)
+{
+    return step_impl(ntiles, tile_b, tile_h, d_k, d_v, group, update_kind, gate_kind, mode,
+                     prec_map, 1, codes, scales, 1, q, k, v, gates, beta, out, seed, step,
+                     nthreads);
+}
+
+int orc_step_pg(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int d_k, int d_v,
+                int group, int update_kind, int gate_kind, int mode, const uint8_t *prec_map,
+                int8_t *codes, float *scales, const float *q, const float *k, const float *v,
+                const float *gates, const float *beta, float *out, uint64_t seed, uint64_t step,
+                int nthreads)
+{
+    if (group <= 0) return -1;
+    return step_impl(ntiles, tile_b, tile_h, d_k, d_v, group, update_kind, gate_kind, mode,
+                     prec_map, d_k / group, codes, scales, 1, q, k, v, gates, beta, out, seed,
+                     step, nthreads);
 }
 
 int orc_chunk_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int d_k, int d_v,
@@ -335,27 +390,21 @@ int orc_chunk_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int
                    const float *v, const float *gates, const float *beta, float *out,
                    uint64_t seed, uint64_t step, int nthreads)
 {
-    if (T < 1) return -1;
-    if (T == 1)
-        return orc_step(ntiles, tile_b, tile_h, d_k, d_v, group, update_kind, gate_kind, mode,
-                        prec_map, codes, scales, q, k, v, gates, beta, out, seed, step, nthreads);
-    if (ntiles < 0 || check_shape(d_k, d_v, group, update_kind, gate_kind) != 0) return -1;
-    if (mode != ORC_ROUND_RTN && mode != ORC_ROUND_SR && mode != ORC_ROUND_BDR) return -1;
-    if (ntiles == 0) return 0;
-    if (!tile_b || !tile_h || !prec_map || !codes || !scales || !q || !k || !v || !gates || !out)
-        return -1;
-    if (update_kind == ORC_UPDATE_DELTA && !beta) return -1;
-    for (int t = 0; t < ntiles; ++t)
-        if (tile_h[t] < 0 || qmax_of(prec_map[tile_h[t]]) < 0) return -1;
-    work_t W;
-    memset(&W, 0, sizeof W);
-    W.ntiles = ntiles; W.d_k = d_k; W.d_v = d_v; W.group = group;
-    W.update_kind = update_kind; W.gate_kind = gate_kind; W.mode = mode; W.T = T;
-    W.tile_b = tile_b; W.tile_h = tile_h; W.prec_map = prec_map;
-    W.codes = codes; W.scales = scales;
-    W.q = q; W.k = k; W.v = v; W.gates = gates; W.beta = beta; W.out = out;
-    W.seed = seed; W.step = step; W.quantized = 1;
-    return run_tiles(&W, nthreads);
+    return step_impl(ntiles, tile_b, tile_h, d_k, d_v, group, update_kind, gate_kind, mode,
+                     prec_map, 1, codes, scales, T, q, k, v, gates, beta, out, seed, step,
+                     nthreads);
+}
+
+int orc_chunk_step_pg(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int d_k, int d_v,
+                      int group, int update_kind, int gate_kind, int mode, const uint8_t *prec_map,
+                      int8_t *codes, float *scales, int T, const float *q, const float *k,
+                      const float *v, const float *gates, const float *beta, float *out,
+                      uint64_t seed, uint64_t step, int nthreads)
+{
+    if (group <= 0) return -1;
+    return step_impl(ntiles, tile_b, tile_h, d_k, d_v, group, update_kind, gate_kind, mode,
+                     prec_map, d_k / group, codes, scales, T, q, k, v, gates, beta, out, seed,
+                     step, nthreads);
 }
 
 uint16_t orc_bf16_rne(float x)
@@ -403,8 +452,9 @@ int orc_fp32_step(int ntiles, int d_k, int d_v, int update_kind, int gate_kind, 
     return run_tiles(&W, nthreads);
 }
 
-int orc_import(int ntiles, const int32_t *tile_h, int d_k, int d_v, int group,
-               const uint8_t *prec_map, const float *S0, int8_t *codes, float *scales)
+static int import_impl(int ntiles, const int32_t *tile_h, int d_k, int d_v, int group,
+                       const uint8_t *prec_map, int prec_groups, const float *S0, int8_t *codes,
+                       float *scales)
 {
     if (ntiles < 0 || check_shape(d_k, d_v, group, ORC_UPDATE_GATED, ORC_GATE_SCALAR) != 0)
         return -1;
@@ -412,13 +462,32 @@ int orc_import(int ntiles, const int32_t *tile_h, int d_k, int d_v, int group,
     if (!tile_h || !prec_map || !S0 || !codes || !scales) return -1;
     size_t n = (size_t)d_k * d_v;
     int G = d_k / group;
-    for (int t = 0; t < ntiles; ++t) {
-        int qmax = qmax_of(prec_map[tile_h[t]]);
-        if (qmax < 0) return -1;
-        requantize_tile(d_k, d_v, group, qmax, ORC_ROUND_RTN, S0 + (size_t)t * n, NULL,
+    int *qm = (int *)malloc((size_t)G * sizeof(int));
+    if (!qm) return -2;
+    int rc = 0;
+    for (int t = 0; t < ntiles && rc == 0; ++t) {
+        if (tile_h[t] < 0 || head_qmaxs(prec_map, prec_groups, G, tile_h[t], qm) != 0) {
+            rc = -1;
+            break;
+        }
+        requantize_tile(d_k, d_v, group, qm, ORC_ROUND_RTN, S0 + (size_t)t * n, NULL,
                         codes + (size_t)t * n, scales + (size_t)t * G * d_v, 0, 0, 0, 0);
     }
-    return 0;
+    free(qm);
+    return rc;
+}
+
+int orc_import(int ntiles, const int32_t *tile_h, int d_k, int d_v, int group,
+               const uint8_t *prec_map, const float *S0, int8_t *codes, float *scales)
+{
+    return import_impl(ntiles, tile_h, d_k, d_v, group, prec_map, 1, S0, codes, scales);
+}
+
+int orc_import_pg(int ntiles, const int32_t *tile_h, int d_k, int d_v, int group,
+                  const uint8_t *prec_map, const float *S0, int8_t *codes, float *scales)
+{
+    if (group <= 0) return -1;
+    return import_impl(ntiles, tile_h, d_k, d_v, group, prec_map, d_k / group, S0, codes, scales);
 }
 
 int orc_dequant(int ntiles, int d_k, int d_v, int group, const int8_t *codes,

@@ -96,6 +96,23 @@ int orc_chunk_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h,
                    const float *q, const float *k, const float *v, const float *gates,
                    const float *beta, float *out, uint64_t seed, uint64_t step, int nthreads);
 
+/* Per-channel precision: the same three entry points with one width per
+ * (head, scale group) -- a block of `group` key channels -- in prec_map
+ * [H][G] (G = d_k / group) instead of one per head. Group g of head h is
+ * requantized with qmax of prec_map[h*G + g]. */
+int orc_step_pg(int ntiles, const int32_t *tile_b, const int32_t *tile_h,
+                int d_k, int d_v, int group, int update_kind, int gate_kind, int mode,
+                const uint8_t *prec_map, int8_t *codes, float *scales,
+                const float *q, const float *k, const float *v, const float *gates,
+                const float *beta, float *out, uint64_t seed, uint64_t step, int nthreads);
+int orc_chunk_step_pg(int ntiles, const int32_t *tile_b, const int32_t *tile_h,
+                      int d_k, int d_v, int group, int update_kind, int gate_kind, int mode,
+                      const uint8_t *prec_map, int8_t *codes, float *scales, int T,
+                      const float *q, const float *k, const float *v, const float *gates,
+                      const float *beta, float *out, uint64_t seed, uint64_t step, int nthreads);
+int orc_import_pg(int ntiles, const int32_t *tile_h, int d_k, int d_v, int group,
+                  const uint8_t *prec_map, const float *S0, int8_t *codes, float *scales);
+
 /* bfloat16 (the upper half of binary32: sign, 8 exponent bits, 7 fraction
  * bits) nearest to x, ties to the even fraction; NaN becomes a quiet NaN of the
  * same sign. Returns the 16-bit pattern. */
