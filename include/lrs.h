@@ -83,8 +83,10 @@ typedef struct {
  *
  * Code layout. One batch row holds the heads' tiles in head order; head h's
  * tile starts at byte head_offsets[h] of the row and has d_k*d_v*bits/8 bytes
- * (bits = prec_map[h]). Tile (b, h) starts at b*batch_stride_bytes +
- * head_offsets[h]. Inside a tile, lane t of 32 owns value columns
+ * (bits = prec_map[h]) -- or, for a state with one width per scale group
+ * (lrs_state_alloc_groups), the sum over its groups g of group*d_v*bits/8
+ * bytes with bits = prec_map[h*G + g], the groups' blocks in order. Tile
+ * (b, h) starts at b*batch_stride_bytes + head_offsets[h]. Inside a tile, lane t of 32 owns value columns
  * [t*C, t*C + C), C = d_v/32, for every key row. Its codes are ordered by
  * scale group, then by column pair p (columns t*C + 2p and t*C + 2p + 1),
  * then by key row, then by column within the pair; this byte stream is cut
@@ -101,7 +103,7 @@ typedef struct {
     lrs_shape shape;
     void *state_codes;
     float *scales;
-    uint8_t *prec_map;        /* [H], 4 or 8 */
+    uint8_t *prec_map;        /* [H], or [H][G] (lrs_state_alloc_groups); 4 or 8 */
     int64_t *head_offsets;    /* [H] */
     int64_t batch_stride_bytes;
     int64_t code_bytes;       /* batch * batch_stride_bytes */
@@ -122,6 +124,22 @@ lrs_status lrs_layout_query(const lrs_shape *shape, const uint8_t *prec_map_host
  * Synchronous. On failure *out is left zeroed. */
 lrs_status lrs_state_alloc(const lrs_shape *shape, const uint8_t *prec_map_host,
                            lrs_state *out);
+
+/* Per-channel precision ([LoReS] abstract: the decay-based width choice can
+ * protect slowly decaying heads or channels). The channel blocks are the
+ * scale groups: prec_map_host [H][G], G = d_k/group, gives each group of
+ * `group` key channels of each head its own width (4 or 8), so the tile's
+ * groups have different widths. Everything else as lrs_layout_query and
+ * lrs_state_alloc; every entry point that takes a prec_map then expects the
+ * [H][G] form for this state. The widths of a state are normally chosen by
+ * ranking the mean decay of each (head, key group) block: lrs_decay_head_means
+ * and lrs_precision_map with heads = H*G and inner = group on a per-key decay
+ * tensor [outer][H][d_k] (the same memory as [outer][H*G][group]). */
+lrs_status lrs_layout_query_groups(const lrs_shape *shape, const uint8_t *prec_map_host,
+                                   int64_t *head_offsets_host, int64_t *batch_stride_bytes,
+                                   int64_t *scale_count);
+lrs_status lrs_state_alloc_groups(const lrs_shape *shape, const uint8_t *prec_map_host,
+                                  lrs_state *out);
 
 /* Release everything lrs_state_alloc allocated and zero *st. NULL and
  * already-freed states are accepted. Synchronous. */

@@ -16,20 +16,11 @@ constexpr int kAuxWarps = 8;
 // Byte offset, inside a group block, of the 16-byte unit `u` of lane `lane`.
 __device__ __forceinline__ int unit_offset(int u, int lane) { return (u * 32 + lane) * 16; }
 
-struct TileRef {
-    uint8_t* codes;   // tile base
-    int prec;         // 4 or 8, 0 when the layout is inconsistent
-};
-
-__device__ __forceinline__ TileRef tile_ref(const LayoutArgs& a, int tile) {
-    const int h = tile % a.H, b = tile / a.H;
-    const int prec = a.prec_map[h];
-    const int64_t off = a.head_offsets[h];
-    const int64_t end = (h + 1 < a.H) ? a.head_offsets[h + 1] : a.batch_stride;
-    const int64_t bytes = static_cast<int64_t>(a.d_k) * a.d_v * prec / 8;
-    TileRef t;
-    t.prec = ((prec == 4 || prec == 8) && off >= 0 && off + bytes <= end) ? prec : 0;
-    t.codes = a.codes + static_cast<int64_t>(b) * a.batch_stride + off;
+// Layout of tile `tile` (b = tile / H, h = tile % H).
+__device__ __forceinline__ TileLayout tile_layout(const LayoutArgs& a, int tile) {
+    TileLayout t;
+    t.load(a.prec_map, a.head_offsets, a.batch_stride, a.H, a.pgroups, a.d_k / a.group,
+           a.group * a.d_v, tile / a.H, tile % a.H);
     return t;
 }
 
@@ -85,17 +76,17 @@ __device__ void decode_pair(const uint8_t* gcodes, int pc, int lane, float2 (&co
 
 enum { kOpFillZero, kOpImportFp32, kOpExportFp32, kOpExportCodes, kOpImportCodes };
 
+// One scale group g of one tile, codes of width BITS at gcodes.
 template <int C, int GROUP, int BITS>
-__device__ void layout_op_tile(const LayoutArgs& a, int op, int tile, uint8_t* tcodes,
-                               const float* S, float* So, int8_t* Co, const int8_t* Ci,
-                               const float* Si, int lane) {
+__device__ void layout_op_group(const LayoutArgs& a, int op, int tile, int g, uint8_t* gcodes,
+                                const float* S, float* So, int8_t* Co, const int8_t* Ci,
+                                const float* Si, int lane) {
     constexpr int DV = 32 * C;
     constexpr int P = C / 2;
     constexpr int QMAX = BITS == 8 ? 127 : 7;
     const int G = a.d_k / GROUP;
     const int64_t tile_elems = static_cast<int64_t>(a.d_k) * DV;
-    for (int g = 0; g < G; ++g) {
-        uint8_t* gcodes = tcodes + static_cast<int64_t>(g) * GROUP * DV * BITS / 8;
+    {
         float* gscales = a.scales + (static_cast<int64_t>(tile) * G + g) * DV;
         for (int pc = 0; pc < P; ++pc) {
             const int j = lane * C + 2 * pc;
@@ -158,6 +149,20 @@ __device__ void layout_op_tile(const LayoutArgs& a, int op, int tile, uint8_t* t
 }
 
 template <int C, int GROUP>
+__device__ void layout_op_tile(const LayoutArgs& a, int op, int tile, const TileLayout& tl,
+                               const float* S, float* So, int8_t* Co, const int8_t* Ci,
+                               const float* Si, int lane) {
+    constexpr int DV = 32 * C;
+    for (int g = 0; g < a.d_k / GROUP; ++g) {
+        uint8_t* gcodes = a.codes + tl.code_off + tl.goff(g, GROUP * DV / 2);
+        if (tl.bits(g) == 8)
+            layout_op_group<C, GROUP, 8>(a, op, tile, g, gcodes, S, So, Co, Ci, Si, lane);
+        else
+            layout_op_group<C, GROUP, 4>(a, op, tile, g, gcodes, S, So, Co, Ci, Si, lane);
+    }
+}
+
+template <int C, int GROUP>
 __global__ void __launch_bounds__(kAuxWarps * 32) layout_kernel(const LayoutArgs a, int op,
                                                                  const float* S, float* So,
                                                                  int8_t* Co, const int8_t* Ci,
@@ -166,15 +171,12 @@ __global__ void __launch_bounds__(kAuxWarps * 32) layout_kernel(const LayoutArgs
     const int ntiles = a.B * a.H;
     for (int tile = blockIdx.x * kAuxWarps + (threadIdx.x >> 5); tile < ntiles;
          tile += gridDim.x * kAuxWarps) {
-        const TileRef t = tile_ref(a, tile);
-        if (t.prec == 0) {
+        const TileLayout t = tile_layout(a, tile);
+        if (!t.ok) {
             if (lane == 0) atomicOr(a.err, kErrLayout);
             continue;
         }
-        if (t.prec == 8)
-            layout_op_tile<C, GROUP, 8>(a, op, tile, t.codes, S, So, Co, Ci, Si, lane);
-        else
-            layout_op_tile<C, GROUP, 4>(a, op, tile, t.codes, S, So, Co, Ci, Si, lane);
+        layout_op_tile<C, GROUP>(a, op, tile, t, S, So, Co, Ci, Si, lane);
     }
 }
 

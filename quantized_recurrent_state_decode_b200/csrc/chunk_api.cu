@@ -106,6 +106,7 @@ lrs_status lrs_chunk_step(const lrs_state* st, void* state_codes, float* scales,
     p.H = sh.heads;
     p.ntiles = static_cast<int32_t>(ntiles);
     p.T = T;
+    p.pgroups = lrs::state_prec_groups(st);
     p.inject = lrs::take_injected_timeout(&p.timeout_ns) ? 1 : 0;
     const int grid = static_cast<int>(std::min<int64_t>(ntiles, int64_t(sms) * per_sm));
     void* args[] = {&p};

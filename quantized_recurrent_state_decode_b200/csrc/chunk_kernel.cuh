@@ -44,6 +44,7 @@ struct ChunkParams {
     unsigned* err;
     uint64_t timeout_ns;
     int32_t H, ntiles, T, inject;
+    int32_t pgroups;      // widths in prec_map per head (1) or per (head, group) (G)
 };
 
 // Shared memory of one CTA: barriers | codes (int8 capacity) | scales |
@@ -69,25 +70,26 @@ struct ColumnPlace {
 };
 
 // Byte offset, inside the tile's codes, of the 16-byte unit `un` of the pair
-// `pc` of owner lane `owner` in scale group g (precision BITS).
-template <int GROUP, int DV, int BITS>
-__device__ __forceinline__ int unit_byte(int g, int pc, int un, int owner) {
+// `pc` of owner lane `owner` in the scale group whose codes start at gbase.
+template <int GROUP, int BITS>
+__device__ __forceinline__ int unit_byte(int gbase, int pc, int un, int owner) {
     using PG = PairGeo<GROUP, BITS>;
-    return g * GROUP * DV * BITS / 8 + ((pc * PG::UNITS + un) * 32 + owner) * 16;
+    return gbase + ((pc * PG::UNITS + un) * 32 + owner) * 16;
 }
 
-// Dequantize scale group g of column j: y[i - g*GROUP] = RN(code_ij * s[g][j]).
+// Dequantize one scale group (codes at gbase, scale row g) of column j:
+// y[r] = RN(code * s[g][j]) for the group's rows r.
 template <int DV, int GROUP, int BITS>
 __device__ __forceinline__ void decode_group(const uint8_t* cs, const float* ss,
-                                             const ColumnPlace& cp, int j, int g,
+                                             const ColumnPlace& cp, int j, int g, int gbase,
                                              float (&y)[GROUP]) {
     using PG = PairGeo<GROUP, BITS>;
     constexpr float K = kTwo23 + Q<BITS>::kBias;
     const float s = ss[g * DV + j];
 #pragma unroll
     for (int un = 0; un < PG::UNITS; ++un) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(
-            cs + unit_byte<GROUP, DV, BITS>(g, cp.pc, un, cp.owner));
+        const uint4 raw =
+            *reinterpret_cast<const uint4*>(cs + unit_byte<GROUP, BITS>(gbase, cp.pc, un, cp.owner));
         const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
@@ -109,32 +111,37 @@ __device__ __forceinline__ void decode_group(const uint8_t* cs, const float* ss,
     }
 }
 
-// Dequantize column j: x[i] = RN(code_ij * s[g][j]).
-template <int DK, int DV, int GROUP, int BITS>
+// Dequantize column j: x[i] = RN(code_ij * s[g][j]), each group at its width.
+template <int DK, int DV, int GROUP>
 __device__ __forceinline__ void decode_column(const uint8_t* cs, const float* ss,
-                                              const ColumnPlace& cp, int j, float (&x)[DK]) {
+                                              const ColumnPlace& cp, int j, const TileLayout& tl,
+                                              float (&x)[DK]) {
 #pragma unroll
     for (int g = 0; g < DK / GROUP; ++g) {
         float y[GROUP];
-        decode_group<DV, GROUP, BITS>(cs, ss, cp, j, g, y);
+        const int gbase = static_cast<int>(tl.goff(g, GROUP * DV / 2));
+        if (tl.bits(g) == 8)
+            decode_group<DV, GROUP, 8>(cs, ss, cp, j, g, gbase, y);
+        else
+            decode_group<DV, GROUP, 4>(cs, ss, cp, j, g, gbase, y);
 #pragma unroll
         for (int r = 0; r < GROUP; ++r) x[g * GROUP + r] = y[r];
     }
 }
 
-// Stored bytes (int8) or nibbles (int4) of column j, already rounded (t[i]:
-// float whose low bits are the stored value), written into the tile's codes
-// in the state layout. Columns c0 = 2m and c1 = 2m + 1 of a pair are adjacent
-// threads: each packs four of its rows, the two trade them with one shuffle,
-// and each writes one of the two words that cover those rows.
-template <int DK, int DV, int GROUP, int BITS>
-__device__ __forceinline__ void store_column(uint8_t* cs, const ColumnPlace& cp,
-                                             const float (&t)[DK]) {
+// Stored bytes (int8) or nibbles (int4) of one group of column j, already
+// rounded (t[r]: float whose low bits are the stored value), written into the
+// tile's codes in the state layout. Columns c0 = 2m and c1 = 2m + 1 of a pair
+// are adjacent threads: each packs four (int8) or eight (int4) of its rows,
+// the two trade them with one shuffle, and each writes one of the two words
+// that cover those rows.
+template <int DV, int GROUP, int BITS>
+__device__ __forceinline__ void store_group(uint8_t* cs, const ColumnPlace& cp, int gbase,
+                                            const float* t) {
     using PG = PairGeo<GROUP, BITS>;
-    // my stored values of rows r..r+3 (int8, one per byte) or r..r+7 (int4)
     constexpr int RPP = BITS == 8 ? 4 : 8;         // rows per packed word
 #pragma unroll
-    for (int r = 0; r < DK; r += RPP) {
+    for (int r = 0; r < GROUP; r += RPP) {
         uint32_t m;
         if constexpr (BITS == 8) {
             m = pack_low_bytes(t[r], t[r + 1], t[r + 2], t[r + 3]);
@@ -150,45 +157,41 @@ __device__ __forceinline__ void store_column(uint8_t* cs, const ColumnPlace& cp,
         // c0 writes the word of the first half of the rows, c1 of the second;
         // byte order within a word: (row, c0), (row, c1), (row+1, c0), ...
         const uint32_t word = cp.cc == 0 ? __byte_perm(m, p, 0x5140u) : __byte_perm(m, p, 0x3726u);
-        const int rw = r + cp.cc * (RPP / 2);      // first row of the word written
-        const int g = rw / GROUP, rr = rw % GROUP;
+        const int rr = r + cp.cc * (RPP / 2);      // first row (in the group) of the word written
         const int un = rr / PG::RPU, w = (rr % PG::RPU) / PG::RPW;
-        *reinterpret_cast<uint32_t*>(cs + unit_byte<GROUP, DV, BITS>(g, cp.pc, un, cp.owner) +
+        *reinterpret_cast<uint32_t*>(cs + unit_byte<GROUP, BITS>(gbase, cp.pc, un, cp.owner) +
                                      w * 4) = word;
     }
 }
 
-// New scales of column j, and its codes (as floats kTwo23 + bias + code, in
-// t, replacing x) by the rounding MODE. deq0 is decoded again from the old
-// codes and scales for BDR.
+// New scale of one group of column j, and its codes (as floats kTwo23 + bias
+// + code, in x[g*GROUP ...], replacing the values) by the rounding MODE. For
+// BDR the group's old values are decoded again from the old codes and scales.
 template <int DK, int DV, int GROUP, int MODE, int BITS>
-__device__ __forceinline__ void requantize_column(float (&x)[DK], float (&snew)[DK / GROUP],
-                                                  const uint8_t* cs, const float* ss,
-                                                  const ColumnPlace& cp, int j, uint64_t hkey) {
+__device__ __forceinline__ float requantize_group(float (&x)[DK], int g, const uint8_t* cs,
+                                                  const float* ss, const ColumnPlace& cp, int j,
+                                                  int gbase, uint64_t hkey) {
     constexpr float QMAX = Q<BITS>::kMax, BIAS = Q<BITS>::kBias;
     constexpr int QM = static_cast<int>(QMAX);
+    float deq0[GROUP];
+    if constexpr (MODE == kBDR) decode_group<DV, GROUP, BITS>(cs, ss, cp, j, g, gbase, deq0);
+    float A = 0.0f;
 #pragma unroll
-    for (int g = 0; g < DK / GROUP; ++g) {
-        float deq0[GROUP];
-        if constexpr (MODE == kBDR) decode_group<DV, GROUP, BITS>(cs, ss, cp, j, g, deq0);
-        float A = 0.0f;
+    for (int r = g * GROUP; r < (g + 1) * GROUP; r += 2) A = max_abs3(A, x[r], x[r + 1]);
+    const float s = A < kTiny ? 0.0f : div_by_qmax<QM>(A);
+    const float inv = A < kTiny ? 0.0f : div_rn_fast(QMAX, A);
+    const float2 inv2 = f2(inv), s2 = f2(s), kb = f2(kTwo23 + BIAS);
 #pragma unroll
-        for (int r = g * GROUP; r < (g + 1) * GROUP; r += 2) A = max_abs3(A, x[r], x[r + 1]);
-        const float s = A < kTiny ? 0.0f : div_by_qmax<QM>(A);
-        const float inv = A < kTiny ? 0.0f : div_rn_fast(QMAX, A);
-        snew[g] = s;
-        const float2 inv2 = f2(inv), s2 = f2(s), kb = f2(kTwo23 + BIAS);
-#pragma unroll
-        for (int r = g * GROUP; r < (g + 1) * GROUP; r += 2) {
-            const int rl = r - g * GROUP;
-            const float2 d0 = MODE == kBDR ? make_float2(deq0[rl], deq0[rl + 1]) : f2(0.0f);
-            const float2 tv = round_rows<MODE, BITS>(make_float2(x[r], x[r + 1]), inv2, d0, s2,
-                                                     kb, hkey, static_cast<uint32_t>(r),
-                                                     static_cast<uint32_t>(j));
-            x[r] = tv.x;
-            x[r + 1] = tv.y;
-        }
+    for (int r = g * GROUP; r < (g + 1) * GROUP; r += 2) {
+        const int rl = r - g * GROUP;
+        const float2 d0 = MODE == kBDR ? make_float2(deq0[rl], deq0[rl + 1]) : f2(0.0f);
+        const float2 tv = round_rows<MODE, BITS>(make_float2(x[r], x[r + 1]), inv2, d0, s2, kb,
+                                                 hkey, static_cast<uint32_t>(r),
+                                                 static_cast<uint32_t>(j));
+        x[r] = tv.x;
+        x[r + 1] = tv.y;
     }
+    return s;
 }
 
 // Token t of the tile into ring slot `slot` (thread 0 only).
@@ -220,19 +223,6 @@ __device__ __forceinline__ float4 lds4(const float* p) {
     return r;
 }
 
-// Layout of tile `tile` (b = tile / H, h = tile % H): byte offset of its
-// codes and its precision, or 0 when prec_map does not fit the offsets.
-__device__ __forceinline__ int tile_layout(const ChunkParams& p, int tile, int dk, int dv,
-                                           int64_t* code_off) {
-    const int b = tile / p.H, h = tile - (tile / p.H) * p.H;
-    const int pr = __ldg(p.prec_map + h);
-    const int64_t off = __ldg(p.head_offsets + h);
-    const int64_t end = (h + 1 < p.H) ? __ldg(p.head_offsets + h + 1) : p.batch_stride;
-    const int64_t bytes = static_cast<int64_t>(dk) * dv * pr / 8;
-    *code_off = static_cast<int64_t>(b) * p.batch_stride + off;
-    return ((pr == 4 || pr == 8) && off >= 0 && off + bytes <= end) ? pr : 0;
-}
-
 template <int DK, int DV, int GROUP, int UPD, int GATE, int MODE>
 __global__ void __launch_bounds__(DV, (3 * 128) / DV) chunk_kernel(const ChunkParams p) {
     using S = ChunkSmem<DK, DV, GROUP, GATE>;
@@ -262,13 +252,15 @@ __global__ void __launch_bounds__(DV, (3 * 128) / DV) chunk_kernel(const ChunkPa
     bool state_pending = false;  // the state copy may still be in flight
 
     for (int tile = blockIdx.x; tile < p.ntiles && ok; tile += gridDim.x) {
-        int64_t code_off = 0;
-        const int prec = tile_layout(p, tile, DK, DV, &code_off);
-        if (prec == 0) {
+        TileLayout tl;
+        tl.load(p.prec_map, p.head_offsets, p.batch_stride, p.H, p.pgroups, G, GROUP * DV,
+                tile / p.H, tile % p.H);
+        if (!tl.ok) {
             if (j == 0) atomicOr(p.err, kErrLayout);
             continue;
         }
-        const uint32_t cbytes = DK * DV * prec / 8;
+        const int64_t code_off = tl.code_off;
+        const uint32_t cbytes = static_cast<uint32_t>(tl.goff(G, GROUP * DV / 2));
         if (j == 0 && !p.inject) {
             // the previous tile's shared-memory reads come before these copies
             fence_proxy_async_smem();
@@ -291,10 +283,7 @@ __global__ void __launch_bounds__(DV, (3 * 128) / DV) chunk_kernel(const ChunkPa
         par_state ^= 1u;
 
         float x[DK];
-        if (prec == 8)
-            decode_column<DK, DV, GROUP, 8>(cs, ss, cp, j, x);
-        else
-            decode_column<DK, DV, GROUP, 4>(cs, ss, cp, j, x);
+        decode_column<DK, DV, GROUP>(cs, ss, cp, j, tl, x);
 
         // Delta rule: u_t = k_t^T S_{t-1} in key order. u_0 is taken here from
         // the dequantized state; u_{t+1} is accumulated while token t updates
@@ -408,15 +397,22 @@ __global__ void __launch_bounds__(DV, (3 * 128) / DV) chunk_kernel(const ChunkPa
                                                           static_cast<uint32_t>(b),
                                                           static_cast<uint32_t>(h))
                                           : 0ull;
-        if (prec == 8)
-            requantize_column<DK, DV, GROUP, MODE, 8>(x, snew, cs, ss, cp, j, hkey);
-        else
-            requantize_column<DK, DV, GROUP, MODE, 4>(x, snew, cs, ss, cp, j, hkey);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const int gbase = static_cast<int>(tl.goff(g, GROUP * DV / 2));
+            snew[g] = tl.bits(g) == 8
+                          ? requantize_group<DK, DV, GROUP, MODE, 8>(x, g, cs, ss, cp, j, gbase, hkey)
+                          : requantize_group<DK, DV, GROUP, MODE, 4>(x, g, cs, ss, cp, j, gbase, hkey);
+        }
         __syncthreads();                     // old codes and scales no longer read
-        if (prec == 8)
-            store_column<DK, DV, GROUP, 8>(cs, cp, x);
-        else
-            store_column<DK, DV, GROUP, 4>(cs, cp, x);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const int gbase = static_cast<int>(tl.goff(g, GROUP * DV / 2));
+            if (tl.bits(g) == 8)
+                store_group<DV, GROUP, 8>(cs, cp, gbase, x + g * GROUP);
+            else
+                store_group<DV, GROUP, 4>(cs, cp, gbase, x + g * GROUP);
+        }
 #pragma unroll
         for (int g = 0; g < G; ++g) ss[g * DV + j] = snew[g];
         __syncthreads();

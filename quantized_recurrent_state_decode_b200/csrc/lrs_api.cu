@@ -100,6 +100,7 @@ constexpr int kDefaultSlots = 2;
 
 struct StatePriv {
     int device = -1;
+    int pgroups = 1;    // widths per head (1) or per (head, scale group) (G)
     std::vector<uint8_t> prec_host;
     std::vector<int64_t> offsets_host;
     // device staging for lrs_decode_step_host (allocated on first use)
@@ -134,17 +135,26 @@ lrs_status check_shape(const lrs_shape* s) {
     return LRS_OK;
 }
 
-lrs_status compute_layout(const lrs_shape* s, const uint8_t* prec, int64_t* offsets,
+// Head offsets within a batch row for widths per head (pgroups == 1,
+// prec [H]) or per (head, scale group) (pgroups == G, prec [H][G]).
+lrs_status compute_layout(const lrs_shape* s, const uint8_t* prec, int pgroups, int64_t* offsets,
                           int64_t* stride, int64_t* scale_count) {
     lrs_status st = check_shape(s);
     if (st != LRS_OK) return st;
     if (!prec) return fail(LRS_ERR_INVALID_ARG, "prec_map is NULL");
+    const int G = s->d_k / s->group;
+    if (pgroups != 1 && pgroups != G)
+        return fail(LRS_ERR_INVALID_ARG, "widths per head or per scale group only");
     int64_t off = 0;
     for (int h = 0; h < s->heads; ++h) {
-        if (prec[h] != 4 && prec[h] != 8)
-            return fail(LRS_ERR_INVALID_ARG, "prec_map[%d]=%d (must be 4 or 8)", h, prec[h]);
         if (offsets) offsets[h] = off;
-        off += static_cast<int64_t>(s->d_k) * s->d_v * prec[h] / 8;
+        for (int g = 0; g < G; ++g) {
+            const int w = pgroups == 1 ? prec[h] : prec[static_cast<int64_t>(h) * G + g];
+            if (w != 4 && w != 8)
+                return fail(LRS_ERR_INVALID_ARG, "prec_map width %d at head %d group %d "
+                            "(must be 4 or 8)", w, h, g);
+            off += static_cast<int64_t>(s->group) * s->d_v * w / 8;
+        }
     }
     if (stride) *stride = off;
     if (scale_count)
@@ -176,6 +186,7 @@ lrs::LayoutArgs layout_args(const lrs_state* st, unsigned* err) {
     a.d_k = st->shape.d_k;
     a.d_v = st->shape.d_v;
     a.group = st->shape.group;
+    a.pgroups = static_cast<const StatePriv*>(st->priv)->pgroups;
     a.err = err;
     return a;
 }
@@ -208,10 +219,12 @@ const void* find_step_kernel(int C, int group, int update_kind, int gate_kind, i
     }
 }
 
-int step_warp_smem(int C, int group, int gate_kind, int slots, int mode, int io, int d_k) {
+int step_warp_smem(int C, int group, int update_kind, int gate_kind, int slots, int mode, int io,
+                   int d_k) {
     const bool xs = stage_x(mode);
-#define LRS_SLOT_IO(CC, GG, IO)                                                              \
-    return gate_kind == kGatePerKey ? Slot<CC, GG, kGatePerKey, IO>::warp_bytes(slots, xs, d_k) \
+#define LRS_SLOT_IO(CC, GG, IO)                                                                   \
+    if (update_kind == kDelta) return Slot<CC, GG, kGate, IO, true>::warp_bytes(slots, xs, d_k);   \
+    return gate_kind == kGatePerKey ? Slot<CC, GG, kGatePerKey, IO>::warp_bytes(slots, xs, d_k)   \
                                     : Slot<CC, GG, kGate, IO>::warp_bytes(slots, xs, d_k);
 #define LRS_SLOT(CC, GG)                                                                     \
     if (C == CC && group == GG) {                                                            \
@@ -256,27 +269,42 @@ int32_t lrs_version(void) { return LRS_VERSION; }
 lrs_status lrs_layout_query(const lrs_shape* shape, const uint8_t* prec_map_host,
                             int64_t* head_offsets_host, int64_t* batch_stride_bytes,
                             int64_t* scale_count) {
-    lrs_status s = compute_layout(shape, prec_map_host, head_offsets_host, batch_stride_bytes,
+    lrs_status s = compute_layout(shape, prec_map_host, 1, head_offsets_host, batch_stride_bytes,
                                   scale_count);
     return s == LRS_OK ? ok() : s;
 }
 
-lrs_status lrs_state_alloc(const lrs_shape* shape, const uint8_t* prec_map_host, lrs_state* out) {
+lrs_status lrs_layout_query_groups(const lrs_shape* shape, const uint8_t* prec_map_host,
+                                   int64_t* head_offsets_host, int64_t* batch_stride_bytes,
+                                   int64_t* scale_count) {
+    lrs_status s = check_shape(shape);
+    if (s != LRS_OK) return s;
+    s = compute_layout(shape, prec_map_host, shape->d_k / shape->group, head_offsets_host,
+                       batch_stride_bytes, scale_count);
+    return s == LRS_OK ? ok() : s;
+}
+
+}  // extern "C"
+
+static lrs_status state_alloc(const lrs_shape* shape, const uint8_t* prec_map_host, int pgroups,
+                              lrs_state* out) {
     if (!out) return fail(LRS_ERR_INVALID_ARG, "out is NULL");
     memset(out, 0, sizeof *out);
     lrs_status s = check_shape(shape);
     if (s != LRS_OK) return s;
     std::vector<int64_t> offs(shape->heads);
     int64_t stride = 0, nscales = 0;
-    s = compute_layout(shape, prec_map_host, offs.data(), &stride, &nscales);
+    s = compute_layout(shape, prec_map_host, pgroups, offs.data(), &stride, &nscales);
     if (s != LRS_OK) return s;
     DeviceCtx* ctx = nullptr;
     s = device_ctx(&ctx);
     if (s != LRS_OK) return s;
+    const int nprec = shape->heads * pgroups;
 
     StatePriv* pv = new StatePriv;
     cudaGetDevice(&pv->device);
-    pv->prec_host.assign(prec_map_host, prec_map_host + shape->heads);
+    pv->pgroups = pgroups;
+    pv->prec_host.assign(prec_map_host, prec_map_host + nprec);
     pv->offsets_host = offs;
 
     lrs_state st;
@@ -299,11 +327,11 @@ lrs_status lrs_state_alloc(const lrs_shape* shape, const uint8_t* prec_map_host,
         return cleanup(e, "cudaMalloc(codes)");
     if ((e = cudaMalloc(&st.scales, std::max<int64_t>(nscales, 4) * sizeof(float))) != cudaSuccess)
         return cleanup(e, "cudaMalloc(scales)");
-    if ((e = cudaMalloc(&st.prec_map, std::max(shape->heads, 16))) != cudaSuccess)
+    if ((e = cudaMalloc(&st.prec_map, std::max(nprec, 16))) != cudaSuccess)
         return cleanup(e, "cudaMalloc(prec_map)");
     if ((e = cudaMalloc(&st.head_offsets, shape->heads * sizeof(int64_t))) != cudaSuccess)
         return cleanup(e, "cudaMalloc(head_offsets)");
-    if ((e = cudaMemcpy(st.prec_map, prec_map_host, shape->heads, cudaMemcpyHostToDevice)) !=
+    if ((e = cudaMemcpy(st.prec_map, prec_map_host, nprec, cudaMemcpyHostToDevice)) !=
         cudaSuccess)
         return cleanup(e, "cudaMemcpy(prec_map)");
     if ((e = cudaMemcpy(st.head_offsets, offs.data(), shape->heads * sizeof(int64_t),
@@ -314,6 +342,22 @@ lrs_status lrs_state_alloc(const lrs_shape* shape, const uint8_t* prec_map_host,
     if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cleanup(e, "zero fill");
     *out = st;
     return ok();
+}
+
+extern "C" {
+
+lrs_status lrs_state_alloc(const lrs_shape* shape, const uint8_t* prec_map_host, lrs_state* out) {
+    return state_alloc(shape, prec_map_host, 1, out);
+}
+
+lrs_status lrs_state_alloc_groups(const lrs_shape* shape, const uint8_t* prec_map_host,
+                                  lrs_state* out) {
+    if (!shape) return fail(LRS_ERR_INVALID_ARG, "shape is NULL");
+    if (!out) return fail(LRS_ERR_INVALID_ARG, "out is NULL");
+    memset(out, 0, sizeof *out);
+    lrs_status s = check_shape(shape);
+    if (s != LRS_OK) return s;
+    return state_alloc(shape, prec_map_host, shape->d_k / shape->group, out);
 }
 
 lrs_status lrs_state_free(lrs_state* st) {
@@ -374,7 +418,8 @@ static lrs_status decode_step_io(const lrs_state* st, void* state_codes, float* 
         slots = std::min(slots, G);
     }
     slots = std::max(1, std::min(slots, lrs::kMaxSlots));
-    const int warp_smem = lrs::step_warp_smem(C, sh.group, sh.gate_kind, slots, mode, io, sh.d_k);
+    const int warp_smem = lrs::step_warp_smem(C, sh.group, sh.update_kind, sh.gate_kind, slots, mode, io,
+                                              sh.d_k);
     constexpr int kSmemLimit = 227 * 1024;
     int warps = step_warps_override();
     if (warps <= 0) warps = kDefaultWarps;
@@ -441,6 +486,7 @@ static lrs_status decode_step_io(const lrs_state* st, void* state_codes, float* 
     p.d_k = sh.d_k;
     p.G = G;
     p.ntiles = ntiles;
+    p.pgroups = static_cast<const StatePriv*>(st->priv)->pgroups;
     p.warp_smem = warp_smem;
     p.slots = slots;
     p.inject = 0;
@@ -711,5 +757,9 @@ lrs_status api_fail(lrs_status s, const char* msg) { return fail(s, "%s", msg); 
 lrs_status api_cuda_fail(cudaError_t e, const char* what) { return cuda_fail(e, what); }
 lrs_status api_ok() { return ok(); }
 lrs_status api_check_state(const lrs_state* st) { return check_state(st); }
+
+int state_prec_groups(const lrs_state* st) {
+    return static_cast<const StatePriv*>(st->priv)->pgroups;
+}
 
 }  // namespace lrs

@@ -25,7 +25,8 @@ const void* find_step_kernel_bdr_bf16(int C, int group, int update_kind, int gat
 
 // Bytes of shared memory one warp of the step kernel uses with `slots` ring
 // slots in rounding mode `mode` with I/O element type `io` and d_k key rows.
-int step_warp_smem(int C, int group, int gate_kind, int slots, int mode, int io, int d_k);
+int step_warp_smem(int C, int group, int update_kind, int gate_kind, int slots, int mode, int io,
+                   int d_k);
 
 // The chunked-update kernel for one shape and rounding mode, with the bytes
 // of shared memory it takes per CTA ({nullptr, 0} when not compiled).
@@ -44,6 +45,7 @@ struct LayoutArgs {
     const int64_t* head_offsets;
     int64_t batch_stride;
     int32_t B, H, d_k, d_v, group;
+    int32_t pgroups;        // widths in prec_map per head (1) or per (head, group) (G)
     unsigned* err;
 };
 
@@ -72,5 +74,8 @@ lrs_status api_fail(lrs_status s, const char* msg);
 lrs_status api_cuda_fail(cudaError_t e, const char* what);
 lrs_status api_ok();
 lrs_status api_check_state(const lrs_state* st);
+
+// Widths per head (1) or per (head, scale group) (G) of an allocated state.
+int state_prec_groups(const lrs_state* st);
 
 }  // namespace lrs

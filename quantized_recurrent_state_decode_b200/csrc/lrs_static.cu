@@ -120,7 +120,8 @@ extern "C" lrs_status lrs_decode_step_host_noalloc(const lrs_state* st, const fl
     // for the delta rule, two slots otherwise, up to the variant's warps)
     int slots = delta ? G : std::min(2, G);
     slots = std::max(1, std::min(slots, lrs::kMaxSlots));
-    const int warp_smem = lrs::step_warp_smem(C, sh.group, sh.gate_kind, slots, mode, lrs::kStepIoF32, sh.d_k);
+    const int warp_smem = lrs::step_warp_smem(C, sh.group, sh.update_kind, sh.gate_kind, slots, mode,
+                                              lrs::kStepIoF32, sh.d_k);
     constexpr int kSmemLimit = 227 * 1024;
     int warps = std::min(12, std::max(1, kSmemLimit / warp_smem));
     warps = std::min(warps, lrs::step_max_warps(sh.group, mode));
@@ -160,6 +161,7 @@ extern "C" lrs_status lrs_decode_step_host_noalloc(const lrs_state* st, const fl
     p.d_k = sh.d_k;
     p.G = G;
     p.ntiles = ntiles;
+    p.pgroups = lrs::state_prec_groups(st);
     p.slots = slots;
     p.warp_smem = warp_smem;
     p.inject = 0;

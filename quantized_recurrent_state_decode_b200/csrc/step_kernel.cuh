@@ -52,30 +52,39 @@ struct StepParams {
     unsigned* err;
     uint64_t timeout_ns;
     int32_t H, d_k, G, ntiles;
+    int32_t pgroups;     // widths in prec_map per head: 1, or one per scale group: G
     int32_t slots;       // ring slots per warp, 1..min(G, 16); the delta rule needs G
     int32_t warp_smem;   // bytes of shared memory per warp
     int32_t inject;      // fault injection: issue no copies
 };
 
-// Shared-memory layout of one warp (ES = bytes of a q, k, v element):
+// Shared-memory layout of one warp (ES = bytes of a q, k, v element).
+// Gated forms (INS = false):
 //   [0, 128)          mbarriers, one per slot
 //   two tile-input buffers of tile_in_bytes(d_k) each, used by the warp's
 //   tiles in turn (tile n in buffer n & 1):
 //     q, k (d_k elements each) | [gate] (d_k fp32) | v (d_v elements)
 //   then `slots` slots of kBytes each, one scale group per item:
 //     codes (GROUP*d_v bytes: room for int8) | scales (d_v fp32)
-//   then, for SR and BDR, the x staging buffer.
 // A tile's inputs come with its first group, in one bulk copy per array.
-template <int C, int GROUP, int GATE, int IO = kIoF32>
+// Delta rule (INS = true; its ring holds a whole tile, and the shared memory
+// of 8 warps leaves no room for two more tiles' inputs):
+//   [0, 128) mbarriers | v (d_v elements, one buffer: read before the tile's
+//   groups are, refilled with the next tile's first group) | slots of kBytes:
+//     codes | scales (d_v fp32) | q, k (GROUP elements each)
+// In both, SR and BDR add the x staging buffer at the end.
+template <int C, int GROUP, int GATE, int IO = kIoF32, bool INS = false>
 struct Slot {
     static constexpr int DV = 32 * C;
     static constexpr int ES = IO == kIoBF16 ? 2 : 4;
     static constexpr int kCodes = GROUP * DV;                     // int8 capacity
     static constexpr int kScales = kCodes;
-    static constexpr int kBytes = kScales + DV * 4;
+    static constexpr int kQ = kScales + DV * 4;                   // INS only
+    static constexpr int kK = kQ + GROUP * ES;                    // INS only
+    static constexpr int kBytes = INS ? kK + GROUP * ES : kQ;
     static_assert(kBytes % 16 == 0, "slot alignment");
     static constexpr int kXsBytes = GROUP * 256;   // x staging (SR, BDR): 16 B per row pair and lane
-    // offsets inside a tile-input buffer
+    // offsets inside a tile-input buffer (!INS)
     __host__ __device__ static int in_k(int d_k) { return d_k * ES; }
     __host__ __device__ static int in_g(int d_k) { return 2 * d_k * ES; }
     __host__ __device__ static int in_v(int d_k) {
@@ -85,7 +94,9 @@ struct Slot {
     __host__ __device__ static int tile_in_bytes(int d_k) {
         return (tile_in_payload(d_k) + 15) / 16 * 16;
     }
-    __host__ __device__ static int header(int d_k) { return 128 + 2 * tile_in_bytes(d_k); }
+    __host__ __device__ static int header(int d_k) {
+        return INS ? 128 + DV * ES : 128 + 2 * tile_in_bytes(d_k);
+    }
     static int warp_bytes(int slots, bool xs, int d_k) {
         return (header(d_k) + slots * kBytes + (xs ? kXsBytes : 0) + 127) / 128 * 128;
     }
@@ -517,15 +528,53 @@ __device__ __forceinline__ void pair_step(const uint8_t* __restrict__ cs, int ub
     }
 }
 
+// Where one tile's codes live and how wide each scale group's codes are.
+// prec_map holds a width (4 or 8) per head (pgroups == 1) or per (head,
+// group) in [H][G] order (pgroups == G); a head's groups are consecutive
+// blocks of GROUP*d_v*width/8 bytes at head_offsets[h] within the batch row.
+struct TileLayout {
+    int64_t code_off;    // byte offset of the tile's codes
+    uint32_t mask8;      // bit g set: group g is int8 (else int4); G <= 16
+    bool ok;             // the widths are valid and fit the head's offsets
+
+    __device__ __forceinline__ int bits(int g) const { return (mask8 >> g) & 1u ? 8 : 4; }
+    // byte offset of group g inside the tile; half = GROUP*d_v/2 (an int4 group)
+    __device__ __forceinline__ int64_t goff(int g, int half) const {
+        return static_cast<int64_t>(half) * (g + __popc(mask8 & ((1u << g) - 1u)));
+    }
+    __device__ __forceinline__ void load(const uint8_t* prec_map, const int64_t* head_offsets,
+                                         int64_t batch_stride, int H, int pgroups, int G,
+                                         int group_bytes8, int b, int h) {
+        const int64_t off = __ldg(head_offsets + h);
+        const int64_t end = (h + 1 < H) ? __ldg(head_offsets + h + 1) : batch_stride;
+        int64_t bytes = 0;
+        bool valid = true;
+        mask8 = 0;
+        if (pgroups <= 1) {
+            const int pr = __ldg(prec_map + h);
+            valid = pr == 4 || pr == 8;
+            mask8 = pr == 8 ? (G >= 32 ? 0xFFFFFFFFu : (1u << G) - 1u) : 0u;
+            bytes = static_cast<int64_t>(G) * group_bytes8 * pr / 8;
+        } else {
+            for (int g = 0; g < G; ++g) {
+                const int pr = __ldg(prec_map + static_cast<int64_t>(h) * G + g);
+                valid = valid && (pr == 4 || pr == 8);
+                if (pr == 8) mask8 |= 1u << g;
+                bytes += static_cast<int64_t>(group_bytes8) * pr / 8;
+            }
+        }
+        ok = valid && off >= 0 && off + bytes <= end;
+        code_off = static_cast<int64_t>(b) * batch_stride + off;
+    }
+};
+
 // A warp's walk over its tiles gw, gw + W, ...: the tile's batch row and
 // head are advanced incrementally (no division per tile), and its layout
-// read from the precision map and head offsets: the byte offset of its codes
-// and its precision, or prec = 0 when prec_map does not fit the offsets.
-struct TileCursor {
+// read from the precision map and head offsets (ok = false when prec_map
+// does not fit the offsets).
+struct TileCursor : TileLayout {
     int tile, b, h;
     int db, dh;          // W / H and W % H
-    int64_t code_off;
-    int prec;
 
     __device__ __forceinline__ void init(const StepParams& p, int first, int W) {
         tile = first;
@@ -543,13 +592,9 @@ struct TileCursor {
             ++b;
         }
     }
-    __device__ __forceinline__ void load(const StepParams& p, int dv) {
-        const int pr = __ldg(p.prec_map + h);
-        const int64_t off = __ldg(p.head_offsets + h);
-        const int64_t end = (h + 1 < p.H) ? __ldg(p.head_offsets + h + 1) : p.batch_stride;
-        const int64_t bytes = static_cast<int64_t>(p.d_k) * dv * pr / 8;
-        prec = ((pr == 4 || pr == 8) && off >= 0 && off + bytes <= end) ? pr : 0;
-        code_off = static_cast<int64_t>(b) * p.batch_stride + off;
+    __device__ __forceinline__ void load(const StepParams& p, int group_bytes8) {
+        TileLayout::load(p.prec_map, p.head_offsets, p.batch_stride, p.H, p.pgroups, p.G,
+                         group_bytes8, b, h);
     }
 };
 
@@ -654,40 +699,50 @@ __device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int
 }
 
 // Fill `slot` with group g of the cursor's tile (lane 0 only); with the
-// first group, also the tile's inputs into `tin`. A tile whose layout does not
-// fit gets a bare arrival, so the slot's phase still completes.
-template <int C, int GROUP, int GATE, int IO>
+// first group, also the tile's inputs (into `tin`, or for INS into the
+// header's v and the slot's q, k rows). A tile whose layout does not fit gets
+// a bare arrival, so the slot's phase still completes.
+template <int C, int GROUP, int GATE, int IO, bool INS>
 __device__ __forceinline__ void issue_item(const StepParams& p, uint8_t* wsm, int slot,
                                            const TileCursor& tc, int g, uint8_t* tin,
                                            uint64_t pol_state, uint64_t pol_in) {
-    using S = Slot<C, GROUP, GATE, IO>;
+    using S = Slot<C, GROUP, GATE, IO, INS>;
     constexpr int DV = 32 * C;
     constexpr int ES = S::ES;
     uint64_t* bar = reinterpret_cast<uint64_t*>(wsm) + slot;
-    if (tc.prec == 0) {
+    if (!tc.ok) {
         mbar_arrive(bar);
         return;
     }
     const int tile = tc.tile;
     const int dk = p.d_k;
     uint8_t* sm = wsm + S::header(dk) + slot * S::kBytes;
-    const uint32_t cbytes = GROUP * DV * tc.prec / 8;
+    const uint32_t cbytes = GROUP * DV * tc.bits(g) / 8;
+    const int64_t rowbase = static_cast<int64_t>(tile) * dk;
     uint32_t total = cbytes + DV * 4;
-    if (g == 0) total += S::tile_in_payload(dk);
+    if (INS) {
+        total += 2 * GROUP * ES;
+        if (g == 0) total += DV * ES;
+    } else if (g == 0) {
+        total += S::tile_in_payload(dk);
+    }
     mbar_arrive_expect_tx(bar, total);
-    bulk_g2s(sm, p.codes + tc.code_off + static_cast<int64_t>(g) * cbytes, cbytes, bar, pol_state);
+    bulk_g2s(sm, p.codes + tc.code_off + tc.goff(g, GROUP * DV / 2), cbytes, bar, pol_state);
     bulk_g2s(sm + S::kScales, p.scales + (static_cast<int64_t>(tile) * p.G + g) * DV, DV * 4, bar,
              pol_state);
-    if (g == 0) {
-        const int64_t rowbase = static_cast<int64_t>(tile) * dk;
+    const uint8_t* vsrc = static_cast<const uint8_t*>(p.v) + static_cast<int64_t>(tile) * DV * ES;
+    if (INS) {
+        const int64_t r0 = rowbase + g * GROUP;
+        bulk_g2s(sm + S::kQ, static_cast<const uint8_t*>(p.q) + r0 * ES, GROUP * ES, bar, pol_in);
+        bulk_g2s(sm + S::kK, static_cast<const uint8_t*>(p.k) + r0 * ES, GROUP * ES, bar, pol_in);
+        if (g == 0) bulk_g2s(wsm + 128, vsrc, DV * ES, bar, pol_in);
+    } else if (g == 0) {
         bulk_g2s(tin, static_cast<const uint8_t*>(p.q) + rowbase * ES, dk * ES, bar, pol_in);
         bulk_g2s(tin + S::in_k(dk), static_cast<const uint8_t*>(p.k) + rowbase * ES, dk * ES, bar,
                  pol_in);
         if (GATE == kGatePerKey)
             bulk_g2s(tin + S::in_g(dk), p.gates + rowbase, dk * 4, bar, pol_in);
-        bulk_g2s(tin + S::in_v(dk),
-                 static_cast<const uint8_t*>(p.v) + static_cast<int64_t>(tile) * DV * ES, DV * ES,
-                 bar, pol_in);
+        bulk_g2s(tin + S::in_v(dk), vsrc, DV * ES, bar, pol_in);
     }
 }
 
@@ -709,7 +764,8 @@ struct Ring {
 template <int C, int GROUP, int UPD, int GATE, int MODE, int IO>
 __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
     step_kernel(const StepParams p) {
-    using S = Slot<C, GROUP, GATE, IO>;
+    constexpr bool INS = UPD == kDelta;
+    using S = Slot<C, GROUP, GATE, IO, INS>;
     constexpr int DV = 32 * C;
     constexpr int P = C / 2;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -741,12 +797,12 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
     int it_n = 0;                // warp-local tile number of item ki
     TileCursor itc;              // tile of item ki
     itc.init(p, gw, W);
-    if (K > 0) itc.load(p, DV);
+    if (K > 0) itc.load(p, GROUP * DV);
 
     auto issue_next = [&]() {
         if (ki < K && !p.inject) {
             if (lane == 0)
-                issue_item<C, GROUP, GATE, IO>(p, wsm, is.slot, itc, it_g,
+                issue_item<C, GROUP, GATE, IO, INS>(p, wsm, is.slot, itc, it_g,
                                                wsm + 128 + (it_n & 1) * tib, pol_state, pol_in);
             ++ki;
             is.advance(NS);
@@ -754,7 +810,7 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
                 it_g = 0;
                 ++it_n;
                 itc.advance(p, W);
-                if (ki < K) itc.load(p, DV);
+                if (ki < K) itc.load(p, GROUP * DV);
             }
         }
     };
@@ -771,8 +827,9 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
     ti.init(p, gw, W);
     for (int n = 0; n < ntw && ok; ++n, ti.advance(p, W)) {
         const int tile = ti.tile;
-        ti.load(p, DV);
-        const uint8_t* tin = wsm + 128 + (n & 1) * tib;   // this tile's q, k, gates, v
+        ti.load(p, GROUP * DV);
+        const uint8_t* tin = wsm + 128 + (n & 1) * tib;   // this tile's q, k, gates, v (!INS)
+        const uint8_t* v_s = INS ? wsm + 128 : tin + in_v;
         const float gscalar = nscal, beta = nbeta;
         if (n + 1 < ntw) {
             if (GATE == kGate) nscal = __ldg(p.gates + tile + W);
@@ -787,7 +844,7 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[ic.slot], ic.par, p.timeout_ns));
         if (!ok) break;
 
-        if (ti.prec == 0) {
+        if (!ti.ok) {
             // no copies were made for this tile: record the mismatch and skip it
             if (lane == 0) atomicOr(p.err, kErrLayout);
             for (int g = 0; g < G; ++g) {
@@ -821,12 +878,12 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
                 if (!ok) break;
                 const uint8_t* sm = wsm + hdr + r.slot * S::kBytes;
                 const float* ss = reinterpret_cast<const float*>(sm + S::kScales) + lane * C;
-                const uint8_t* ks = tin + in_k + g * GROUP * S::ES;
+                const uint8_t* ks = INS ? sm + S::kK : tin + in_k + g * GROUP * S::ES;
                 float2 up = u[0], uq = u[P - 1];
 #pragma unroll 1
                 for (int pc = 0; pc < P; ++pc) {
                     const float2 sc = *reinterpret_cast<const float2*>(ss + 2 * pc);
-                    if (ti.prec == 8)
+                    if (ti.bits(g) == 8)
                         pair_ktS<GROUP, 8, IO>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, ks, lane, up);
                     else
                         pair_ktS<GROUP, 4, IO>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, ks, lane, up);
@@ -841,7 +898,7 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
             }
 #pragma unroll
             for (int pc = 0; pc < P; ++pc) {
-                const float2 vv = ld_pair<IO>(tin + in_v, lane * C + 2 * pc);
+                const float2 vv = ld_pair<IO>(v_s, lane * C + 2 * pc);
                 // w = beta (v - alpha u): three separate roundings
                 const float d0 = __fsub_rn(vv.x, __fmul_rn(gscalar, u[pc].x));
                 const float d1 = __fsub_rn(vv.y, __fmul_rn(gscalar, u[pc].y));
@@ -850,12 +907,11 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
         } else {
 #pragma unroll
             for (int pc = 0; pc < P; ++pc)
-                w[pc] = ld_pair<IO>(tin + in_v, lane * C + 2 * pc);
+                w[pc] = ld_pair<IO>(v_s, lane * C + 2 * pc);
         }
 
         if (!ok) break;
         uint8_t* gcodes_tile = p.codes + ti.code_off;
-        const uint32_t cbytes = GROUP * DV * ti.prec / 8;
         for (int g = 0; g < G; ++g) {
             if (UPD != kDelta && g > 0) {
                 ok = __all_sync(0xffffffffu,
@@ -864,11 +920,12 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
             }
             const uint8_t* sm = wsm + hdr + ic.slot * S::kBytes;
             const float* ss = reinterpret_cast<const float*>(sm + S::kScales) + lane * C;
-            const uint8_t* qs = tin + g * GROUP * S::ES;
-            const uint8_t* ks = tin + in_k + g * GROUP * S::ES;
+            const uint8_t* qs = INS ? sm + S::kQ : tin + g * GROUP * S::ES;
+            const uint8_t* ks = INS ? sm + S::kK : tin + in_k + g * GROUP * S::ES;
             const float* gs = reinterpret_cast<const float*>(tin + in_g) + g * GROUP;
             float* gscale = p.scales + (static_cast<int64_t>(tile) * G + g) * DV + lane * C;
-            uint8_t* gcodes = gcodes_tile + static_cast<int64_t>(g) * cbytes;
+            uint8_t* gcodes = gcodes_tile + ti.goff(g, GROUP * DV / 2);
+            const bool int8g = ti.bits(g) == 8;
             // The column pairs run one after the other through one copy of the
             // (large) pair code; the pairs' w and o rotate through (wp, op).
             float2 wp = w[0], op = o[0], wq = w[P - 1], oq = o[P - 1];
@@ -877,7 +934,7 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
                 const float2 sc = *reinterpret_cast<const float2*>(ss + 2 * pc);
                 const uint32_t j0 = static_cast<uint32_t>(lane * C + 2 * pc);
                 if constexpr (stage_x(MODE)) {
-                    if (ti.prec == 8)
+                    if (int8g)
                         pair_step_xs<GROUP, GATE, MODE, 8, IO>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs,
                                                            ks, gs, gscalar, wp, op, gcodes,
                                                            gscale + 2 * pc, hkey, g * GROUP, j0,
@@ -888,7 +945,7 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
                                                            gscale + 2 * pc, hkey, g * GROUP, j0,
                                                            lane, xs);
                 } else {
-                    if (ti.prec == 8)
+                    if (int8g)
                         pair_step<GROUP, GATE, MODE, 8, IO>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs, ks,
                                                         gs, gscalar, wp, op, gcodes,
                                                         gscale + 2 * pc, hkey, g * GROUP, j0, lane);

@@ -54,6 +54,8 @@ _P = ctypes.c_void_p
 _SIGS = {
     "lrs_layout_query": [ctypes.POINTER(lrs_shape), _P, _P, _P, _P],
     "lrs_state_alloc": [ctypes.POINTER(lrs_shape), _P, ctypes.POINTER(lrs_state)],
+    "lrs_layout_query_groups": [ctypes.POINTER(lrs_shape), _P, _P, _P, _P],
+    "lrs_state_alloc_groups": [ctypes.POINTER(lrs_shape), _P, ctypes.POINTER(lrs_state)],
     "lrs_state_free": [ctypes.POINTER(lrs_state)],
     "lrs_decode_step": [ctypes.POINTER(lrs_state), _P, _P, _P, _P, _P, _P, _P, _P, _P,
                         ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int32, _P],
@@ -154,11 +156,30 @@ def lrs_layout_query(shp, prec_map_host):
     return offs, stride.value, count.value
 
 
+def lrs_layout_query_groups(shp, prec_map_host):
+    """prec_map_host [H][G] -> (head_offsets, batch_stride_bytes, scale_count). Host only."""
+    import numpy as np
+    pm = np.ascontiguousarray(prec_map_host, dtype=np.uint8)
+    offs = np.zeros(shp.heads, np.int64)
+    stride = ctypes.c_int64()
+    count = ctypes.c_int64()
+    _check(lib().lrs_layout_query_groups(ctypes.byref(shp), pm.ctypes.data, offs.ctypes.data,
+                                         ctypes.addressof(stride), ctypes.addressof(count)))
+    return offs, stride.value, count.value
+
+
 def lrs_state_alloc(shp, prec_map_host):
+    """prec_map_host [H]: one width per head; [H][G]: one per (head, scale group)
+    (lrs_state_alloc_groups)."""
     import numpy as np
     pm = np.ascontiguousarray(prec_map_host, dtype=np.uint8)
     st = lrs_state()
-    _check(lib().lrs_state_alloc(ctypes.byref(shp), pm.ctypes.data, ctypes.byref(st)))
+    if pm.ndim == 2:
+        if pm.shape != (shp.heads, shp.d_k // shp.group):
+            raise ValueError("prec_map must be [H] or [H][d_k/group]")
+        _check(lib().lrs_state_alloc_groups(ctypes.byref(shp), pm.ctypes.data, ctypes.byref(st)))
+    else:
+        _check(lib().lrs_state_alloc(ctypes.byref(shp), pm.ctypes.data, ctypes.byref(st)))
     return st
 
 

@@ -40,6 +40,29 @@ def prec_map_for(w, device="cuda", steps=None):
     return pm
 
 
+def group_prec_map_for(w, device="cuda", steps=None):
+    """Per-(head, scale group) widths: the mean decay of each block of `group`
+    key channels ranked over all H*G blocks (library and oracle must agree),
+    the top int8_fraction of blocks int8. For scalar decays every block of a
+    head has the head's mean, so ties order the blocks by index."""
+    G = w.d_k // w.group
+    decay = I.decay_tensor(w, steps=steps, device=device)        # [T*B][H][inner]
+    outer, H, inner = decay.shape
+    if inner == w.d_k:
+        blocks = decay.reshape(outer, H * G, w.group)
+    else:                                                        # one decay per head
+        blocks = decay.expand(outer, H, w.d_k).reshape(outer, H * G, w.group).contiguous()
+    means = torch.zeros(H * G, dtype=torch.float64, device=device)
+    lrs.lrs_decay_head_means(blocks, outer, H * G, w.group, means)
+    torch.cuda.synchronize()
+    n8 = int(round(w.int8_fraction * H * G))
+    pm = lrs.lrs_precision_map(means.cpu().numpy(), n8)
+    ref_means = oracle.decay_means(blocks.cpu().numpy())
+    np.testing.assert_allclose(means.cpu().numpy(), ref_means, rtol=1e-12)
+    np.testing.assert_array_equal(pm, oracle.precision_map(ref_means, n8))
+    return pm.reshape(H, G)
+
+
 def make_shape(w, batch=None):
     return lrs.shape(w.batch if batch is None else batch, w.heads, w.d_k, w.d_v, w.group,
                      w.update_kind, w.gate_kind)
@@ -49,8 +72,9 @@ def sample_tiles(w, pm, n_b=8, n_h=8):
     """Tiles spread over batch rows and heads, both precisions when mixed,
     always including the first and last tile."""
     bs = np.unique(np.linspace(0, w.batch - 1, min(n_b, w.batch)).round().astype(int))
-    heads8 = [h for h in range(w.heads) if pm[h] == 8]
-    heads4 = [h for h in range(w.heads) if pm[h] == 4]
+    pm = np.asarray(pm).reshape(w.heads, -1)          # [H] or [H][G] widths
+    heads8 = [h for h in range(w.heads) if (pm[h] == 8).all()]
+    heads4 = [h for h in range(w.heads) if not (pm[h] == 8).all()]
     hs = []
     for group in (heads8, heads4):
         if group:
@@ -189,10 +213,11 @@ def check_out_bf16(gpu, ref, where=""):
 
 
 def run_parity(w, steps, tiles=None, mode=None, check_every=None, device="cuda", stats=None,
-               io="f32"):
+               io="f32", pm=None):
     """Free-running parity over `steps` steps; full state compared at
     step 0 (import), 1, 2, steps//2 and steps (or every step if check_every=1)."""
-    pm = prec_map_for(w, device=device)
+    if pm is None:
+        pm = prec_map_for(w, device=device)
     if tiles == "sample":
         tiles = sample_tiles(w, pm)
     pair = Pair(w, pm, tiles=tiles, mode=mode, device=device, io=io)

@@ -54,6 +54,24 @@ def test_layout_offsets_are_prefix_sums():
     assert nsc == 3 * 5 * (128 // 32) * 64
 
 
+def test_group_layout_offsets_are_prefix_sums():
+    pm = np.array([[8, 4, 4, 8], [4, 4, 4, 4], [8, 8, 8, 4]], np.uint8)
+    shp = lrs.shape(2, 3, 128, 64, 32, lrs.LRS_UPDATE_GATED, lrs.LRS_GATE_SCALAR)
+    offs, stride, nsc = lrs.lrs_layout_query_groups(shp, pm)
+    sizes = (32 * 64 * pm.astype(np.int64) // 8).sum(axis=1)
+    np.testing.assert_array_equal(offs, np.concatenate([[0], np.cumsum(sizes)[:-1]]))
+    assert stride == sizes.sum()
+    assert nsc == 2 * 3 * 4 * 64
+    # a uniform group map is the head map's layout
+    o2, s2, _ = lrs.lrs_layout_query(shp, pm[:, 0].copy())
+    o3, s3, _ = lrs.lrs_layout_query_groups(shp, np.repeat(pm[:, :1], 4, axis=1))
+    np.testing.assert_array_equal(o2, o3)
+    assert s2 == s3
+    with pytest.raises(lrs.LrsError) as ei:
+        lrs.lrs_layout_query_groups(shp, np.full((3, 4), 6, np.uint8))
+    assert ei.value.status == lrs.LRS_ERR_INVALID_ARG
+
+
 @pytest.mark.parametrize("args,status", [
     ((2, 2, 128, 96, 32, 0, 1), lrs.LRS_ERR_UNSUPPORTED),   # d_v
     ((2, 2, 128, 128, 64, 0, 1), lrs.LRS_ERR_UNSUPPORTED),  # group*d_v too large

@@ -14,9 +14,10 @@ from tests.test_gpu_parity import _small
 pytestmark = pytest.mark.gpu
 
 
-def run_chunks(w, T, n_chunks=1, tiles=None, mode=None):
+def run_chunks(w, T, n_chunks=1, tiles=None, mode=None, pm=None):
     mode = w.mode if mode is None else mode
-    pm = P.prec_map_for(w)
+    if pm is None:
+        pm = P.prec_map_for(w)
     if tiles == "sample":
         tiles = P.sample_tiles(w, pm)
     pair = P.Pair(w, pm, tiles=tiles, mode=mode)
