@@ -407,6 +407,153 @@ int orc_chunk_step_pg(int ntiles, const int32_t *tile_b, const int32_t *tile_h, 
                      step, nthreads);
 }
 
+/* ------------------------------------------------- Low-Rank Bypass --- */
+
+/* [LRB/BDR] Low-Rank Bypass: small updates are accumulated in a compact
+ * low-rank buffer and the buffer's sufficiently large elements are merged
+ * into the state from time to time. The sources give neither the rank, the
+ * merge period nor the threshold; the readings taken here:
+ *   - buffer L = sum_l U_l V_l^T, l < r, U_l in R^{d_k}, V_l in R^{d_v}, fp32;
+ *     the effective state is deq(S_q) + L;
+ *   - each step appends the step's rank-1 update k w^T as the next component
+ *     (U_m = k, V_m = w, m = step mod r components were already there) instead
+ *     of adding it to the quantized state, and decays the older components
+ *     with the state (U_l <- g * U_l, per key or scalar);
+ *   - the quantized part is decayed and requantized every step as before;
+ *   - every r-th step (when the buffer is full) the dense product M = U V^T
+ *     is formed and every element with |M_ij| >= s_ij / 2 (half the element's
+ *     quantization step before the step) is added to the state before it is
+ *     requantized; the buffer is then emptied (the smaller elements, which
+ *     rounding would have removed from the state too, are dropped);
+ *   - the delta rule reads k^T of the effective state: u = k^T deq +
+ *     sum_l (k . U_l) V_l;
+ *   - the output is read from the effective state after the step:
+ *     o = x^T q + sum_l (q . U_l) V_l, before any merge.
+ * Order of operations (one rounding per operation, as in the decode step):
+ *   e_l = sum_i k_i U_li (key order, undecayed U)      [delta rule only]
+ *   u_j = sum_i k_i deq_ij (key order), then u_j = fma(e_l, V_lj, u_j), l order
+ *   w_j = RN(beta RN(v_j - RN(alpha u_j)))  (gated: w = v)
+ *   U_l <- RN(g_i U_li) for l < m;  U_m = k, V_m = w
+ *   x_ij = RN(g_i deq_ij)
+ *   o_j = sum_i q_i x_ij (key order), then f_l = sum_i q_i U_li (key order)
+ *         and o_j = fma(f_l, V_lj, o_j), l order, l <= m
+ *   merge (m + 1 == r): M_ij = fma chain over l of U_li V_lj from 0;
+ *         if M_ij != 0 and |M_ij| >= RN(0.5 s_old): x_ij = RN(x_ij + M_ij);
+ *         U, V <- 0
+ *   then new scales and codes from x by the rounding mode (BDR: update x - deq).
+ * x_out (may be NULL) receives x before rounding, for the pins. */
+static void lrb_tile(int d_k, int d_v, int group, const int *qmaxs, int update_kind,
+                     int gate_kind, int mode, int r, int m, int8_t *c, float *s, float *U,
+                     float *V, const float *q, const float *k, const float *v, const float *gate,
+                     float beta, float *out, float *deq, float *x, float *w, float *M,
+                     uint64_t seed, uint64_t step, uint32_t b, uint32_t h, float *x_out)
+{
+    for (int i = 0; i < d_k; ++i)
+        for (int j = 0; j < d_v; ++j)
+            deq[i * d_v + j] = (float)c[i * d_v + j] * s[(i / group) * d_v + j];
+    float alpha = gate[0];
+    if (update_kind == ORC_UPDATE_DELTA) {
+        for (int j = 0; j < d_v; ++j) {
+            float u = 0.0f;
+            for (int i = 0; i < d_k; ++i) u = fmaf(k[i], deq[i * d_v + j], u);
+            w[j] = u;
+        }
+        for (int l = 0; l < m; ++l) {
+            float e = 0.0f;
+            for (int i = 0; i < d_k; ++i) e = fmaf(k[i], U[l * d_k + i], e);
+            for (int j = 0; j < d_v; ++j) w[j] = fmaf(e, V[l * d_v + j], w[j]);
+        }
+        for (int j = 0; j < d_v; ++j) {
+            float t = alpha * w[j];
+            float d = v[j] - t;
+            w[j] = beta * d;
+        }
+    } else {
+        for (int j = 0; j < d_v; ++j) w[j] = v[j];
+    }
+    for (int l = 0; l < m; ++l)
+        for (int i = 0; i < d_k; ++i) {
+            float gi = (gate_kind == ORC_GATE_PER_KEY) ? gate[i] : alpha;
+            U[l * d_k + i] = gi * U[l * d_k + i];
+        }
+    for (int i = 0; i < d_k; ++i) U[m * d_k + i] = k[i];
+    for (int j = 0; j < d_v; ++j) V[m * d_v + j] = w[j];
+    for (int i = 0; i < d_k; ++i) {
+        float gi = (gate_kind == ORC_GATE_PER_KEY) ? gate[i] : alpha;
+        for (int j = 0; j < d_v; ++j) x[i * d_v + j] = gi * deq[i * d_v + j];
+    }
+    for (int j = 0; j < d_v; ++j) {
+        float acc = 0.0f;
+        for (int i = 0; i < d_k; ++i) acc = fmaf(q[i], x[i * d_v + j], acc);
+        out[j] = acc;
+    }
+    for (int l = 0; l <= m; ++l) {
+        float f = 0.0f;
+        for (int i = 0; i < d_k; ++i) f = fmaf(q[i], U[l * d_k + i], f);
+        for (int j = 0; j < d_v; ++j) out[j] = fmaf(f, V[l * d_v + j], out[j]);
+    }
+    if (m + 1 == r) {
+        for (int i = 0; i < d_k; ++i)
+            for (int j = 0; j < d_v; ++j) {
+                float acc = 0.0f;
+                for (int l = 0; l < r; ++l) acc = fmaf(U[l * d_k + i], V[l * d_v + j], acc);
+                M[i * d_v + j] = acc;
+            }
+        for (int i = 0; i < d_k; ++i)
+            for (int j = 0; j < d_v; ++j) {
+                float mij = M[i * d_v + j];
+                float half = 0.5f * s[(i / group) * d_v + j];
+                if (mij != 0.0f && fabsf(mij) >= half) x[i * d_v + j] = x[i * d_v + j] + mij;
+            }
+        memset(U, 0, (size_t)r * d_k * sizeof(float));
+        memset(V, 0, (size_t)r * d_v * sizeof(float));
+    }
+    if (x_out) memcpy(x_out, x, (size_t)d_k * d_v * sizeof(float));
+    requantize_tile(d_k, d_v, group, qmaxs, mode, x, deq, c, s, seed, step, b, h);
+}
+
+int orc_lrb_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int d_k, int d_v,
+                 int group, int update_kind, int gate_kind, int mode, const uint8_t *prec_map,
+                 int8_t *codes, float *scales, int rank, float *U, float *V, const float *q,
+                 const float *k, const float *v, const float *gates, const float *beta,
+                 float *out, uint64_t seed, uint64_t step, float *x_out)
+{
+    if (ntiles < 0 || check_shape(d_k, d_v, group, update_kind, gate_kind) != 0) return -1;
+    if (mode != ORC_ROUND_RTN && mode != ORC_ROUND_SR && mode != ORC_ROUND_BDR) return -1;
+    if (rank < 1) return -1;
+    if (ntiles == 0) return 0;
+    if (!tile_b || !tile_h || !prec_map || !codes || !scales || !U || !V || !q || !k || !v ||
+        !gates || !out)
+        return -1;
+    if (update_kind == ORC_UPDATE_DELTA && !beta) return -1;
+    int G = d_k / group;
+    int rc = check_prec(ntiles, tile_h, prec_map, 1, G);
+    if (rc != 0) return rc;
+    size_t n = (size_t)d_k * d_v;
+    float *deq = (float *)malloc(n * sizeof(float));
+    float *x = (float *)malloc(n * sizeof(float));
+    float *M = (float *)malloc(n * sizeof(float));
+    float *w = (float *)malloc((size_t)d_v * sizeof(float));
+    int *qm = (int *)malloc((size_t)G * sizeof(int));
+    if (!deq || !x || !M || !w || !qm) {
+        free(deq); free(x); free(M); free(w); free(qm);
+        return -2;
+    }
+    int m = (int)(step % (uint64_t)rank);
+    size_t gate_len = (gate_kind == ORC_GATE_PER_KEY) ? (size_t)d_k : 1;
+    for (int t = 0; t < ntiles; ++t) {
+        head_qmaxs(prec_map, 1, G, tile_h[t], qm);
+        lrb_tile(d_k, d_v, group, qm, update_kind, gate_kind, mode, rank, m, codes + t * n,
+                 scales + (size_t)t * G * d_v, U + (size_t)t * rank * d_k,
+                 V + (size_t)t * rank * d_v, q + (size_t)t * d_k, k + (size_t)t * d_k,
+                 v + (size_t)t * d_v, gates + t * gate_len, beta ? beta[t] : 0.0f,
+                 out + (size_t)t * d_v, deq, x, w, M, seed, step, (uint32_t)tile_b[t],
+                 (uint32_t)tile_h[t], x_out ? x_out + t * n : NULL);
+    }
+    free(deq); free(x); free(M); free(w); free(qm);
+    return 0;
+}
+
 uint16_t orc_bf16_rne(float x)
 {
     uint32_t u;

@@ -113,6 +113,19 @@ int orc_chunk_step_pg(int ntiles, const int32_t *tile_b, const int32_t *tile_h,
 int orc_import_pg(int ntiles, const int32_t *tile_h, int d_k, int d_v, int group,
                   const uint8_t *prec_map, const float *S0, int8_t *codes, float *scales);
 
+/* Decode step with Low-Rank Bypass ([LRB/BDR] abstract): the step's rank-1
+ * update goes into a rank-`rank` buffer (U [ntiles][rank][d_k], V
+ * [ntiles][rank][d_v], updated in place; step mod rank components filled),
+ * and every rank-th step the buffer's elements of at least half a
+ * quantization step are merged into the state. The readings and the order of
+ * operations are stated at the definition. x_out (NULL or [ntiles][d_k][d_v])
+ * receives the values before rounding. Per-head widths. */
+int orc_lrb_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h,
+                 int d_k, int d_v, int group, int update_kind, int gate_kind, int mode,
+                 const uint8_t *prec_map, int8_t *codes, float *scales, int rank, float *U,
+                 float *V, const float *q, const float *k, const float *v, const float *gates,
+                 const float *beta, float *out, uint64_t seed, uint64_t step, float *x_out);
+
 /* bfloat16 (the upper half of binary32: sign, 8 exponent bits, 7 fraction
  * bits) nearest to x, ties to the even fraction; NaN becomes a quiet NaN of the
  * same sign. Returns the 16-bit pattern. */
