@@ -220,6 +220,32 @@ lrs_status lrs_chunk_step(const lrs_state *st, void *state_codes, float *scales,
                           const float *v, const float *gates, const float *beta, float *out,
                           uint64_t seed, uint64_t step, int32_t mode, void *stream);
 
+/* The decode step with a Low-Rank Bypass buffer ([LRB/BDR] abstract: small
+ * updates accumulate in a compact low-rank buffer whose sufficiently large
+ * elements are merged into the state from time to time). The sources fix no
+ * rank, period or threshold; this entry point takes:
+ *   - buffer L = U V^T of rank `rank` (1..8): U [B][H][rank][d_k] and
+ *     V [B][H][rank][d_v], fp32 device memory owned by the caller, zero at
+ *     the start, updated in place; step mod rank components are filled before
+ *     the call, so calls must pass consecutive steps (the buffer empties at
+ *     every step with step mod rank == rank - 1);
+ *   - each step appends its rank-1 update k w^T to the buffer instead of the
+ *     quantized state, and the older components decay with the state;
+ *   - the quantized state is decayed (x = RN(g deq)) and requantized as in
+ *     lrs_decode_step; the delta rule's k^T S and the output read the
+ *     effective state deq + U V^T;
+ *   - at the step that fills the buffer, every element of U V^T whose
+ *     magnitude is at least half of its quantization step (old scale / 2) is
+ *     added to x before the requantization, and the buffer is emptied.
+ * Other arguments, layouts, errors and asynchrony as lrs_decode_step; states
+ * with per-group widths are not supported (LRS_ERR_UNSUPPORTED); d_k and d_v
+ * in {64, 128}. */
+lrs_status lrs_lrb_step(const lrs_state *st, void *state_codes, float *scales,
+                        const uint8_t *prec_map, int32_t rank, float *U, float *V,
+                        const float *q, const float *k, const float *v, const float *gates,
+                        const float *beta, float *out, uint64_t seed, uint64_t step,
+                        int32_t mode, void *stream);
+
 /* The same step with HOST inputs and output: copies q, k, v, gates, beta
  * from host memory into device staging buffers owned by the state (allocated
  * on first use), runs lrs_decode_step on the state's own buffers, and copies

@@ -38,6 +38,10 @@ ChunkKernel find_chunk_kernel_rtn(int d_k, int d_v, int group, int update_kind, 
 ChunkKernel find_chunk_kernel_sr(int d_k, int d_v, int group, int update_kind, int gate_kind);
 ChunkKernel find_chunk_kernel_bdr(int d_k, int d_v, int group, int update_kind, int gate_kind);
 
+ChunkKernel find_lrb_kernel_rtn(int d_k, int d_v, int group, int update_kind, int gate_kind);
+ChunkKernel find_lrb_kernel_sr(int d_k, int d_v, int group, int update_kind, int gate_kind);
+ChunkKernel find_lrb_kernel_bdr(int d_k, int d_v, int group, int update_kind, int gate_kind);
+
 struct LayoutArgs {
     uint8_t* codes;
     float* scales;

@@ -63,6 +63,8 @@ _SIGS = {
                              ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int32, _P],
     "lrs_chunk_step": [ctypes.POINTER(lrs_state), _P, _P, _P, ctypes.c_int32, _P, _P, _P, _P, _P,
                        _P, ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int32, _P],
+    "lrs_lrb_step": [ctypes.POINTER(lrs_state), _P, _P, _P, ctypes.c_int32, _P, _P, _P, _P, _P, _P,
+                     _P, _P, ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int32, _P],
     "lrs_decode_step_host": [ctypes.POINTER(lrs_state), _P, _P, _P, _P, _P, _P,
                              ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int32, _P],
     "lrs_decode_step_host_noalloc": [ctypes.POINTER(lrs_state), _P, _P, _P, _P, _P, _P, _P,
@@ -208,6 +210,14 @@ def lrs_chunk_step(st, state_codes, scales, prec_map, T, q, k, v, gates, beta, o
     _check(lib().lrs_chunk_step(ctypes.byref(st), _ptr(state_codes), _ptr(scales), _ptr(prec_map),
                                 T, _ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(beta), _ptr(out),
                                 seed, step, mode, _stream(stream)))
+
+
+def lrs_lrb_step(st, state_codes, scales, prec_map, rank, U, V, q, k, v, gates, beta, out, seed,
+                 step, mode, stream=None):
+    """Decode step with a Low-Rank Bypass buffer U [B][H][rank][d_k], V [B][H][rank][d_v]."""
+    _check(lib().lrs_lrb_step(ctypes.byref(st), _ptr(state_codes), _ptr(scales), _ptr(prec_map),
+                              rank, _ptr(U), _ptr(V), _ptr(q), _ptr(k), _ptr(v), _ptr(gates),
+                              _ptr(beta), _ptr(out), seed, step, mode, _stream(stream)))
 
 
 def lrs_decode_step_host(st, q_host, k_host, v_host, gates_host, beta_host, out_host, seed, step,
