@@ -471,6 +471,7 @@ def run_extras(args, w, wl, states, xs, out, seed, stream, L, NI, mode, dev, pm)
     del g
     lrs.lrs_sync()
     res["chunk"] = run_chunk_extra(w, wl, states, seed, stream, L, mode, dev, pm)
+    res["lrb"] = run_lrb_extra(w, wl, states, xs, out, seed, stream, L, NI, mode, dev, pm)
     # fp32 state kernel: 4 rotated fp32 states
     shp = lrs.shape(wl.batch, w.heads, w.d_k, w.d_v, w.group, w.update_kind, w.gate_kind)
     Ls = 4
@@ -553,6 +554,49 @@ def run_chunk_extra(w, wl, states, seed, stream, L, mode, dev, pm, T=16, n=32):
                          "flops_per_element_token": flops_el},
             "state_bytes": state_bytes(wl, pm),
             "io_bytes_per_chunk": io}
+
+
+def run_lrb_extra(w, wl, states, xs, out, seed, stream, L, NI, mode, dev, pm, rank=4, n=64):
+    """The decode step with a Low-Rank Bypass buffer of rank `rank` on the same
+    states and inputs (one buffer per layer state; n steps cover n/rank merges).
+    Algorithmic bytes per step: the state's codes and scales read and written,
+    plus the buffer rows read (filled components) and written (filled + the new
+    one), averaged over the rank-step cycle: rank * (d_k + d_v) * 4 per tile."""
+    import torch
+    from quantized_recurrent_state_decode_b200 import lrs
+    if w.d_k not in (64, 128) or w.d_v not in (64, 128):
+        return None
+    Us = [torch.zeros(wl.batch, w.heads, rank, w.d_k, device=dev) for _ in range(L)]
+    Vs = [torch.zeros(wl.batch, w.heads, rank, w.d_v, device=dev) for _ in range(L)]
+
+    def launch(i):
+        st, x = states[i % L], xs[i % NI]
+        lrs.lrs_lrb_step(st, st.state_codes, st.scales, st.prec_map, rank, Us[i % L], Vs[i % L],
+                         x["q"], x["k"], x["v"], x["gates"], x["beta"], out, seed, i // L, mode,
+                         stream)
+    for i in range(L * rank):
+        launch(i)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            launch(i + L * rank)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    del g
+    lrs.lrs_sync()
+    tiles = wl.batch * w.heads
+    nbytes = state_bytes(wl, pm) + tiles * rank * (w.d_k + w.d_v) * 4
+    peak, peak_kind = measured_peaks()
+    achieved = nbytes / (ms / 1e3) / 1e9
+    return {"rank": rank, "ms_per_step": ms, "steps_per_s": 1e3 / ms, "api": "lrs_lrb_step",
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "algorithmic_bytes_per_launch": nbytes}}
 
 
 def _sm_max_mhz():

@@ -97,8 +97,13 @@ struct Slot {
     __host__ __device__ static int header(int d_k) {
         return INS ? 128 + DV * ES : 128 + 2 * tile_in_bytes(d_k);
     }
+    // bfloat16 tile inputs (gated forms) are widened to fp32 once per tile
+    // into a buffer after the slots: q, k (d_k each), v (d_v)
+    static constexpr bool CVT = IO == kIoBF16 && !INS;
+    __host__ __device__ static int cvt_bytes(int d_k) { return CVT ? (2 * d_k + DV) * 4 : 0; }
     static int warp_bytes(int slots, bool xs, int d_k) {
-        return (header(d_k) + slots * kBytes + (xs ? kXsBytes : 0) + 127) / 128 * 128;
+        return (header(d_k) + slots * kBytes + cvt_bytes(d_k) + (xs ? kXsBytes : 0) + 127) / 128 *
+               128;
     }
 };
 
@@ -779,7 +784,11 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
     const int G = p.G, NS = p.slots;
     const int hdr = S::header(p.d_k), tib = S::tile_in_bytes(p.d_k);
     const int in_k = S::in_k(p.d_k), in_g = S::in_g(p.d_k), in_v = S::in_v(p.d_k);
-    float4* xs = reinterpret_cast<float4*>(wsm + hdr + NS * S::kBytes);   // SR, BDR
+    float* cvt = reinterpret_cast<float*>(wsm + hdr + NS * S::kBytes);   // bf16 widened (CVT)
+    float4* xs = reinterpret_cast<float4*>(wsm + hdr + NS * S::kBytes +
+                                           S::cvt_bytes(p.d_k));              // SR, BDR
+    constexpr int IOR = S::CVT ? kIoF32 : IO;     // element type the pair code reads
+    constexpr int ESR = IOR == kIoBF16 ? 2 : 4;
     const int ntw = gw < p.ntiles ? (p.ntiles - gw + W - 1) / W : 0;   // this warp's tiles
     const int64_t K = static_cast<int64_t>(ntw) * G;                    // this warp's items
 
@@ -844,6 +853,34 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[ic.slot], ic.par, p.timeout_ns));
         if (!ok) break;
 
+        // where this tile's q, k, v are read from (widened to fp32 for CVT)
+        const uint8_t* tq = tin;
+        const uint8_t* tk = tin + in_k;
+        const uint8_t* tv = v_s;
+        if constexpr (S::CVT) {
+            if (ti.ok) {
+                const int dk = p.d_k;
+                __syncwarp();                 // the previous tile is done with cvt
+                for (int e = 2 * lane; e < dk; e += 64) {
+                    const uint32_t wq = *reinterpret_cast<const uint32_t*>(tin + e * 2);
+                    const uint32_t wk = *reinterpret_cast<const uint32_t*>(tin + in_k + e * 2);
+                    cvt[e] = bf16_lo(wq);
+                    cvt[e + 1] = bf16_hi(wq);
+                    cvt[dk + e] = bf16_lo(wk);
+                    cvt[dk + e + 1] = bf16_hi(wk);
+                }
+                for (int e = 2 * lane; e < DV; e += 64) {
+                    const uint32_t wv = *reinterpret_cast<const uint32_t*>(v_s + e * 2);
+                    cvt[2 * dk + e] = bf16_lo(wv);
+                    cvt[2 * dk + e + 1] = bf16_hi(wv);
+                }
+                __syncwarp();
+                tq = reinterpret_cast<const uint8_t*>(cvt);
+                tk = reinterpret_cast<const uint8_t*>(cvt + dk);
+                tv = reinterpret_cast<const uint8_t*>(cvt + 2 * dk);
+            }
+        }
+
         if (!ti.ok) {
             // no copies were made for this tile: record the mismatch and skip it
             if (lane == 0) atomicOr(p.err, kErrLayout);
@@ -878,15 +915,15 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
                 if (!ok) break;
                 const uint8_t* sm = wsm + hdr + r.slot * S::kBytes;
                 const float* ss = reinterpret_cast<const float*>(sm + S::kScales) + lane * C;
-                const uint8_t* ks = INS ? sm + S::kK : tin + in_k + g * GROUP * S::ES;
+                const uint8_t* ks = INS ? sm + S::kK : tk + g * GROUP * ESR;
                 float2 up = u[0], uq = u[P - 1];
 #pragma unroll 1
                 for (int pc = 0; pc < P; ++pc) {
                     const float2 sc = *reinterpret_cast<const float2*>(ss + 2 * pc);
                     if (ti.bits(g) == 8)
-                        pair_ktS<GROUP, 8, IO>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, ks, lane, up);
+                        pair_ktS<GROUP, 8, IOR>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, ks, lane, up);
                     else
-                        pair_ktS<GROUP, 4, IO>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, ks, lane, up);
+                        pair_ktS<GROUP, 4, IOR>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, ks, lane, up);
                     if constexpr (P == 2) {
                         const float2 t = up;
                         up = uq; uq = t;
@@ -898,7 +935,7 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
             }
 #pragma unroll
             for (int pc = 0; pc < P; ++pc) {
-                const float2 vv = ld_pair<IO>(v_s, lane * C + 2 * pc);
+                const float2 vv = ld_pair<IOR>(tv, lane * C + 2 * pc);
                 // w = beta (v - alpha u): three separate roundings
                 const float d0 = __fsub_rn(vv.x, __fmul_rn(gscalar, u[pc].x));
                 const float d1 = __fsub_rn(vv.y, __fmul_rn(gscalar, u[pc].y));
@@ -907,7 +944,7 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
         } else {
 #pragma unroll
             for (int pc = 0; pc < P; ++pc)
-                w[pc] = ld_pair<IO>(v_s, lane * C + 2 * pc);
+                w[pc] = ld_pair<IOR>(tv, lane * C + 2 * pc);
         }
 
         if (!ok) break;
@@ -920,8 +957,8 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
             }
             const uint8_t* sm = wsm + hdr + ic.slot * S::kBytes;
             const float* ss = reinterpret_cast<const float*>(sm + S::kScales) + lane * C;
-            const uint8_t* qs = INS ? sm + S::kQ : tin + g * GROUP * S::ES;
-            const uint8_t* ks = INS ? sm + S::kK : tin + in_k + g * GROUP * S::ES;
+            const uint8_t* qs = INS ? sm + S::kQ : tq + g * GROUP * ESR;
+            const uint8_t* ks = INS ? sm + S::kK : tk + g * GROUP * ESR;
             const float* gs = reinterpret_cast<const float*>(tin + in_g) + g * GROUP;
             float* gscale = p.scales + (static_cast<int64_t>(tile) * G + g) * DV + lane * C;
             uint8_t* gcodes = gcodes_tile + ti.goff(g, GROUP * DV / 2);
@@ -935,22 +972,22 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
                 const uint32_t j0 = static_cast<uint32_t>(lane * C + 2 * pc);
                 if constexpr (stage_x(MODE)) {
                     if (int8g)
-                        pair_step_xs<GROUP, GATE, MODE, 8, IO>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs,
+                        pair_step_xs<GROUP, GATE, MODE, 8, IOR>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs,
                                                            ks, gs, gscalar, wp, op, gcodes,
                                                            gscale + 2 * pc, hkey, g * GROUP, j0,
                                                            lane, xs);
                     else
-                        pair_step_xs<GROUP, GATE, MODE, 4, IO>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs,
+                        pair_step_xs<GROUP, GATE, MODE, 4, IOR>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs,
                                                            ks, gs, gscalar, wp, op, gcodes,
                                                            gscale + 2 * pc, hkey, g * GROUP, j0,
                                                            lane, xs);
                 } else {
                     if (int8g)
-                        pair_step<GROUP, GATE, MODE, 8, IO>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs, ks,
+                        pair_step<GROUP, GATE, MODE, 8, IOR>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs, ks,
                                                         gs, gscalar, wp, op, gcodes,
                                                         gscale + 2 * pc, hkey, g * GROUP, j0, lane);
                     else
-                        pair_step<GROUP, GATE, MODE, 4, IO>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs, ks,
+                        pair_step<GROUP, GATE, MODE, 4, IOR>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs, ks,
                                                         gs, gscalar, wp, op, gcodes,
                                                         gscale + 2 * pc, hkey, g * GROUP, j0, lane);
                 }
