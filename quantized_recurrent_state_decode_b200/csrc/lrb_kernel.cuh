@@ -45,23 +45,63 @@ struct LrbParams {
     int32_t H, ntiles, rank, pgroups, inject;
 };
 
-// Shared memory of one CTA: barrier | codes | scales | U (kLrbMaxRank rows) |
-// q, k, [gate] (d_k fp32 each), v (d_v) | e, f (kLrbMaxRank each).
+// Shared memory of one CTA: two barriers, two stages (a tile is processed in
+// one while the next tile's copies land in the other), then e and f:
+//   stage: codes | scales | U (kLrbMaxRank rows) | q, k, [gate] (d_k fp32) | v
 template <int DK, int DV, int GROUP, int GATE>
 struct LrbSmem {
     static constexpr int G = DK / GROUP;
-    static constexpr int kCodes = 128;
+    static constexpr int kCodes = 0;
     static constexpr int kScales = kCodes + DK * DV;
     static constexpr int kU = kScales + G * DV * 4;
     static constexpr int kQ = kU + kLrbMaxRank * DK * 4;
     static constexpr int kK = kQ + DK * 4;
     static constexpr int kG = kK + DK * 4;
     static constexpr int kV = kG + (GATE == kGatePerKey ? DK * 4 : 0);
-    static constexpr int kE = kV + DV * 4;
+    static constexpr int kStage = (kV + DV * 4 + 127) / 128 * 128;
+    static constexpr int kStage0 = 128;
+    static constexpr int kE = kStage0 + 2 * kStage;
     static constexpr int kF = kE + kLrbMaxRank * 4;
     static constexpr int kBytes = kF + kLrbMaxRank * 4;
     static_assert(kU % 16 == 0 && kQ % 16 == 0 && kV % 16 == 0, "alignment");
 };
+
+// The copies of one tile into a stage (thread 0). A tile whose layout does
+// not fit gets a bare arrival, so the stage's phase still completes.
+template <int DK, int DV, int GROUP, int GATE>
+__device__ __forceinline__ void lrb_issue(const LrbParams& p, uint64_t* bar, uint8_t* st,
+                                          const TileLayout& tl, int tile, int m) {
+    using S = LrbSmem<DK, DV, GROUP, GATE>;
+    constexpr int G = DK / GROUP;
+    if (!tl.ok) {
+        mbar_arrive(bar);
+        return;
+    }
+    fence_proxy_async_smem();                // earlier shared reads before the copies land
+    const uint32_t cbytes = static_cast<uint32_t>(tl.goff(G, GROUP * DV / 2));
+    const uint64_t pol = policy_evict_first();
+    const int64_t row = static_cast<int64_t>(tile) * DK;
+    uint32_t bytes = cbytes + G * DV * 4 + 2 * DK * 4 + DV * 4;
+    if (GATE == kGatePerKey) bytes += DK * 4;
+    if (m > 0) bytes += m * DK * 4;
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_g2s(st + S::kCodes, p.codes + tl.code_off, cbytes, bar, pol);
+    bulk_g2s(st + S::kScales, p.scales + static_cast<int64_t>(tile) * G * DV, G * DV * 4, bar, pol);
+    if (m > 0)
+        bulk_g2s(st + S::kU, p.U + static_cast<int64_t>(tile) * p.rank * DK, m * DK * 4, bar, pol);
+    bulk_g2s(st + S::kQ, p.q + row, DK * 4, bar, pol);
+    bulk_g2s(st + S::kK, p.k + row, DK * 4, bar, pol);
+    if (GATE == kGatePerKey) bulk_g2s(st + S::kG, p.gates + row, DK * 4, bar, pol);
+    bulk_g2s(st + S::kV, p.v + static_cast<int64_t>(tile) * DV, DV * 4, bar, pol);
+}
+
+__device__ __forceinline__ TileLayout lrb_layout(const LrbParams& p, int tile, int G, int gbytes8) {
+    TileLayout tl;
+    const int b = tile / p.H;
+    tl.load(p.prec_map, p.head_offsets, p.batch_stride, p.H, p.pgroups, G, gbytes8, b,
+            tile - b * p.H);
+    return tl;
+}
 
 template <int DK, int DV, int GROUP, int UPD, int GATE, int MODE>
 __global__ void __launch_bounds__(DV, (3 * 128) / DV) lrb_kernel(const LrbParams p) {
@@ -69,14 +109,7 @@ __global__ void __launch_bounds__(DV, (3 * 128) / DV) lrb_kernel(const LrbParams
     constexpr int G = DK / GROUP;
     constexpr int C = DV / 32;
     extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
-    uint8_t* cs = smem + S::kCodes;
-    float* ss = reinterpret_cast<float*>(smem + S::kScales);
-    float* Us = reinterpret_cast<float*>(smem + S::kU);
-    const float* qs = reinterpret_cast<const float*>(smem + S::kQ);
-    const float* ks = reinterpret_cast<const float*>(smem + S::kK);
-    const float* gs = reinterpret_cast<const float*>(smem + S::kG);
-    const float* vs = reinterpret_cast<const float*>(smem + S::kV);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
     float* es = reinterpret_cast<float*>(smem + S::kE);
     float* fs = reinterpret_cast<float*>(smem + S::kF);
     const int j = threadIdx.x;
@@ -86,53 +119,70 @@ __global__ void __launch_bounds__(DV, (3 * 128) / DV) lrb_kernel(const LrbParams
     const bool merge = m + 1 == r;
 
     if (j == 0) {
-        mbar_init(bar, 1);
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
         fence_mbar_init();
     }
     __syncthreads();
-    uint32_t par = 0;
     bool ok = true;
+    int issued = 0;              // tiles whose copies thread 0 has issued (for draining)
 
-    for (int tile = blockIdx.x; tile < p.ntiles && ok; tile += gridDim.x) {
-        const int b = tile / p.H, h = tile - (tile / p.H) * p.H;
-        TileLayout tl;
-        tl.load(p.prec_map, p.head_offsets, p.batch_stride, p.H, p.pgroups, G, GROUP * DV, b, h);
+    // V[l][j] of the filled components of a tile (plain loads, coalesced across j)
+    auto load_v = [&](int tile, float (&Vr)[kLrbMaxRank]) {
+        const float* Vg = p.V + static_cast<int64_t>(tile) * r * DV;
+#pragma unroll
+        for (int l = 0; l < kLrbMaxRank; ++l) Vr[l] = l < m ? __ldcs(Vg + l * DV + j) : 0.0f;
+    };
+
+    const int first = blockIdx.x;
+    float Vn[kLrbMaxRank];       // the next tile's V
+    if (first < p.ntiles) {
+        if (j == 0 && !p.inject) {
+            lrb_issue<DK, DV, GROUP, GATE>(p, &bars[0], smem + S::kStage0,
+                                           lrb_layout(p, first, G, GROUP * DV), first, m);
+            issued = 1;
+        }
+        load_v(first, Vn);
+    }
+    int n = 0;
+    for (int tile = first; tile < p.ntiles && ok; tile += gridDim.x, ++n) {
+        const int stage = n & 1;
+        uint8_t* st = smem + S::kStage0 + stage * S::kStage;
+        uint8_t* cs = st + S::kCodes;
+        float* ss = reinterpret_cast<float*>(st + S::kScales);
+        float* Us = reinterpret_cast<float*>(st + S::kU);
+        const float* qs = reinterpret_cast<const float*>(st + S::kQ);
+        const float* ks = reinterpret_cast<const float*>(st + S::kK);
+        const float* gs = reinterpret_cast<const float*>(st + S::kG);
+        const float* vs = reinterpret_cast<const float*>(st + S::kV);
+        float Vr[kLrbMaxRank];
+#pragma unroll
+        for (int l = 0; l < kLrbMaxRank; ++l) Vr[l] = Vn[l];
+        // the next tile's copies go to the other stage, freed at the end of
+        // the previous tile
+        const int next = tile + gridDim.x;
+        if (next < p.ntiles) {
+            if (j == 0 && !p.inject) {
+                lrb_issue<DK, DV, GROUP, GATE>(p, &bars[stage ^ 1],
+                                               smem + S::kStage0 + (stage ^ 1) * S::kStage,
+                                               lrb_layout(p, next, G, GROUP * DV), next, m);
+                ++issued;
+            }
+            load_v(next, Vn);
+        }
+        const TileLayout tl = lrb_layout(p, tile, G, GROUP * DV);
+        ok = __syncthreads_and(
+            mbar_wait_bounded(&bars[stage], static_cast<uint32_t>((n >> 1) & 1), p.timeout_ns));
+        if (!ok) break;
         if (!tl.ok) {
             if (j == 0) atomicOr(p.err, kErrLayout);
+            __syncthreads();
             continue;
         }
+        const int b = tile / p.H, h = tile - b * p.H;
         const uint32_t cbytes = static_cast<uint32_t>(tl.goff(G, GROUP * DV / 2));
         float* Ug = p.U + static_cast<int64_t>(tile) * r * DK;
         float* Vg = p.V + static_cast<int64_t>(tile) * r * DV;
-        if (j == 0 && !p.inject) {
-            fence_proxy_async_smem();        // earlier shared reads before the copies land
-            const uint64_t pol = policy_evict_first();
-            const int64_t row = static_cast<int64_t>(tile) * DK;
-            uint32_t bytes = cbytes + G * DV * 4 + 2 * DK * 4 + DV * 4;
-            if (GATE == kGatePerKey) bytes += DK * 4;
-            if (m > 0) bytes += m * DK * 4;
-            mbar_arrive_expect_tx(bar, bytes);
-            bulk_g2s(cs, p.codes + tl.code_off, cbytes, bar, pol);
-            bulk_g2s(ss, p.scales + static_cast<int64_t>(tile) * G * DV, G * DV * 4, bar, pol);
-            if (m > 0) bulk_g2s(Us, Ug, m * DK * 4, bar, pol);
-            bulk_g2s(smem + S::kQ, p.q + row, DK * 4, bar, pol);
-            bulk_g2s(smem + S::kK, p.k + row, DK * 4, bar, pol);
-            if (GATE == kGatePerKey) bulk_g2s(smem + S::kG, p.gates + row, DK * 4, bar, pol);
-            bulk_g2s(smem + S::kV, p.v + static_cast<int64_t>(tile) * DV, DV * 4, bar, pol);
-        }
-        // V[l][j] of the filled components, plain loads (coalesced across j)
-        float Vr[kLrbMaxRank];
-#pragma unroll
-        for (int l = 0; l < kLrbMaxRank; ++l) Vr[l] = l < m ? __ldcs(Vg + l * DV + j) : 0.0f;
-        ok = __syncthreads_and(mbar_wait_bounded(bar, par, p.timeout_ns));
-        if (!ok) {
-            if (j == 0) {
-                atomicOr(p.err, kErrTimeout);
-                mbar_wait_bounded(bar, par, p.timeout_ns);   // bounded drain of the copies
-            }
-            break;
-        }
-        par ^= 1u;
         const float alpha = GATE == kGate ? __ldg(p.gates + tile) : 0.0f;
 
         float x[DK];
@@ -256,7 +306,13 @@ __global__ void __launch_bounds__(DV, (3 * 128) / DV) lrb_kernel(const LrbParams
         float* gsc = p.scales + static_cast<int64_t>(tile) * G * DV;
         for (int off = j * 4; off < G * DV; off += DV * 4)
             *reinterpret_cast<float4*>(gsc + off) = *reinterpret_cast<const float4*>(ss + off);
-        __syncthreads();                    // before the next tile's copies land
+        __syncthreads();                    // the stage is free for the tile after next
+    }
+    if (!ok && j == 0) {
+        // record the timeout, then wait (bounded) for copies still in flight
+        atomicOr(p.err, kErrTimeout);
+        for (int q = n; q < issued; ++q)
+            mbar_wait_bounded(&bars[q & 1], static_cast<uint32_t>((q >> 1) & 1), p.timeout_ns);
     }
 }
 
