@@ -1,0 +1,534 @@
+// lrb_stream.cuh -- the Low-Rank Bypass decode step on the step kernel's
+// streaming design (ranks up to 4).
+//
+// The readings are those of lrb_kernel.cuh. The mapping is the decode step's:
+// a warp owns a tile, lane t owns value columns [t*C, t*C + C) over all key
+// rows, the tile streams through a ring of scale-group slots. What the bypass
+// adds per tile:
+//   - the buffer's U rows (filled components) arrive with the tile's first
+//     group, in the tile-input buffer; each lane loads its columns of V;
+//   - the per-component chains e_l = k . U_l (delta rule) and
+//     f_l = q . RN(g U_l) (and f_m = q . k) run in key order on lanes 0..3
+//     and 16..20 at once, then reach every lane by shuffles;
+//   - U is decayed in place and k appended; the lane appends w to its V;
+//   - the quantized part takes x = RN(g deq); at a merge step every element
+//     adds its buffer value sum_l U'_l,i V'_l,j when it is at least half a
+//     quantization step;
+//   - the output adds sum_l f_l V'_l,j after the key-order chain;
+//   - U' and V' (or zeros after a merge) go back to global memory.
+// All modes use the staged pair code (updated values in shared memory).
+#pragma once
+
+#include "step_kernel.cuh"
+
+namespace lrs {
+
+constexpr int kLrbStreamMaxRank = 4;
+
+struct LrbStreamParams {
+    StepParams s;         // the decode step's parameters (state, inputs, ring)
+    float* U;             // [ntiles][rank][d_k]
+    float* V;             // [ntiles][rank][d_v]
+    int32_t rank, m;      // rank, components filled before the step (step mod rank)
+};
+
+// Per-warp shared memory: barriers | two tile-input buffers | slots | x staging.
+// Tile-input buffer: q, k, [gate] (d_k fp32 each) | v (d_v) | U (4 rows of d_k).
+template <int C, int GROUP, int GATE>
+struct LrbSlot {
+    static constexpr int DV = 32 * C;
+    static constexpr int kCodes = GROUP * DV;
+    static constexpr int kScales = kCodes;
+    static constexpr int kBytes = kScales + DV * 4;
+    static constexpr int kXsBytes = GROUP * 256;
+    __host__ __device__ static int in_k(int d_k) { return d_k * 4; }
+    __host__ __device__ static int in_g(int d_k) { return 2 * d_k * 4; }
+    __host__ __device__ static int in_v(int d_k) {
+        return 2 * d_k * 4 + (GATE == kGatePerKey ? d_k * 4 : 0);
+    }
+    __host__ __device__ static int in_u(int d_k) { return in_v(d_k) + DV * 4; }
+    __host__ __device__ static int tile_in_bytes(int d_k) {
+        return (in_u(d_k) + kLrbStreamMaxRank * d_k * 4 + 15) / 16 * 16;
+    }
+    __host__ __device__ static int header(int d_k) { return 128 + 2 * tile_in_bytes(d_k); }
+    static int warp_bytes(int slots, int d_k) {
+        return (header(d_k) + slots * kBytes + kXsBytes + 127) / 128 * 128;
+    }
+};
+
+// Group g of the cursor's tile into `slot` (lane 0); with the first group the
+// tile's q, k, gates, v and filled U rows into `tin`.
+template <int C, int GROUP, int GATE>
+__device__ __forceinline__ void lrb_issue_item(const LrbStreamParams& lp, uint8_t* wsm, int slot,
+                                               const TileCursor& tc, int g, uint8_t* tin,
+                                               uint64_t pol_state, uint64_t pol_in) {
+    using S = LrbSlot<C, GROUP, GATE>;
+    constexpr int DV = 32 * C;
+    const StepParams& p = lp.s;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(wsm) + slot;
+    if (!tc.ok) {
+        mbar_arrive(bar);
+        return;
+    }
+    const int tile = tc.tile;
+    const int dk = p.d_k;
+    uint8_t* sm = wsm + S::header(dk) + slot * S::kBytes;
+    const uint32_t cbytes = GROUP * DV * tc.bits(g) / 8;
+    uint32_t total = cbytes + DV * 4;
+    if (g == 0) total += S::in_u(dk) + lp.m * dk * 4;
+    mbar_arrive_expect_tx(bar, total);
+    bulk_g2s(sm, p.codes + tc.code_off + tc.goff(g, GROUP * DV / 2), cbytes, bar, pol_state);
+    bulk_g2s(sm + S::kScales, p.scales + (static_cast<int64_t>(tile) * p.G + g) * DV, DV * 4, bar,
+             pol_state);
+    if (g == 0) {
+        const int64_t rowbase = static_cast<int64_t>(tile) * dk;
+        bulk_g2s(tin, static_cast<const float*>(p.q) + rowbase, dk * 4, bar, pol_in);
+        bulk_g2s(tin + S::in_k(dk), static_cast<const float*>(p.k) + rowbase, dk * 4, bar, pol_in);
+        if (GATE == kGatePerKey) bulk_g2s(tin + S::in_g(dk), p.gates + rowbase, dk * 4, bar, pol_in);
+        bulk_g2s(tin + S::in_v(dk), static_cast<const float*>(p.v) + static_cast<int64_t>(tile) * DV,
+                 DV * 4, bar, pol_in);
+        if (lp.m > 0)
+            bulk_g2s(tin + S::in_u(dk), lp.U + static_cast<int64_t>(tile) * lp.rank * dk,
+                     lp.m * dk * 4, bar, pol_state);
+    }
+}
+
+// One column pair of one scale group with the bypass: x = RN(g deq), plus at
+// a merge step the buffer's element where it reaches half a quantization
+// step; then the output chain, new scales and codes as pair_step_xs.
+// Ut: U' (decayed, appended; component-major, d_k floats per component) at
+// the group's first row. vc0, vc1: V'[l] of the pair's two columns.
+template <int GROUP, int GATE, int MODE, int BITS>
+__device__ __forceinline__ void pair_step_lrb(const uint8_t* __restrict__ cs, int ubase, float2 sc,
+                                              const float* __restrict__ qs,
+                                              const float* __restrict__ gs, float gscalar,
+                                              float2& o, uint8_t* __restrict__ gcodes,
+                                              float* __restrict__ gscale, uint64_t hkey, int row0,
+                                              uint32_t j0, int lane, float4* __restrict__ xs,
+                                              bool merge, int R, const float* __restrict__ Ut,
+                                              int dk, const float (&vc0)[kLrbStreamMaxRank],
+                                              const float (&vc1)[kLrbStreamMaxRank]) {
+    using G = PairGeo<GROUP, BITS>;
+    constexpr float BIAS = Q<BITS>::kBias;
+    constexpr int RPUH = G::RPU / 2;
+    const float2 s0 = f2(sc.x), s1 = f2(sc.y);
+    const float2 gsc = f2(gscalar);
+    const float half0 = __fmul_rn(0.5f, sc.x), half1 = __fmul_rn(0.5f, sc.y);
+    float a0 = 0.0f, b0 = 0.0f;
+
+#pragma unroll 1
+    for (int un = 0; un < G::UNITS; ++un) {
+        const uint4 raw = lds_unit(cs, ubase + un, lane);
+        const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+        float qq[G::RPU], gg[G::RPU];
+        ld_smem_rows<G::RPU>(qs + un * G::RPU, qq);
+        if constexpr (GATE == kGatePerKey) ld_smem_rows<G::RPU>(gs + un * G::RPU, gg);
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+            float f[G::EPW];
+            decode_word_biased<BITS>(wd[wi], f);
+#pragma unroll
+            for (int rp = 0; rp < G::RPW / 2; ++rp) {
+                const int rl = wi * G::RPW + 2 * rp;
+                const float2 qr = make_float2(qq[rl], qq[rl + 1]);
+                const float2 gr = GATE == kGatePerKey ? make_float2(gg[rl], gg[rl + 1]) : gsc;
+                const float2 c0 = add2(make_float2(f[4 * rp], f[4 * rp + 2]), f2(-(kTwo23 + BIAS)));
+                const float2 c1 = add2(make_float2(f[4 * rp + 1], f[4 * rp + 3]), f2(-(kTwo23 + BIAS)));
+                float2 x0 = mul2(gr, mul2(c0, s0));
+                float2 x1 = mul2(gr, mul2(c1, s1));
+                // the output reads the state part before a merge (the buffer's
+                // share is added from f_l after the tile)
+                o.x = __fmaf_rn(qr.x, x0.x, o.x);
+                o.x = __fmaf_rn(qr.y, x0.y, o.x);
+                o.y = __fmaf_rn(qr.x, x1.x, o.y);
+                o.y = __fmaf_rn(qr.y, x1.y, o.y);
+                if (merge) {
+                    // M = sum_l U'_l,i V'_l,j (fma chain in component order)
+                    const int r = un * G::RPU + rl;
+                    float2 m0 = f2(0.0f), m1 = f2(0.0f);
+#pragma unroll
+                    for (int l = 0; l < kLrbStreamMaxRank; ++l) {
+                        if (l < R) {
+                            const float2 u = *reinterpret_cast<const float2*>(Ut + l * dk + r);
+                            m0 = fma2(u, f2(vc0[l]), m0);
+                            m1 = fma2(u, f2(vc1[l]), m1);
+                        }
+                    }
+                    const float2 y0 = add2(x0, m0), y1 = add2(x1, m1);
+                    x0.x = (m0.x != 0.0f && fabsf(m0.x) >= half0) ? y0.x : x0.x;
+                    x0.y = (m0.y != 0.0f && fabsf(m0.y) >= half0) ? y0.y : x0.y;
+                    x1.x = (m1.x != 0.0f && fabsf(m1.x) >= half1) ? y1.x : x1.x;
+                    x1.y = (m1.y != 0.0f && fabsf(m1.y) >= half1) ? y1.y : x1.y;
+                }
+                a0 = max_abs3(a0, x0.x, x0.y);
+                b0 = max_abs3(b0, x1.x, x1.y);
+                xs[(un * RPUH + rl / 2) * 32 + lane] = make_float4(x0.x, x0.y, x1.x, x1.y);
+            }
+        }
+    }
+
+    float2 snew, inv;
+    new_scales<BITS>(a0, b0, snew, inv);
+    st_cs_f2(gscale, snew);
+    const float2 inv0 = f2(inv.x), inv1 = f2(inv.y);
+    const float2 sn0 = f2(snew.x), sn1 = f2(snew.y);
+
+#pragma unroll 1
+    for (int un = 0; un < G::UNITS; ++un) {
+        uint32_t ow[4];
+        uint32_t wd[4] = {0u, 0u, 0u, 0u};
+        if constexpr (MODE == kBDR) {
+            const uint4 raw = lds_unit(cs, ubase + un, lane);
+            wd[0] = raw.x; wd[1] = raw.y; wd[2] = raw.z; wd[3] = raw.w;
+        }
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+            float f[G::EPW];
+            if constexpr (MODE == kBDR) decode_word_biased<BITS>(wd[wi], f);
+            float t[G::EPW];
+#pragma unroll
+            for (int rp = 0; rp < G::RPW / 2; ++rp) {
+                const int rl = wi * G::RPW + 2 * rp;
+                const float4 xv = xs[(un * RPUH + rl / 2) * 32 + lane];
+                float2 dq0 = f2(0.0f), dq1 = f2(0.0f);
+                if constexpr (MODE == kBDR) {
+                    dq0 = mul2(add2(make_float2(f[4 * rp], f[4 * rp + 2]), f2(-(kTwo23 + BIAS))), s0);
+                    dq1 = mul2(add2(make_float2(f[4 * rp + 1], f[4 * rp + 3]), f2(-(kTwo23 + BIAS))), s1);
+                }
+                const uint32_t i = static_cast<uint32_t>(row0 + un * G::RPU + rl);
+                const float2 kb0 = make_float2(word_bias<BITS>(4 * rp), word_bias<BITS>(4 * rp + 2));
+                const float2 kb1 = make_float2(word_bias<BITS>(4 * rp + 1), word_bias<BITS>(4 * rp + 3));
+                const float2 t0 = round_rows<MODE, BITS>(make_float2(xv.x, xv.y), inv0, dq0, sn0,
+                                                         kb0, hkey, i, j0);
+                const float2 t1 = round_rows<MODE, BITS>(make_float2(xv.z, xv.w), inv1, dq1, sn1,
+                                                         kb1, hkey, i, j0 + 1);
+                t[4 * rp] = t0.x;
+                t[4 * rp + 2] = t0.y;
+                t[4 * rp + 1] = t1.x;
+                t[4 * rp + 3] = t1.y;
+            }
+            ow[wi] = encode_word<BITS>(t);
+        }
+        st_cs_u4(gcodes + ((ubase + un) * 32 + lane) * 16, ow[0], ow[1], ow[2], ow[3]);
+    }
+}
+
+// Key-order chain c = sum_i a_i * RN(gm_i * b_i) over n rows (gm = 1 when
+// !decay, exactly b_i then), for one lane's role.
+__device__ __forceinline__ float lrb_chain(const float* a, const float* b, const float* gk,
+                                           float gscalar, bool per_key, bool decay, int n) {
+    float c = 0.0f;
+#pragma unroll 4
+    for (int i = 0; i < n; ++i) {
+        float bi = b[i];
+        if (decay) bi = __fmul_rn(per_key ? gk[i] : gscalar, bi);
+        c = __fmaf_rn(a[i], bi, c);
+    }
+    return c;
+}
+
+// The warp's items are (tile, group) pairs as in step_kernel.
+template <int C, int GROUP, int UPD, int GATE, int MODE>
+__global__ void __launch_bounds__(8 * 32, 1) lrb_step_kernel(const LrbStreamParams lp) {
+    using S = LrbSlot<C, GROUP, GATE>;
+    constexpr int DV = 32 * C;
+    constexpr int P = C / 2;
+    constexpr int MR = kLrbStreamMaxRank;
+    const StepParams& p = lp.s;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int lane = threadIdx.x & 31;
+    const int wib = threadIdx.x >> 5;
+    const int nw = blockDim.x >> 5;
+    const int W = gridDim.x * nw;
+    const int gw = blockIdx.x * nw + wib;
+    uint8_t* wsm = smem + wib * p.warp_smem;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(wsm);
+    const int G = p.G, NS = p.slots, dk = p.d_k;
+    const int hdr = S::header(dk), tib = S::tile_in_bytes(dk);
+    const int in_k = S::in_k(dk), in_g = S::in_g(dk), in_v = S::in_v(dk), in_u = S::in_u(dk);
+    float4* xs = reinterpret_cast<float4*>(wsm + hdr + NS * S::kBytes);
+    const int ntw = gw < p.ntiles ? (p.ntiles - gw + W - 1) / W : 0;
+    const int64_t K = static_cast<int64_t>(ntw) * G;
+    const int R = lp.rank, m = lp.m;
+    const bool merge = m + 1 == R;
+
+    if (lane == 0) {
+        for (int s = 0; s < NS; ++s) mbar_init(&bars[s], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    const uint64_t pol_state = policy_evict_first();
+    const uint64_t pol_in = policy_evict_first();
+    Ring ic, is;
+    int64_t kc = 0, ki = 0;
+    int it_g = 0, it_n = 0;
+    TileCursor itc;
+    itc.init(p, gw, W);
+    if (K > 0) itc.load(p, GROUP * DV);
+
+    auto issue_next = [&]() {
+        if (ki < K && !p.inject) {
+            if (lane == 0)
+                lrb_issue_item<C, GROUP, GATE>(lp, wsm, is.slot, itc, it_g,
+                                               wsm + 128 + (it_n & 1) * tib, pol_state, pol_in);
+            ++ki;
+            is.advance(NS);
+            if (++it_g == G) {
+                it_g = 0;
+                ++it_n;
+                itc.advance(p, W);
+                if (ki < K) itc.load(p, GROUP * DV);
+            }
+        }
+    };
+    for (int s = 0; s < NS; ++s) issue_next();
+
+    bool ok = true;
+    TileCursor ti;
+    ti.init(p, gw, W);
+    for (int n = 0; n < ntw && ok; ++n, ti.advance(p, W)) {
+        const int tile = ti.tile;
+        ti.load(p, GROUP * DV);
+        uint8_t* tin = wsm + 128 + (n & 1) * tib;
+        const float gscalar = GATE == kGate ? __ldg(p.gates + tile) : 0.0f;
+        const float beta = UPD == kDelta ? __ldg(p.beta + tile) : 0.0f;
+        const uint64_t hkey = MODE == kSR ? tile_hash_key(p.seed, p.step,
+                                                          static_cast<uint32_t>(ti.b),
+                                                          static_cast<uint32_t>(ti.h))
+                                          : 0ull;
+        // V of this lane's columns for the filled components
+        float Vc[MR][C];
+        const float* Vg = lp.V + static_cast<int64_t>(tile) * R * DV + lane * C;
+#pragma unroll
+        for (int l = 0; l < MR; ++l)
+#pragma unroll
+            for (int c = 0; c < C; ++c) Vc[l][c] = (l < m && ti.ok) ? __ldcs(Vg + l * DV + c) : 0.0f;
+
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[ic.slot], ic.par, p.timeout_ns));
+        if (!ok) break;
+        if (!ti.ok) {
+            if (lane == 0) atomicOr(p.err, kErrLayout);
+            for (int g = 0; g < G; ++g) {
+                if (g > 0) {
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait_bounded(&bars[ic.slot], ic.par, p.timeout_ns));
+                    if (!ok) break;
+                }
+                ++kc;
+                ic.advance(NS);
+                __syncwarp();
+                issue_next();
+            }
+            continue;
+        }
+        const float* qs_t = reinterpret_cast<const float*>(tin);
+        const float* ks_t = reinterpret_cast<const float*>(tin + in_k);
+        const float* gs_t = reinterpret_cast<const float*>(tin + in_g);
+        const uint8_t* vs_t = tin + in_v;
+        float* Ut = reinterpret_cast<float*>(tin + in_u);
+
+        // the component chains: e_l = k . U_l (lanes 0..m-1, delta rule) and
+        // f_l = q . RN(g U_l), f_m = q . k (lanes 16..16+m), all at once
+        float chain = 0.0f;
+        {
+            const int le = lane, lf = lane - 16;
+            if (UPD == kDelta && le < m)
+                chain = lrb_chain(ks_t, Ut + le * dk, gs_t, gscalar, false, false, dk);
+            else if (lf >= 0 && lf <= m)
+                chain = lf < m ? lrb_chain(qs_t, Ut + lf * dk, gs_t, gscalar, GATE == kGatePerKey,
+                                           true, dk)
+                               : lrb_chain(qs_t, ks_t, gs_t, gscalar, false, false, dk);
+        }
+        float e[MR], f[MR + 1];
+#pragma unroll
+        for (int l = 0; l < MR; ++l) e[l] = __shfl_sync(0xffffffffu, chain, l);
+#pragma unroll
+        for (int l = 0; l <= MR; ++l) f[l] = __shfl_sync(0xffffffffu, chain, 16 + l);
+        __syncwarp();
+        // decay the buffer in place and append k
+        for (int i = lane; i < dk; i += 32) {
+            const float gi = GATE == kGatePerKey ? gs_t[i] : gscalar;
+            for (int l = 0; l < m; ++l) Ut[l * dk + i] = __fmul_rn(gi, Ut[l * dk + i]);
+            Ut[m * dk + i] = ks_t[i];
+        }
+        __syncwarp();
+
+        float2 w[P], o[P];
+#pragma unroll
+        for (int pc = 0; pc < P; ++pc) o[pc] = f2(0.0f);
+        if (UPD == kDelta) {
+            float2 u[P];
+#pragma unroll
+            for (int pc = 0; pc < P; ++pc) u[pc] = f2(0.0f);
+            Ring r = ic;
+            for (int g = 0; g < G && ok; ++g) {
+                if (g > 0)
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait_bounded(&bars[r.slot], r.par, p.timeout_ns));
+                if (!ok) break;
+                const uint8_t* sm = wsm + hdr + r.slot * S::kBytes;
+                const float* ss = reinterpret_cast<const float*>(sm + S::kScales) + lane * C;
+                const uint8_t* ks = tin + in_k + g * GROUP * 4;
+                float2 up = u[0], uq = u[P - 1];
+#pragma unroll 1
+                for (int pc = 0; pc < P; ++pc) {
+                    const float2 sc = *reinterpret_cast<const float2*>(ss + 2 * pc);
+                    if (ti.bits(g) == 8)
+                        pair_ktS<GROUP, 8, kIoF32>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, ks, lane, up);
+                    else
+                        pair_ktS<GROUP, 4, kIoF32>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, ks, lane, up);
+                    if constexpr (P == 2) {
+                        const float2 t = up;
+                        up = uq; uq = t;
+                    }
+                }
+                u[0] = up;
+                u[P - 1] = P == 2 ? uq : up;
+                r.advance(NS);
+            }
+            if (!ok) break;
+#pragma unroll
+            for (int pc = 0; pc < P; ++pc) {
+                // u += sum_l e_l V_l (undecayed buffer), component order
+#pragma unroll
+                for (int l = 0; l < MR; ++l)
+                    if (l < m) {
+                        u[pc].x = __fmaf_rn(e[l], Vc[l][2 * pc], u[pc].x);
+                        u[pc].y = __fmaf_rn(e[l], Vc[l][2 * pc + 1], u[pc].y);
+                    }
+                const float2 vv = ld_pair<kIoF32>(vs_t, lane * C + 2 * pc);
+                const float d0 = __fsub_rn(vv.x, __fmul_rn(gscalar, u[pc].x));
+                const float d1 = __fsub_rn(vv.y, __fmul_rn(gscalar, u[pc].y));
+                w[pc] = make_float2(__fmul_rn(beta, d0), __fmul_rn(beta, d1));
+            }
+        } else {
+#pragma unroll
+            for (int pc = 0; pc < P; ++pc) w[pc] = ld_pair<kIoF32>(vs_t, lane * C + 2 * pc);
+        }
+        // append w to V
+#pragma unroll
+        for (int l = 0; l < MR; ++l)
+            if (l == m) {
+#pragma unroll
+                for (int pc = 0; pc < P; ++pc) {
+                    Vc[l][2 * pc] = w[pc].x;
+                    Vc[l][2 * pc + 1] = w[pc].y;
+                }
+            }
+
+        uint8_t* gcodes_tile = p.codes + ti.code_off;
+        for (int g = 0; g < G; ++g) {
+            if (UPD != kDelta && g > 0) {
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait_bounded(&bars[ic.slot], ic.par, p.timeout_ns));
+                if (!ok) break;
+            }
+            const uint8_t* sm = wsm + hdr + ic.slot * S::kBytes;
+            const float* ss = reinterpret_cast<const float*>(sm + S::kScales) + lane * C;
+            const float* qs = qs_t + g * GROUP;
+            const float* gs = gs_t + g * GROUP;
+            float* gscale = p.scales + (static_cast<int64_t>(tile) * G + g) * DV + lane * C;
+            uint8_t* gcodes = gcodes_tile + ti.goff(g, GROUP * DV / 2);
+            const bool int8g = ti.bits(g) == 8;
+            const float* Ug = Ut + g * GROUP;
+            float2 op = o[0], oq = o[P - 1];
+#pragma unroll 1
+            for (int pc = 0; pc < P; ++pc) {
+                const float2 sc = *reinterpret_cast<const float2*>(ss + 2 * pc);
+                const uint32_t j0 = static_cast<uint32_t>(lane * C + 2 * pc);
+                float vc0[MR], vc1[MR];
+#pragma unroll
+                for (int l = 0; l < MR; ++l) {
+                    vc0[l] = pc == 0 ? Vc[l][0] : Vc[l][C - 2];
+                    vc1[l] = pc == 0 ? Vc[l][1] : Vc[l][C - 1];
+                }
+                if (int8g)
+                    pair_step_lrb<GROUP, GATE, MODE, 8>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs, gs,
+                                                        gscalar, op, gcodes, gscale + 2 * pc, hkey,
+                                                        g * GROUP, j0, lane, xs, merge, R, Ug, dk,
+                                                        vc0, vc1);
+                else
+                    pair_step_lrb<GROUP, GATE, MODE, 4>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs, gs,
+                                                        gscalar, op, gcodes, gscale + 2 * pc, hkey,
+                                                        g * GROUP, j0, lane, xs, merge, R, Ug, dk,
+                                                        vc0, vc1);
+                if constexpr (P == 2) {
+                    const float2 to = op;
+                    op = oq; oq = to;
+                }
+            }
+            o[0] = op;
+            o[P - 1] = P == 2 ? oq : op;
+            ++kc;
+            ic.advance(NS);
+            __syncwarp();
+            if (lane == 0) fence_proxy_async_smem();
+            issue_next();
+        }
+        if (!ok) break;
+        // output: the state part's chain, then the buffer's share in component order
+        float ov[C];
+#pragma unroll
+        for (int pc = 0; pc < P; ++pc) {
+            ov[2 * pc] = o[pc].x;
+            ov[2 * pc + 1] = o[pc].y;
+        }
+#pragma unroll
+        for (int l = 0; l <= MR; ++l)
+            if (l <= m)
+#pragma unroll
+                for (int c = 0; c < C; ++c) ov[c] = __fmaf_rn(f[l], Vc[l < MR ? l : 0][c], ov[c]);
+        float* outp = static_cast<float*>(p.out) + static_cast<int64_t>(tile) * DV + lane * C;
+#pragma unroll
+        for (int c = 0; c < C; ++c) outp[c] = ov[c];
+        // the buffer back to global memory (emptied after a merge)
+        float* Ugl = lp.U + static_cast<int64_t>(tile) * R * dk;
+        for (int idx = lane * 4; idx < (m + 1) * dk; idx += 128) {
+            const float4 t = merge ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                   : *reinterpret_cast<const float4*>(Ut + idx);
+            *reinterpret_cast<float4*>(Ugl + idx) = t;
+        }
+        float* Vgl = lp.V + static_cast<int64_t>(tile) * R * DV + lane * C;
+#pragma unroll
+        for (int l = 0; l < MR; ++l)
+            if (l <= m)
+#pragma unroll
+                for (int c = 0; c < C; ++c) Vgl[l * DV + c] = merge ? 0.0f : Vc[l][c];
+        __syncwarp();
+    }
+    if (!ok) {
+        if (lane == 0) atomicOr(p.err, kErrTimeout);
+        Ring r = ic;
+        for (int64_t k = kc; k < ki; ++k) {
+            mbar_wait_bounded(&bars[r.slot], r.par, p.timeout_ns);
+            r.advance(NS);
+        }
+    }
+}
+
+// Defines `ChunkKernel NAME(C, group, update_kind, gate_kind)`: the streaming
+// bypass kernel with rounding MODE; smem is the per-warp bytes for d_k = 128
+// (the host recomputes it for the actual d_k).
+#define LRS_LRB_STREAM_PICK1(MODE, CC, GG)                                                     \
+    if (C == CC && group == GG) {                                                              \
+        if (update_kind == kGated && gate_kind == kGatePerKey)                                 \
+            return reinterpret_cast<const void*>(                                              \
+                &lrb_step_kernel<CC, GG, kGated, kGatePerKey, MODE>);                          \
+        if (update_kind == kGated && gate_kind == kGate)                                       \
+            return reinterpret_cast<const void*>(&lrb_step_kernel<CC, GG, kGated, kGate, MODE>); \
+        if (update_kind == kDelta && gate_kind == kGate)                                       \
+            return reinterpret_cast<const void*>(&lrb_step_kernel<CC, GG, kDelta, kGate, MODE>); \
+        return nullptr;                                                                        \
+    }
+#define LRS_LRB_STREAM_VARIANTS(NAME, MODE)                                                    \
+    const void* NAME(int C, int group, int update_kind, int gate_kind) {                       \
+        LRS_LRB_STREAM_PICK1(MODE, 4, 16)                                                      \
+        LRS_LRB_STREAM_PICK1(MODE, 4, 32)                                                      \
+        LRS_LRB_STREAM_PICK1(MODE, 2, 16)                                                      \
+        LRS_LRB_STREAM_PICK1(MODE, 2, 32)                                                      \
+        LRS_LRB_STREAM_PICK1(MODE, 2, 64)                                                      \
+        return nullptr;                                                                        \
+    }
+
+}  // namespace lrs

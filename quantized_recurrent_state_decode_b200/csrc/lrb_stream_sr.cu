@@ -1,0 +1,8 @@
+// lrb_stream_sr.cu -- compiled variants of the streaming Low-Rank Bypass
+// decode step, SR rounding.
+#include "lrb_stream.cuh"
+#include "lrs_internal.h"
+
+namespace lrs {
+LRS_LRB_STREAM_VARIANTS(find_lrb_stream_sr, kSR)
+}  // namespace lrs

@@ -57,11 +57,14 @@ GRID = [(fam, mode) for fam in ("gla", "gdn", "mamba2")
 
 @pytest.mark.parametrize("fam,mode", GRID)
 @pytest.mark.parametrize("prec", ["int8", "mixed"])
-def test_lrb_family_mode_grid(fam, mode, prec):
+@pytest.mark.parametrize("rank", [4, 6])
+def test_lrb_family_mode_grid(fam, mode, prec, rank):
+    """Ranks up to 4 run the streaming kernel, larger ones the one-CTA-per-tile
+    kernel; both must match the oracle."""
     d_v = 64 if fam == "mamba2" else 128
     group = {"gla": 32, "gdn": 16, "mamba2": 64}[fam]
-    w = _small(fam, 3, 5, 128, d_v, group, mode, prec, steps=9)
-    run_lrb(w, rank=4, steps=9)
+    w = _small(fam, 3, 5, 128, d_v, group, mode, prec, steps=rank + 3)
+    run_lrb(w, rank=rank, steps=rank + 3)
 
 
 @pytest.mark.parametrize("rank", [1, 2, 3, 8])
