@@ -70,12 +70,12 @@ const void* find_lrb_stream(int C, int group, int update_kind, int gate_kind, in
     }
 }
 
-int lrb_stream_warp_smem(int C, int group, int gate_kind, int slots, int d_k) {
+int lrb_stream_warp_smem(int C, int group, int gate_kind, int slots, int d_k, bool staged) {
 #define LRS_LRB_SLOT(CC, GG)                                                                  \
     if (C == CC && group == GG)                                                               \
         return gate_kind == lrs::kGatePerKey                                                  \
-                   ? lrs::LrbSlot<CC, GG, lrs::kGatePerKey>::warp_bytes(slots, d_k)            \
-                   : lrs::LrbSlot<CC, GG, lrs::kGate>::warp_bytes(slots, d_k);
+                   ? lrs::LrbSlot<CC, GG, lrs::kGatePerKey>::warp_bytes(slots, d_k, staged)    \
+                   : lrs::LrbSlot<CC, GG, lrs::kGate>::warp_bytes(slots, d_k, staged);
     LRS_LRB_SLOT(4, 16)
     LRS_LRB_SLOT(4, 32)
     LRS_LRB_SLOT(2, 16)
@@ -99,9 +99,10 @@ lrs_status launch_lrb_stream(const lrs_state* st, void* state_codes, float* scal
     if (!fn || rank > lrs::kLrbStreamMaxRank) return LRS_ERR_UNSUPPORTED;
     int slots = sh.update_kind == LRS_UPDATE_DELTA ? G : std::min(2, G);
     slots = std::max(1, std::min(slots, lrs::kMaxSlots));
-    const int warp_smem = lrb_stream_warp_smem(C, sh.group, sh.gate_kind, slots, sh.d_k);
+    const int warp_smem =
+        lrb_stream_warp_smem(C, sh.group, sh.gate_kind, slots, sh.d_k, mode != LRS_ROUND_RTN);
     constexpr int kSmemLimit = 227 * 1024;
-    const int warps = std::min(8, kSmemLimit / warp_smem);
+    const int warps = std::min(lrs::lrb_max_warps(mode), kSmemLimit / warp_smem);
     if (warps < 1) return LRS_ERR_UNSUPPORTED;
     const int smem = warps * warp_smem;
     static std::mutex mu;

@@ -33,7 +33,8 @@ struct LrbStreamParams {
 };
 
 // Per-warp shared memory: barriers | two tile-input buffers | slots | x staging.
-// Tile-input buffer: q, k, [gate] (d_k fp32 each) | v (d_v) | U (4 rows of d_k).
+// Tile-input buffer: q, k, [gate] (d_k fp32 each) | v (d_v) | U (4 rows of
+// d_k) | V (4 rows of d_v).
 template <int C, int GROUP, int GATE>
 struct LrbSlot {
     static constexpr int DV = 32 * C;
@@ -47,12 +48,13 @@ struct LrbSlot {
         return 2 * d_k * 4 + (GATE == kGatePerKey ? d_k * 4 : 0);
     }
     __host__ __device__ static int in_u(int d_k) { return in_v(d_k) + DV * 4; }
+    __host__ __device__ static int in_vb(int d_k) { return in_u(d_k) + kLrbStreamMaxRank * d_k * 4; }
     __host__ __device__ static int tile_in_bytes(int d_k) {
-        return (in_u(d_k) + kLrbStreamMaxRank * d_k * 4 + 15) / 16 * 16;
+        return (in_vb(d_k) + kLrbStreamMaxRank * DV * 4 + 15) / 16 * 16;
     }
     __host__ __device__ static int header(int d_k) { return 128 + 2 * tile_in_bytes(d_k); }
-    static int warp_bytes(int slots, int d_k) {
-        return (header(d_k) + slots * kBytes + kXsBytes + 127) / 128 * 128;
+    static int warp_bytes(int slots, int d_k, bool staged) {
+        return (header(d_k) + slots * kBytes + (staged ? kXsBytes : 0) + 127) / 128 * 128;
     }
 };
 
@@ -75,7 +77,7 @@ __device__ __forceinline__ void lrb_issue_item(const LrbStreamParams& lp, uint8_
     uint8_t* sm = wsm + S::header(dk) + slot * S::kBytes;
     const uint32_t cbytes = GROUP * DV * tc.bits(g) / 8;
     uint32_t total = cbytes + DV * 4;
-    if (g == 0) total += S::in_u(dk) + lp.m * dk * 4;
+    if (g == 0) total += S::in_u(dk) + lp.m * (dk + DV) * 4;
     mbar_arrive_expect_tx(bar, total);
     bulk_g2s(sm, p.codes + tc.code_off + tc.goff(g, GROUP * DV / 2), cbytes, bar, pol_state);
     bulk_g2s(sm + S::kScales, p.scales + (static_cast<int64_t>(tile) * p.G + g) * DV, DV * 4, bar,
@@ -87,9 +89,12 @@ __device__ __forceinline__ void lrb_issue_item(const LrbStreamParams& lp, uint8_
         if (GATE == kGatePerKey) bulk_g2s(tin + S::in_g(dk), p.gates + rowbase, dk * 4, bar, pol_in);
         bulk_g2s(tin + S::in_v(dk), static_cast<const float*>(p.v) + static_cast<int64_t>(tile) * DV,
                  DV * 4, bar, pol_in);
-        if (lp.m > 0)
+        if (lp.m > 0) {
             bulk_g2s(tin + S::in_u(dk), lp.U + static_cast<int64_t>(tile) * lp.rank * dk,
                      lp.m * dk * 4, bar, pol_state);
+            bulk_g2s(tin + S::in_vb(dk), lp.V + static_cast<int64_t>(tile) * lp.rank * DV,
+                     lp.m * DV * 4, bar, pol_state);
+        }
     }
 }
 
@@ -213,6 +218,113 @@ __device__ __forceinline__ void pair_step_lrb(const uint8_t* __restrict__ cs, in
     }
 }
 
+// The RTN form of pair_step_lrb with the group's updated values in registers
+// (the staged form's shared-memory round trip costs more than the longer
+// per-element code of SR and BDR saves).
+template <int GROUP, int GATE, int BITS>
+__device__ __forceinline__ void pair_step_lrb_rtn(const uint8_t* __restrict__ cs, int ubase,
+                                                  float2 sc, const float* __restrict__ qs,
+                                                  const float* __restrict__ gs, float gscalar,
+                                                  float2& o, uint8_t* __restrict__ gcodes,
+                                                  float* __restrict__ gscale, int lane, bool merge,
+                                                  int R, const float* __restrict__ Ut, int dk,
+                                                  const float (&vc0)[kLrbStreamMaxRank],
+                                                  const float (&vc1)[kLrbStreamMaxRank]) {
+    using G = PairGeo<GROUP, BITS>;
+    constexpr float BIAS = Q<BITS>::kBias;
+    const float2 s0 = f2(sc.x), s1 = f2(sc.y);
+    const float2 gsc = f2(gscalar);
+    const float half0 = __fmul_rn(0.5f, sc.x), half1 = __fmul_rn(0.5f, sc.y);
+    float2 x[GROUP / 2][2];
+
+#pragma unroll
+    for (int un = 0; un < G::UNITS; ++un) {
+        const uint4 raw = lds_unit(cs, ubase + un, lane);
+        const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+        float qq[G::RPU], gg[G::RPU];
+        ld_smem_rows<G::RPU>(qs + un * G::RPU, qq);
+        if constexpr (GATE == kGatePerKey) ld_smem_rows<G::RPU>(gs + un * G::RPU, gg);
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+            float f[G::EPW];
+            decode_word_biased<BITS>(wd[wi], f);
+#pragma unroll
+            for (int rp = 0; rp < G::RPW / 2; ++rp) {
+                const int rl = wi * G::RPW + 2 * rp;
+                const int r = un * G::RPU + rl;
+                const float2 qr = make_float2(qq[rl], qq[rl + 1]);
+                const float2 gr = GATE == kGatePerKey ? make_float2(gg[rl], gg[rl + 1]) : gsc;
+                const float2 c0 = add2(make_float2(f[4 * rp], f[4 * rp + 2]), f2(-(kTwo23 + BIAS)));
+                const float2 c1 = add2(make_float2(f[4 * rp + 1], f[4 * rp + 3]), f2(-(kTwo23 + BIAS)));
+                float2 x0 = mul2(gr, mul2(c0, s0));
+                float2 x1 = mul2(gr, mul2(c1, s1));
+                o.x = __fmaf_rn(qr.x, x0.x, o.x);
+                o.x = __fmaf_rn(qr.y, x0.y, o.x);
+                o.y = __fmaf_rn(qr.x, x1.x, o.y);
+                o.y = __fmaf_rn(qr.y, x1.y, o.y);
+                x[r / 2][0] = x0;
+                x[r / 2][1] = x1;
+            }
+        }
+    }
+    if (merge) {
+        // a separate pass over the group, so the merge's values are not live
+        // beside the decode's
+#pragma unroll
+        for (int rp = 0; rp < GROUP / 2; ++rp) {
+            float2 m0 = f2(0.0f), m1 = f2(0.0f);
+#pragma unroll
+            for (int l = 0; l < kLrbStreamMaxRank; ++l) {
+                if (l < R) {
+                    const float2 u = *reinterpret_cast<const float2*>(Ut + l * dk + 2 * rp);
+                    m0 = fma2(u, f2(vc0[l]), m0);
+                    m1 = fma2(u, f2(vc1[l]), m1);
+                }
+            }
+            const float2 x0 = x[rp][0], x1 = x[rp][1];
+            const float2 y0 = add2(x0, m0), y1 = add2(x1, m1);
+            x[rp][0].x = (m0.x != 0.0f && fabsf(m0.x) >= half0) ? y0.x : x0.x;
+            x[rp][0].y = (m0.y != 0.0f && fabsf(m0.y) >= half0) ? y0.y : x0.y;
+            x[rp][1].x = (m1.x != 0.0f && fabsf(m1.x) >= half1) ? y1.x : x1.x;
+            x[rp][1].y = (m1.y != 0.0f && fabsf(m1.y) >= half1) ? y1.y : x1.y;
+        }
+    }
+    float a0 = 0.0f, a1 = 0.0f, b0 = 0.0f, b1 = 0.0f;
+#pragma unroll
+    for (int rp = 0; rp < GROUP / 2; rp += 2) {
+        a0 = max_abs3(a0, x[rp][0].x, x[rp][0].y);
+        a1 = max_abs3(a1, x[rp + 1][0].x, x[rp + 1][0].y);
+        b0 = max_abs3(b0, x[rp][1].x, x[rp][1].y);
+        b1 = max_abs3(b1, x[rp + 1][1].x, x[rp + 1][1].y);
+    }
+    float2 snew, inv;
+    new_scales<BITS>(fmaxf(a0, a1), fmaxf(b0, b1), snew, inv);
+    st_cs_f2(gscale, snew);
+    const float2 inv0 = f2(inv.x), inv1 = f2(inv.y);
+#pragma unroll
+    for (int un = 0; un < G::UNITS; ++un) {
+        uint32_t ow[4];
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+            float t[G::EPW];
+#pragma unroll
+            for (int rp = 0; rp < G::RPW / 2; ++rp) {
+                const int r = un * G::RPU + wi * G::RPW + 2 * rp;
+                const float2 kb0 = make_float2(word_bias<BITS>(4 * rp), word_bias<BITS>(4 * rp + 2));
+                const float2 kb1 = make_float2(word_bias<BITS>(4 * rp + 1), word_bias<BITS>(4 * rp + 3));
+                const float2 t0 = fma2(x[r / 2][0], inv0, kb0);
+                const float2 t1 = fma2(x[r / 2][1], inv1, kb1);
+                t[4 * rp] = t0.x;
+                t[4 * rp + 2] = t0.y;
+                t[4 * rp + 1] = t1.x;
+                t[4 * rp + 3] = t1.y;
+            }
+            ow[wi] = encode_word<BITS>(t);
+        }
+        st_cs_u4(gcodes + ((ubase + un) * 32 + lane) * 16, ow[0], ow[1], ow[2], ow[3]);
+    }
+}
+
 // Key-order chain c = sum_i a_i * RN(gm_i * b_i) over n rows (gm = 1 when
 // !decay, exactly b_i then), for one lane's role.
 __device__ __forceinline__ float lrb_chain(const float* a, const float* b, const float* gk,
@@ -228,8 +340,12 @@ __device__ __forceinline__ float lrb_chain(const float* a, const float* b, const
 }
 
 // The warp's items are (tile, group) pairs as in step_kernel.
+// Launch bound in warps: 8, so up to 255 registers (the bypass's extra
+// per-tile values do not fit beside a register-resident group in 168).
+__host__ __device__ constexpr int lrb_max_warps(int) { return 8; }
+
 template <int C, int GROUP, int UPD, int GATE, int MODE>
-__global__ void __launch_bounds__(8 * 32, 1) lrb_step_kernel(const LrbStreamParams lp) {
+__global__ void __launch_bounds__(lrb_max_warps(MODE) * 32, 1) lrb_step_kernel(const LrbStreamParams lp) {
     using S = LrbSlot<C, GROUP, GATE>;
     constexpr int DV = 32 * C;
     constexpr int P = C / 2;
@@ -297,14 +413,6 @@ __global__ void __launch_bounds__(8 * 32, 1) lrb_step_kernel(const LrbStreamPara
                                                           static_cast<uint32_t>(ti.b),
                                                           static_cast<uint32_t>(ti.h))
                                           : 0ull;
-        // V of this lane's columns for the filled components
-        float Vc[MR][C];
-        const float* Vg = lp.V + static_cast<int64_t>(tile) * R * DV + lane * C;
-#pragma unroll
-        for (int l = 0; l < MR; ++l)
-#pragma unroll
-            for (int c = 0; c < C; ++c) Vc[l][c] = (l < m && ti.ok) ? __ldcs(Vg + l * DV + c) : 0.0f;
-
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[ic.slot], ic.par, p.timeout_ns));
         if (!ok) break;
         if (!ti.ok) {
@@ -327,6 +435,7 @@ __global__ void __launch_bounds__(8 * 32, 1) lrb_step_kernel(const LrbStreamPara
         const float* gs_t = reinterpret_cast<const float*>(tin + in_g);
         const uint8_t* vs_t = tin + in_v;
         float* Ut = reinterpret_cast<float*>(tin + in_u);
+        float* Vt = reinterpret_cast<float*>(tin + S::in_vb(dk)) + lane * C;   // this lane's V
 
         // the component chains: e_l = k . U_l (lanes 0..m-1, delta rule) and
         // f_l = q . RN(g U_l), f_m = q . k (lanes 16..16+m), all at once
@@ -340,11 +449,6 @@ __global__ void __launch_bounds__(8 * 32, 1) lrb_step_kernel(const LrbStreamPara
                                            true, dk)
                                : lrb_chain(qs_t, ks_t, gs_t, gscalar, false, false, dk);
         }
-        float e[MR], f[MR + 1];
-#pragma unroll
-        for (int l = 0; l < MR; ++l) e[l] = __shfl_sync(0xffffffffu, chain, l);
-#pragma unroll
-        for (int l = 0; l <= MR; ++l) f[l] = __shfl_sync(0xffffffffu, chain, 16 + l);
         __syncwarp();
         // decay the buffer in place and append k
         for (int i = lane; i < dk; i += 32) {
@@ -388,15 +492,20 @@ __global__ void __launch_bounds__(8 * 32, 1) lrb_step_kernel(const LrbStreamPara
                 r.advance(NS);
             }
             if (!ok) break;
+            // u += sum_l e_l V_l (undecayed buffer), component order
+#pragma unroll
+            for (int l = 0; l < MR; ++l) {
+                const float el = __shfl_sync(0xffffffffu, chain, l);
+                if (l < m) {
+#pragma unroll
+                    for (int pc = 0; pc < P; ++pc) {
+                        u[pc].x = __fmaf_rn(el, Vt[l * DV + 2 * pc], u[pc].x);
+                        u[pc].y = __fmaf_rn(el, Vt[l * DV + 2 * pc + 1], u[pc].y);
+                    }
+                }
+            }
 #pragma unroll
             for (int pc = 0; pc < P; ++pc) {
-                // u += sum_l e_l V_l (undecayed buffer), component order
-#pragma unroll
-                for (int l = 0; l < MR; ++l)
-                    if (l < m) {
-                        u[pc].x = __fmaf_rn(e[l], Vc[l][2 * pc], u[pc].x);
-                        u[pc].y = __fmaf_rn(e[l], Vc[l][2 * pc + 1], u[pc].y);
-                    }
                 const float2 vv = ld_pair<kIoF32>(vs_t, lane * C + 2 * pc);
                 const float d0 = __fsub_rn(vv.x, __fmul_rn(gscalar, u[pc].x));
                 const float d1 = __fsub_rn(vv.y, __fmul_rn(gscalar, u[pc].y));
@@ -406,16 +515,10 @@ __global__ void __launch_bounds__(8 * 32, 1) lrb_step_kernel(const LrbStreamPara
 #pragma unroll
             for (int pc = 0; pc < P; ++pc) w[pc] = ld_pair<kIoF32>(vs_t, lane * C + 2 * pc);
         }
-        // append w to V
+        // append w to V (the lane's own columns)
 #pragma unroll
-        for (int l = 0; l < MR; ++l)
-            if (l == m) {
-#pragma unroll
-                for (int pc = 0; pc < P; ++pc) {
-                    Vc[l][2 * pc] = w[pc].x;
-                    Vc[l][2 * pc + 1] = w[pc].y;
-                }
-            }
+        for (int pc = 0; pc < P; ++pc)
+            *reinterpret_cast<float2*>(Vt + m * DV + 2 * pc) = w[pc];
 
         uint8_t* gcodes_tile = p.codes + ti.code_off;
         for (int g = 0; g < G; ++g) {
@@ -438,12 +541,24 @@ __global__ void __launch_bounds__(8 * 32, 1) lrb_step_kernel(const LrbStreamPara
                 const float2 sc = *reinterpret_cast<const float2*>(ss + 2 * pc);
                 const uint32_t j0 = static_cast<uint32_t>(lane * C + 2 * pc);
                 float vc0[MR], vc1[MR];
+                if (merge) {
 #pragma unroll
-                for (int l = 0; l < MR; ++l) {
-                    vc0[l] = pc == 0 ? Vc[l][0] : Vc[l][C - 2];
-                    vc1[l] = pc == 0 ? Vc[l][1] : Vc[l][C - 1];
+                    for (int l = 0; l < MR; ++l) {
+                        const float2 vv = *reinterpret_cast<const float2*>(Vt + l * DV + 2 * pc);
+                        vc0[l] = vv.x;
+                        vc1[l] = vv.y;
+                    }
                 }
-                if (int8g)
+                if constexpr (MODE == kRTN) {
+                    if (int8g)
+                        pair_step_lrb_rtn<GROUP, GATE, 8>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs,
+                                                          gs, gscalar, op, gcodes, gscale + 2 * pc,
+                                                          lane, merge, R, Ug, dk, vc0, vc1);
+                    else
+                        pair_step_lrb_rtn<GROUP, GATE, 4>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs,
+                                                          gs, gscalar, op, gcodes, gscale + 2 * pc,
+                                                          lane, merge, R, Ug, dk, vc0, vc1);
+                } else if (int8g)
                     pair_step_lrb<GROUP, GATE, MODE, 8>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs, gs,
                                                         gscalar, op, gcodes, gscale + 2 * pc, hkey,
                                                         g * GROUP, j0, lane, xs, merge, R, Ug, dk,
@@ -475,10 +590,12 @@ __global__ void __launch_bounds__(8 * 32, 1) lrb_step_kernel(const LrbStreamPara
             ov[2 * pc + 1] = o[pc].y;
         }
 #pragma unroll
-        for (int l = 0; l <= MR; ++l)
+        for (int l = 0; l < MR; ++l) {
+            const float fl = __shfl_sync(0xffffffffu, chain, 16 + l);
             if (l <= m)
 #pragma unroll
-                for (int c = 0; c < C; ++c) ov[c] = __fmaf_rn(f[l], Vc[l < MR ? l : 0][c], ov[c]);
+                for (int c = 0; c < C; ++c) ov[c] = __fmaf_rn(fl, Vt[l * DV + c], ov[c]);
+        }
         float* outp = static_cast<float*>(p.out) + static_cast<int64_t>(tile) * DV + lane * C;
 #pragma unroll
         for (int c = 0; c < C; ++c) outp[c] = ov[c];
@@ -490,11 +607,9 @@ __global__ void __launch_bounds__(8 * 32, 1) lrb_step_kernel(const LrbStreamPara
             *reinterpret_cast<float4*>(Ugl + idx) = t;
         }
         float* Vgl = lp.V + static_cast<int64_t>(tile) * R * DV + lane * C;
+        for (int l = 0; l <= m; ++l)
 #pragma unroll
-        for (int l = 0; l < MR; ++l)
-            if (l <= m)
-#pragma unroll
-                for (int c = 0; c < C; ++c) Vgl[l * DV + c] = merge ? 0.0f : Vc[l][c];
+            for (int c = 0; c < C; ++c) Vgl[l * DV + c] = merge ? 0.0f : Vt[l * DV + c];
         __syncwarp();
     }
     if (!ok) {
