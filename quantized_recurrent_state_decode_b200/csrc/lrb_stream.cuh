@@ -325,16 +325,27 @@ __device__ __forceinline__ void pair_step_lrb_rtn(const uint8_t* __restrict__ cs
     }
 }
 
-// Key-order chain c = sum_i a_i * RN(gm_i * b_i) over n rows (gm = 1 when
-// !decay, exactly b_i then), for one lane's role.
-__device__ __forceinline__ float lrb_chain(const float* a, const float* b, const float* gk,
-                                           float gscalar, bool per_key, bool decay, int n) {
+// One lane's key-order chain c = sum_i a_i * b'_i over n rows (n a multiple
+// of 4), b'_i = RN(g_i * b_i) when `decay`, else b_i: every chain lane runs
+// this one loop, each with its own operands, so the roles do not diverge.
+__device__ __forceinline__ float lrb_chain(const float* a, const float* b, const float* g,
+                                           bool decay, int n) {
     float c = 0.0f;
-#pragma unroll 4
-    for (int i = 0; i < n; ++i) {
-        float bi = b[i];
-        if (decay) bi = __fmul_rn(per_key ? gk[i] : gscalar, bi);
-        c = __fmaf_rn(a[i], bi, c);
+#pragma unroll 2
+    for (int i = 0; i < n; i += 4) {
+        const float4 av = *reinterpret_cast<const float4*>(a + i);
+        float4 bv = *reinterpret_cast<const float4*>(b + i);
+        const float4 gv = *reinterpret_cast<const float4*>(g + i);
+        if (decay) {
+            bv.x = __fmul_rn(gv.x, bv.x);
+            bv.y = __fmul_rn(gv.y, bv.y);
+            bv.z = __fmul_rn(gv.z, bv.z);
+            bv.w = __fmul_rn(gv.w, bv.w);
+        }
+        c = __fmaf_rn(av.x, bv.x, c);
+        c = __fmaf_rn(av.y, bv.y, c);
+        c = __fmaf_rn(av.z, bv.z, c);
+        c = __fmaf_rn(av.w, bv.w, c);
     }
     return c;
 }
@@ -437,24 +448,50 @@ __global__ void __launch_bounds__(lrb_max_warps(MODE) * 32, 1) lrb_step_kernel(c
         float* Ut = reinterpret_cast<float*>(tin + in_u);
         float* Vt = reinterpret_cast<float*>(tin + S::in_vb(dk)) + lane * C;   // this lane's V
 
-        // the component chains: e_l = k . U_l (lanes 0..m-1, delta rule) and
-        // f_l = q . RN(g U_l), f_m = q . k (lanes 16..16+m), all at once
+        // the component chains, all lanes of one loop at once: e_l = k . U_l
+        // (lanes 0..m-1, delta rule; undecayed U) and f_l = q . RN(g U_l) for
+        // l < m, f_m = q . k (lanes 16..16+m). U_m = k is appended first.
+        for (int i = lane; i < dk; i += 32) Ut[m * dk + i] = ks_t[i];
+        __syncwarp();
         float chain = 0.0f;
         {
             const int le = lane, lf = lane - 16;
-            if (UPD == kDelta && le < m)
-                chain = lrb_chain(ks_t, Ut + le * dk, gs_t, gscalar, false, false, dk);
-            else if (lf >= 0 && lf <= m)
-                chain = lf < m ? lrb_chain(qs_t, Ut + lf * dk, gs_t, gscalar, GATE == kGatePerKey,
-                                           true, dk)
-                               : lrb_chain(qs_t, ks_t, gs_t, gscalar, false, false, dk);
+            const bool is_e = UPD == kDelta && le < m;
+            const bool is_f = lf >= 0 && lf <= m;
+            if (is_e || is_f) {
+                const float* a = is_e ? ks_t : qs_t;
+                const float* b = Ut + (is_e ? le : lf) * dk;
+                // scalar decays multiply by the head's gate: a row of it is
+                // not stored, so the per-key array stands in with a select
+                const bool decay = is_f && lf < m;
+                if (GATE == kGatePerKey) {
+                    chain = lrb_chain(a, b, gs_t, decay, dk);
+                } else {
+                    float c = 0.0f;
+#pragma unroll 2
+                    for (int i = 0; i < dk; i += 4) {
+                        const float4 av = *reinterpret_cast<const float4*>(a + i);
+                        float4 bv = *reinterpret_cast<const float4*>(b + i);
+                        if (decay) {
+                            bv.x = __fmul_rn(gscalar, bv.x);
+                            bv.y = __fmul_rn(gscalar, bv.y);
+                            bv.z = __fmul_rn(gscalar, bv.z);
+                            bv.w = __fmul_rn(gscalar, bv.w);
+                        }
+                        c = __fmaf_rn(av.x, bv.x, c);
+                        c = __fmaf_rn(av.y, bv.y, c);
+                        c = __fmaf_rn(av.z, bv.z, c);
+                        c = __fmaf_rn(av.w, bv.w, c);
+                    }
+                    chain = c;
+                }
+            }
         }
         __syncwarp();
-        // decay the buffer in place and append k
+        // decay the buffer in place (k was appended above)
         for (int i = lane; i < dk; i += 32) {
             const float gi = GATE == kGatePerKey ? gs_t[i] : gscalar;
             for (int l = 0; l < m; ++l) Ut[l * dk + i] = __fmul_rn(gi, Ut[l * dk + i]);
-            Ut[m * dk + i] = ks_t[i];
         }
         __syncwarp();
 
