@@ -248,8 +248,14 @@ lrs_status lrs_lrb_step(const lrs_state *st, void *state_codes, float *scales,
 
 /* The same step with HOST inputs and output: copies q, k, v, gates, beta
  * from host memory into device staging buffers owned by the state (allocated
- * on first use), runs lrs_decode_step on the state's own buffers, and copies
- * out back to host memory, all on stream. Pinned host memory makes the copies
+ * on first use), runs lrs_decode_step on the state's own buffers on stream,
+ * and copies out back to host memory on stream. Consecutive calls on a state
+ * alternate between two staging buffers and make their input copies on a
+ * stream of the state's own, so the input copies of one call overlap the
+ * kernel and output copy of the previous one; the kernel waits for its
+ * inputs. The input copies wait only for the previous use of their staging
+ * buffer, not for other work on `stream`: the host input buffers must not be
+ * written by work still pending there. Pinned host memory makes the copies
  * asynchronous; the host buffers must stay valid until the stream reaches the
  * end of the step. */
 lrs_status lrs_decode_step_host(const lrs_state *st, const float *q_host, const float *k_host,

@@ -103,9 +103,15 @@ struct StatePriv {
     int pgroups = 1;    // widths per head (1) or per (head, scale group) (G)
     std::vector<uint8_t> prec_host;
     std::vector<int64_t> offsets_host;
-    // device staging for lrs_decode_step_host (allocated on first use)
-    float* stage = nullptr;
+    // lrs_decode_step_host (set up on first use): two staging buffers used by
+    // alternate calls, a stream for their input copies, and per buffer the
+    // events "inputs copied" and "buffer free again" (after the output copy)
+    float* stage[2] = {nullptr, nullptr};
     size_t stage_floats = 0;
+    cudaStream_t copy_stream = nullptr;
+    cudaEvent_t h2d_done[2] = {nullptr, nullptr};
+    cudaEvent_t free_again[2] = {nullptr, nullptr};
+    uint64_t host_calls = 0;
 };
 
 // ------------------------------------------------------------- layout ---
@@ -371,7 +377,13 @@ lrs_status lrs_state_free(lrs_state* st) {
     cudaFree(st->scales);
     cudaFree(st->prec_map);
     cudaFree(st->head_offsets);
-    cudaFree(pv->stage);
+    cudaFree(pv->stage[0]);
+    cudaFree(pv->stage[1]);
+    for (int b = 0; b < 2; ++b) {
+        if (pv->h2d_done[b]) cudaEventDestroy(pv->h2d_done[b]);
+        if (pv->free_again[b]) cudaEventDestroy(pv->free_again[b]);
+    }
+    if (pv->copy_stream) cudaStreamDestroy(pv->copy_stream);
     if (prev != pv->device && prev >= 0) cudaSetDevice(prev);
     delete pv;
     memset(st, 0, sizeof *st);
@@ -545,36 +557,64 @@ lrs_status lrs_decode_step_host(const lrs_state* st, const float* q_host, const 
     const size_t ng = rnd(sh.gate_kind == LRS_GATE_PER_KEY ? T * sh.d_k : T), nb = rnd(T);
     const size_t need = 2 * nq + 2 * nv + ng + nb;
     StatePriv* pv = static_cast<StatePriv*>(st->priv);
+    cudaError_t e;
+    if (!pv->copy_stream) {
+        if ((e = cudaStreamCreateWithFlags(&pv->copy_stream, cudaStreamNonBlocking)) != cudaSuccess)
+            return cuda_fail(e, "cudaStreamCreate(copies)");
+        for (int b = 0; b < 2; ++b)
+            if ((e = cudaEventCreateWithFlags(&pv->h2d_done[b], cudaEventDisableTiming)) !=
+                    cudaSuccess ||
+                (e = cudaEventCreateWithFlags(&pv->free_again[b], cudaEventDisableTiming)) !=
+                    cudaSuccess)
+                return cuda_fail(e, "cudaEventCreate(staging)");
+    }
     if (pv->stage_floats < need) {
-        cudaFree(pv->stage);
-        pv->stage = nullptr;
+        // no staging buffer may be in use when it is replaced
+        if ((e = cudaStreamSynchronize(pv->copy_stream)) != cudaSuccess ||
+            (e = cudaEventSynchronize(pv->free_again[0])) != cudaSuccess ||
+            (e = cudaEventSynchronize(pv->free_again[1])) != cudaSuccess)
+            return cuda_fail(e, "waiting for the staging buffers");
+        for (int b = 0; b < 2; ++b) {
+            cudaFree(pv->stage[b]);
+            pv->stage[b] = nullptr;
+        }
         pv->stage_floats = 0;
-        cudaError_t e = cudaMalloc(&pv->stage, need * sizeof(float));
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(staging)");
+        for (int b = 0; b < 2; ++b)
+            if ((e = cudaMalloc(&pv->stage[b], need * sizeof(float))) != cudaSuccess)
+                return cuda_fail(e, "cudaMalloc(staging)");
         pv->stage_floats = need;
     }
-    float* dq = pv->stage;
+    // Alternate calls use alternate buffers, so the input copies of one call
+    // overlap the kernel and output copy of the previous one. The copies of a
+    // buffer wait for its previous use to end (its output copy); they are not
+    // ordered after other work on `stream`.
+    const int b = static_cast<int>(pv->host_calls++ & 1);
+    float* dq = pv->stage[b];
     float* dk = dq + nq;
     float* dv = dk + nq;
     float* dout = dv + nv;
     float* dg = dout + nv;
     float* db = dg + ng;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaStream_t cp = pv->copy_stream;
     const cudaMemcpyKind h2d = cudaMemcpyHostToDevice;
-    cudaError_t e;
-    if ((e = cudaMemcpyAsync(dq, q_host, T * sh.d_k * 4, h2d, cs)) != cudaSuccess ||
-        (e = cudaMemcpyAsync(dk, k_host, T * sh.d_k * 4, h2d, cs)) != cudaSuccess ||
-        (e = cudaMemcpyAsync(dv, v_host, T * sh.d_v * 4, h2d, cs)) != cudaSuccess ||
+    if ((e = cudaStreamWaitEvent(cp, pv->free_again[b], 0)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(dq, q_host, T * sh.d_k * 4, h2d, cp)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(dk, k_host, T * sh.d_k * 4, h2d, cp)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(dv, v_host, T * sh.d_v * 4, h2d, cp)) != cudaSuccess ||
         (e = cudaMemcpyAsync(dg, gates_host,
-                             (sh.gate_kind == LRS_GATE_PER_KEY ? T * sh.d_k : T) * 4, h2d, cs)) !=
+                             (sh.gate_kind == LRS_GATE_PER_KEY ? T * sh.d_k : T) * 4, h2d, cp)) !=
             cudaSuccess ||
-        (delta && (e = cudaMemcpyAsync(db, beta_host, T * 4, h2d, cs)) != cudaSuccess))
+        (delta && (e = cudaMemcpyAsync(db, beta_host, T * 4, h2d, cp)) != cudaSuccess) ||
+        (e = cudaEventRecord(pv->h2d_done[b], cp)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(cs, pv->h2d_done[b], 0)) != cudaSuccess)
         return cuda_fail(e, "host-to-device copy of the step inputs");
     s = lrs_decode_step(st, st->state_codes, st->scales, st->prec_map, dq, dk, dv, dg,
                         delta ? db : nullptr, dout, seed, step, mode, stream);
     if (s != LRS_OK) return s;
     if ((e = cudaMemcpyAsync(out_host, dout, T * sh.d_v * 4, cudaMemcpyDeviceToHost, cs)) !=
-        cudaSuccess)
+            cudaSuccess ||
+        (e = cudaEventRecord(pv->free_again[b], cs)) != cudaSuccess)
         return cuda_fail(e, "device-to-host copy of the output");
     return ok();
 }

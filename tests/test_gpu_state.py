@@ -216,6 +216,43 @@ def test_host_buffer_step_matches_device_step():
         lrs.lrs_state_free(b)
 
 
+def test_host_buffer_steps_back_to_back():
+    """Consecutive host-buffer steps with no synchronization between them (the
+    input copies of one step overlap the previous step): every step's output
+    and the final state equal the device-buffer steps'."""
+    w = I.Workload("host_pipe", "gla", 6, 5, 128, 128, 32, 7, I.ROUND_BDR, "mixed", s0_std=0.02,
+                   gate_mu=-3.0, seed_id=81)
+    pm = np.array([8, 4, 8, 4, 8], np.uint8)
+    shp = P.make_shape(w)
+    a = lrs.lrs_state_alloc(shp, pm)
+    b = lrs.lrs_state_alloc(shp, pm)
+    try:
+        S0 = I.initial_state(w, device="cuda")
+        lrs.lrs_state_import_fp32(a, S0)
+        lrs.lrs_state_import_fp32(b, S0)
+        xs = [I.step_inputs(w, t, device="cuda") for t in range(w.steps)]
+        xh = [{n: (None if v is None else v.cpu().pin_memory()) for n, v in x.items()} for x in xs]
+        outs_h = [torch.empty(w.batch, w.heads, w.d_v).pin_memory() for _ in range(w.steps)]
+        torch.cuda.synchronize()
+        for t in range(w.steps):
+            x = xh[t]
+            lrs.lrs_decode_step_host(b, x["q"], x["k"], x["v"], x["gates"], x["beta"], outs_h[t],
+                                     5, t, w.mode)
+        lrs.lrs_sync()
+        out_d = torch.empty(w.batch, w.heads, w.d_v, device="cuda")
+        for t in range(w.steps):
+            x = xs[t]
+            lrs.lrs_decode_step(a, a.state_codes, a.scales, a.prec_map, x["q"], x["k"], x["v"],
+                                x["gates"], x["beta"], out_d, 5, t, w.mode)
+            lrs.lrs_sync()
+            assert torch.equal(out_d.cpu(), outs_h[t]), t
+        np.testing.assert_array_equal(_snapshot(a)[0], _snapshot(b)[0])
+        np.testing.assert_array_equal(_snapshot(a)[1], _snapshot(b)[1])
+    finally:
+        lrs.lrs_state_free(a)
+        lrs.lrs_state_free(b)
+
+
 def test_precision_map_mismatch_is_detected_and_skipped():
     w = I.Workload("mismatch", "gla", 4, 2, 128, 128, 32, 1, I.ROUND_RTN, "mixed", s0_std=0.02,
                    gate_mu=-4.0, seed_id=80)
