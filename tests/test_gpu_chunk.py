@@ -160,3 +160,10 @@ def test_chunk_injected_timeout_reports_and_leaves_state():
         lrs.lrs_sync()
     finally:
         pair.free()
+
+
+@pytest.mark.parametrize("name,T", [("mamba2_mixed_sr_b128h64", 8), ("gla_bdr_int4_b256h32_128", 8),
+                                    ("gdn_sr_int8_b64h16_128", 8)])
+def test_chunk_full_size_workloads_sampled(name, T):
+    """The full-size workloads (every tile updated, a spread sample compared)."""
+    run_chunks(I.WORKLOADS[name], T=T, n_chunks=2, tiles="sample")

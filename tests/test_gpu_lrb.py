@@ -111,3 +111,11 @@ def test_lrb_rejects_bad_rank_and_group_widths():
         assert ei.value.status == lrs.LRS_ERR_UNSUPPORTED
     finally:
         lrs.lrs_state_free(st)
+
+
+@pytest.mark.parametrize("name", ["gla_rtn_int8_b256h32_128", "mamba2_mixed_sr_b128h64",
+                                  "gla_bdr_int4_b256h32_128"])
+def test_lrb_full_size_workloads_sampled(name):
+    """The full-size workloads through two merges (every tile updated, a spread
+    sample compared, buffers included)."""
+    run_lrb(I.WORKLOADS[name], rank=4, steps=8, tiles="sample")

@@ -87,3 +87,10 @@ def test_uniform_group_map_has_the_head_layout():
 def test_chunk_with_group_widths(fam):
     w = _small(fam, 3, 5, 128, 128, 32, I.ROUND_BDR, "mixed", steps=2)
     run_chunks(w, T=5, n_chunks=2, pm=_random_map(w, 21))
+
+
+def test_decay_ranked_group_map_gdn_mixed_sampled():
+    w = I.WORKLOADS["gdn_mixed_sr_h32_128"].with_batch(256)
+    pm = P.group_prec_map_for(w, steps=8)
+    assert 0 < (pm == 8).sum() < pm.size
+    P.run_parity(w, 6, tiles="sample", pm=pm)
