@@ -367,6 +367,8 @@ def run_gpu(args, w):
 
     for st in states:
         lrs.lrs_state_free(st)
+    if not args.no_extras and rank == 0 and args.drift_steps > 0:
+        extras["drift"] = run_drift(dev, stream, args.drift_steps)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -599,6 +601,77 @@ def run_lrb_extra(w, wl, states, xs, out, seed, stream, L, NI, mode, dev, pm, ra
                          "frac": achieved / peak, "algorithmic_bytes_per_launch": nbytes}}
 
 
+DRIFT_WORKLOAD = "gla_bdr_int4_b256h32_128"
+
+
+def run_drift(dev, stream, steps=1024, batch=None):
+    """Output drift of the int4 GLA workload against the fp32-state kernel on
+    the same inputs: e_t = ||o_q - o_fp32||_2 / ||o_fp32||_2 over every
+    (b, h, j) of step t, at t = 1, 2, 4, ..., for round to nearest, bounded
+    directional rounding, stochastic rounding and the rank-4 Low-Rank Bypass
+    with RTN and with BDR. Every variant starts from the same state and reads
+    the same inputs; the norms are taken after the step, outside any timing."""
+    import torch
+    from quantized_recurrent_state_decode_b200 import inputs as I
+    from quantized_recurrent_state_decode_b200 import lrs
+    w = I.WORKLOADS[DRIFT_WORKLOAD]
+    if batch:
+        w = w.with_batch(batch)
+    pm = I.uniform_prec_map(w).numpy()
+    shp = lrs.shape(w.batch, w.heads, w.d_k, w.d_v, w.group, w.update_kind, w.gate_kind)
+    seed = I.sr_seed(w)
+    rank = 4
+    variants = [("rtn", I.ROUND_RTN, 0), ("bdr", I.ROUND_BDR, 0), ("sr", I.ROUND_SR, 0),
+                ("lrb4_rtn", I.ROUND_RTN, rank), ("lrb4_bdr", I.ROUND_BDR, rank)]
+    S0 = I.initial_state(w, device=dev)
+    S = S0.clone()
+    states, bufs, outs = {}, {}, {}
+    try:
+        for name, _, r in variants:
+            st = lrs.lrs_state_alloc(shp, pm)
+            states[name] = st
+            lrs.lrs_state_import_fp32(st, S0)
+            if r:
+                bufs[name] = (torch.zeros(w.batch, w.heads, r, w.d_k, device=dev),
+                              torch.zeros(w.batch, w.heads, r, w.d_v, device=dev))
+            outs[name] = torch.empty(w.batch, w.heads, w.d_v, device=dev)
+        del S0
+        of = torch.empty(w.batch, w.heads, w.d_v, device=dev)
+        samples = [1 << i for i in range(steps.bit_length()) if (1 << i) <= steps]
+        series = {name: [] for name, _, _ in variants}
+        with torch.cuda.stream(stream):
+            for t in range(steps):
+                x = I.step_inputs(w, t, device=dev)
+                lrs.lrs_fp32_decode_step(shp, S, x["q"], x["k"], x["v"], x["gates"], x["beta"],
+                                         of, stream)
+                for name, mode, r in variants:
+                    st = states[name]
+                    if r:
+                        U, V = bufs[name]
+                        lrs.lrs_lrb_step(st, st.state_codes, st.scales, st.prec_map, r, U, V,
+                                         x["q"], x["k"], x["v"], x["gates"], x["beta"],
+                                         outs[name], seed, t, mode, stream)
+                    else:
+                        lrs.lrs_decode_step(st, st.state_codes, st.scales, st.prec_map, x["q"],
+                                            x["k"], x["v"], x["gates"], x["beta"], outs[name],
+                                            seed, t, mode, stream)
+                if t + 1 in samples:
+                    ref = torch.linalg.vector_norm(of)
+                    for name, _, _ in variants:
+                        series[name].append(
+                            (torch.linalg.vector_norm(outs[name] - of) / ref).item())
+        lrs.lrs_sync(stream)
+    finally:
+        for st in states.values():
+            lrs.lrs_state_free(st)
+    res = {"workload": w.name, "batch": w.batch, "state": "int4", "group": w.group,
+           "lrb_rank": rank,
+           "measure": "||o_q - o_fp32||_2 / ||o_fp32||_2 over all (b, h, j) of step t",
+           "reference": "lrs_fp32_decode_step on the same inputs", "t": samples}
+    res.update(series)
+    return res
+
+
 def _sm_max_mhz():
     try:
         out = subprocess.run(["nvidia-smi", "--query-gpu=clocks.max.sm", "--format=csv,noheader,"
@@ -656,6 +729,8 @@ def main():
     ap.add_argument("--layers", type=int, default=4)
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch")
     ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--drift-steps", type=int, default=1024,
+                    help="steps of the int4 output-drift series (0: skip it)")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -778,7 +778,9 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
     const int wib = threadIdx.x >> 5;
     const int nw = blockDim.x >> 5;
     const int W = gridDim.x * nw;
-    const int gw = blockIdx.x * nw + wib;
+    // warp-major numbering: the tiles of the last round (ntiles mod W of
+    // them) spread over every SM instead of filling the first CTAs
+    const int gw = wib * gridDim.x + blockIdx.x;
     uint8_t* wsm = smem + wib * p.warp_smem;
     uint64_t* bars = reinterpret_cast<uint64_t*>(wsm);
     const int G = p.G, NS = p.slots;
