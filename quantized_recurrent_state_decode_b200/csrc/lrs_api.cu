@@ -227,7 +227,7 @@ const void* find_step_kernel(int C, int group, int update_kind, int gate_kind, i
 
 int step_warp_smem(int C, int group, int update_kind, int gate_kind, int slots, int mode, int io,
                    int d_k) {
-    const bool xs = stage_x(mode);
+    const bool xs = stage_x(mode, update_kind);
 #define LRS_SLOT_IO(CC, GG, IO)                                                                   \
     if (update_kind == kDelta) return Slot<CC, GG, kGate, IO, true>::warp_bytes(slots, xs, d_k);   \
     return gate_kind == kGatePerKey ? Slot<CC, GG, kGatePerKey, IO>::warp_bytes(slots, xs, d_k)   \
@@ -436,7 +436,7 @@ static lrs_status decode_step_io(const lrs_state* st, void* state_codes, float* 
     int warps = step_warps_override();
     if (warps <= 0) warps = kDefaultWarps;
     warps = std::min(warps, std::max(1, kSmemLimit / warp_smem));
-    warps = std::min(warps, lrs::step_max_warps(sh.group, mode));
+    warps = std::min(warps, lrs::step_max_warps(sh.group, mode, sh.update_kind));
     const int smem = warps * warp_smem;
 
     // Per kernel and device, raise the dynamic shared memory limit once to the

@@ -124,7 +124,7 @@ extern "C" lrs_status lrs_decode_step_host_noalloc(const lrs_state* st, const fl
                                               lrs::kStepIoF32, sh.d_k);
     constexpr int kSmemLimit = 227 * 1024;
     int warps = std::min(12, std::max(1, kSmemLimit / warp_smem));
-    warps = std::min(warps, lrs::step_max_warps(sh.group, mode));
+    warps = std::min(warps, lrs::step_max_warps(sh.group, mode, sh.update_kind));
     const int smem = warps * warp_smem;
     int dev = 0, sms = 0, per_sm = 0;
     cudaGetDevice(&dev);

@@ -29,10 +29,22 @@ constexpr int kGated = 0, kDelta = 1;            // matches lrs_update_kind
 constexpr int kRTN = 0, kSR = 1, kBDR = 2;       // matches lrs_round_mode
 constexpr int kIoF32 = 0, kIoBF16 = 1;           // element type of q, k, v and out
 constexpr int kMaxSlots = 16;
+// Variants that stage the group's updated values in shared memory for the
+// rounding pass: SR, and BDR of the delta rule. Gated BDR recomputes them
+// from the codes still in the slot instead (two two-wide operations per row
+// pair), which saves the 8 KB buffer so that 12 warps fit beside the ring:
+// measured 9% faster than staging at 8 warps. For SR the same change measured
+// within 2% either way (its longer rounding keeps the issue slots busier), so
+// SR keeps the buffer and its fewer instructions.
+__host__ __device__ constexpr bool stage_x(int mode, int upd) {
+    return mode == kSR || (mode == kBDR && upd == kDelta);
+}
 // Launch bound of a step variant in warps: 12 (at most 168 registers a thread)
 // where the live state fits, 8 (255 registers) for the wider groups and for
-// the rounding modes that carry more temporaries.
-__host__ __device__ constexpr int step_max_warps(int group, int mode) { return (mode != 0 || group > 32) ? 8 : 12; }
+// the staging variants, whose buffer leaves shared memory for 8 warps.
+__host__ __device__ constexpr int step_max_warps(int group, int mode, int upd) {
+    return (stage_x(mode, upd) || group > 32) ? 8 : 12;
+}
 constexpr float kTiny = 0x1p-100f;               // absmax below this: stored as zero
 
 struct StepParams {
@@ -107,8 +119,6 @@ struct Slot {
     }
 };
 
-// Modes that stage the group's updated values in shared memory.
-__host__ __device__ constexpr bool stage_x(int mode) { return mode != 0; }
 
 // ------------------------------------------------------- packed fp32 math ---
 // Two consecutive key rows of one column go through the sm_100 two-wide fp32
@@ -147,6 +157,29 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
         "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
         : "=f"(r.x), "=f"(r.y)
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return r;
+}
+
+// fma with rounding toward minus infinity, two-wide.
+__device__ __forceinline__ float2 fma2_rm(float2 a, float2 b, float2 c) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rm.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return r;
+}
+
+// Three-input minimum and maximum.
+__device__ __forceinline__ float min3(float a, float b, float c) {
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
 }
 
@@ -261,10 +294,10 @@ __device__ __forceinline__ void new_scales(float A0, float A1, float2& snew, flo
     inv = make_float2(A0 < kTiny ? 0.0f : iv.x, A1 < kTiny ? 0.0f : iv.y);
 }
 
-// Codes of two elements (key rows i, i+1 of value column j), returned as the
-// floats kb + code (kb: word_bias of the two elements' word positions) whose
-// low bits are the stored byte (nibble). inv, s_new: the column's values in
-// both halves. The value rounded is the exact product x*inv: one fused
+// Codes of two elements (key rows i, i+1 of value column j; i even), returned
+// as the floats kb + code (kb: word_bias of the two elements' word positions)
+// whose low bits are the stored byte (nibble). inv, s_new: the column's values
+// in both halves. The value rounded is the exact product x*inv: one fused
 // multiply-add rounds it straight to an integer.
 template <int MODE, int BITS>
 __device__ __forceinline__ float2 round_rows(float2 x, float2 inv, float2 deq, float2 s_new,
@@ -275,33 +308,41 @@ __device__ __forceinline__ float2 round_rows(float2 x, float2 inv, float2 deq, f
         // the nearest integer never leaves [-qmax, qmax], no clamp needed.
         return fma2(x, inv, kb);
     } else {
-        const float2 n = add2(fma2(x, inv, f2(kRound)), f2(-kRound));  // nearest integer
-        const float2 d = fma2(x, inv, neg2(n));                          // sign of x*inv - n
         float2 c;
         if constexpr (MODE == kSR) {
-            const float2 f = make_float2(d.x < 0.0f ? n.x - 1.0f : n.x,
-                                         d.y < 0.0f ? n.y - 1.0f : n.y);  // floor
+            // floor(x*inv): the exact product plus 1.5*2^23, rounded toward
+            // minus infinity, lands on the integer below it (|x*inv| < 2^22)
+            const float2 f = add2(fma2_rm(x, inv, f2(kRound)), f2(-kRound));
             const float2 fr = fma2(x, inv, neg2(f));                      // fraction, rounded once
-            const float u0 = element_uniform(hkey, i, j);
-            const float u1 = element_uniform(hkey, i + 1, j);
-            c.x = u0 < fr.x ? f.x + 1.0f : f.x;
-            c.y = u1 < fr.y ? f.y + 1.0f : f.y;
+            const float2 f1 = add2(f, f2(1.0f));
+            const HashColumn hc = hash_column(hkey, j);
+            const uint32_t khi = static_cast<uint32_t>(hkey >> 32) ^ i;
+            const float u0 = hash_uniform(khi, hc);
+            const float u1 = hash_uniform(khi ^ 1u, hc);                 // row i + 1 (i even)
+            c.x = u0 < fr.x ? f1.x : f.x;
+            c.y = u1 < fr.y ? f1.y : f.y;
         } else {
-            // the update and the move; the move's product and difference are
-            // two separate roundings (scalar _rn operations are never fused)
-            const float2 delta = add2(x, neg2(deq));
-            const float2 m = make_float2(__fsub_rn(__fmul_rn(n.x, s_new.x), deq.x),
-                                         __fsub_rn(__fmul_rn(n.y, s_new.y), deq.y));
-            // A reversal (update and move of opposite signs) takes ceil(x*inv)
-            // when the update is positive and floor(x*inv) when it is
-            // negative; ceil = n + 1 exactly when x*inv > n, floor = n - 1
-            // exactly when x*inv < n. Written with selects, no branches.
-            const bool up0 = (delta.x > 0.0f) & (m.x < 0.0f) & (d.x > 0.0f);
-            const bool dn0 = (delta.x < 0.0f) & (m.x > 0.0f) & (d.x < 0.0f);
-            const bool up1 = (delta.y > 0.0f) & (m.y < 0.0f) & (d.y > 0.0f);
-            const bool dn1 = (delta.y < 0.0f) & (m.y > 0.0f) & (d.y < 0.0f);
-            c.x = n.x + (up0 ? 1.0f : 0.0f) - (dn0 ? 1.0f : 0.0f);
-            c.y = n.y + (up1 ? 1.0f : 0.0f) - (dn1 ? 1.0f : 0.0f);
+            const float2 n = add2(fma2(x, inv, f2(kRound)), f2(-kRound));  // nearest integer
+            const float2 d = fma2(x, inv, neg2(n));                          // sign of x*inv - n
+            // The update a = RN(x - deq) and the move b = RN(p - deq),
+            // p = RN(n s'), enter only through their signs. A reversal (a
+            // and b of opposite signs) takes ceil(x*inv) when the update is
+            // positive and floor(x*inv) when it is negative; ceil = n + 1
+            // exactly when d > 0, floor = n - 1 exactly when d < 0. So the
+            // code moves up when a > 0, b < 0 and d > 0, i.e. when
+            // min(a, -b, d) > 0, and down when max(a, -b, d) < 0: one
+            // three-input minimum or maximum and one compare each, no
+            // branches. (The subtractions are exact in sign: a rounded
+            // difference of two floats is zero only when they are equal.)
+            const float2 p = mul2(n, s_new);
+            const float2 a = add2(x, neg2(deq));
+            const float2 nb = add2(deq, neg2(p));                         // -b
+            const bool up0 = min3(a.x, nb.x, d.x) > 0.0f;
+            const bool dn0 = max3(a.x, nb.x, d.x) < 0.0f;
+            const bool up1 = min3(a.y, nb.y, d.y) > 0.0f;
+            const bool dn1 = max3(a.y, nb.y, d.y) < 0.0f;
+            c.x = up0 ? n.x + 1.0f : (dn0 ? n.x - 1.0f : n.x);
+            c.y = up1 ? n.y + 1.0f : (dn1 ? n.y - 1.0f : n.y);
         }
         c.x = fminf(fmaxf(c.x, -QMAX), QMAX);
         c.y = fminf(fmaxf(c.y, -QMAX), QMAX);
@@ -603,12 +644,15 @@ struct TileCursor : TileLayout {
     }
 };
 
-// The same step for modes whose per-element rounding is long (SR, BDR): the
-// group's updated values are staged in the warp's shared-memory x buffer
-// instead of registers, so both phases are short loops over 16-byte units and
-// the kernel's code stays small enough for the instruction cache. xs holds
-// (x[r][c0], x[r+1][c0], x[r][c1], x[r+1][c1]) per row pair r and lane.
-template <int GROUP, int GATE, int MODE, int BITS, int IO>
+// The same step for modes whose per-element rounding is long (SR, BDR): two
+// short loops over 16-byte units, so the kernel's code stays small enough for
+// the instruction cache. The first computes x, the output and the absmax; the
+// second rounds. Between them, the group's updated values are either staged
+// in the warp's shared-memory x buffer (STAGE; xs holds (x[r][c0],
+// x[r+1][c0], x[r][c1], x[r+1][c1]) per row pair r and lane) or recomputed
+// from the codes, scales, k, gates and w, by the same operations in the same
+// order, so bit for bit the same values.
+template <int GROUP, int GATE, int MODE, int BITS, int IO, bool STAGE>
 __device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int ubase, float2 sc,
                                              const uint8_t* __restrict__ qs,
                                              const uint8_t* __restrict__ ks,
@@ -652,7 +696,8 @@ __device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int
                 o.y = __fmaf_rn(qr.y, x1.y, o.y);
                 a0 = max_abs3(a0, x0.x, x0.y);
                 b0 = max_abs3(b0, x1.x, x1.y);
-                xs[(un * RPUH + rl / 2) * 32 + lane] = make_float4(x0.x, x0.y, x1.x, x1.y);
+                if constexpr (STAGE)
+                    xs[(un * RPUH + rl / 2) * 32 + lane] = make_float4(x0.x, x0.y, x1.x, x1.y);
             }
         }
     }
@@ -663,27 +708,43 @@ __device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int
     const float2 inv0 = f2(inv.x), inv1 = f2(inv.y);
     const float2 sn0 = f2(snew.x), sn1 = f2(snew.y);
 
+    constexpr bool DECODE = MODE == kBDR || !STAGE;   // phase 2 reads the old codes
 #pragma unroll 1
     for (int un = 0; un < G::UNITS; ++un) {
         uint32_t ow[4];
         uint32_t wd[4] = {0u, 0u, 0u, 0u};
-        if constexpr (MODE == kBDR) {
+        if constexpr (DECODE) {
             const uint4 raw = lds_unit(cs, ubase + un, lane);
             wd[0] = raw.x; wd[1] = raw.y; wd[2] = raw.z; wd[3] = raw.w;
+        }
+        float kk[STAGE ? 1 : G::RPU], gg[STAGE || GATE != kGatePerKey ? 1 : G::RPU];
+        if constexpr (!STAGE) {
+            ld_rows<IO, G::RPU>(ks, un * G::RPU, kk);
+            if constexpr (GATE == kGatePerKey) ld_smem_rows<G::RPU>(gs + un * G::RPU, gg);
         }
 #pragma unroll
         for (int wi = 0; wi < 4; ++wi) {
             float f[G::EPW];
-            if constexpr (MODE == kBDR) decode_word_biased<BITS>(wd[wi], f);
+            if constexpr (DECODE) decode_word_biased<BITS>(wd[wi], f);
             float t[G::EPW];
 #pragma unroll
             for (int rp = 0; rp < G::RPW / 2; ++rp) {
                 const int rl = wi * G::RPW + 2 * rp;
-                const float4 xv = xs[(un * RPUH + rl / 2) * 32 + lane];
                 float2 dq0 = f2(0.0f), dq1 = f2(0.0f);
-                if constexpr (MODE == kBDR) {
+                if constexpr (DECODE) {
                     dq0 = mul2(add2(make_float2(f[4 * rp], f[4 * rp + 2]), f2(-(kTwo23 + BIAS))), s0);
                     dq1 = mul2(add2(make_float2(f[4 * rp + 1], f[4 * rp + 3]), f2(-(kTwo23 + BIAS))), s1);
+                }
+                float4 xv;
+                if constexpr (STAGE) {
+                    xv = xs[(un * RPUH + rl / 2) * 32 + lane];
+                } else {
+                    // the first loop's x, recomputed by the same operations
+                    const float2 kr = make_float2(kk[rl], kk[rl + 1]);
+                    const float2 gr = GATE == kGatePerKey ? make_float2(gg[rl], gg[rl + 1]) : gsc;
+                    const float2 x0 = fma2(gr, dq0, mul2(kr, w0));
+                    const float2 x1 = fma2(gr, dq1, mul2(kr, w1));
+                    xv = make_float4(x0.x, x0.y, x1.x, x1.y);
                 }
                 const uint32_t i = static_cast<uint32_t>(row0 + un * G::RPU + rl);
                 const float2 kb0 = make_float2(word_bias<BITS>(4 * rp), word_bias<BITS>(4 * rp + 2));
@@ -767,7 +828,7 @@ struct Ring {
 // The warp's items are (tile, group) pairs in order: item k is group k % G of
 // the warp's tile k / G (tiles gw, gw + W, ...).
 template <int C, int GROUP, int UPD, int GATE, int MODE, int IO>
-__global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
+__global__ void __launch_bounds__(step_max_warps(GROUP, MODE, UPD) * 32, 1)
     step_kernel(const StepParams p) {
     constexpr bool INS = UPD == kDelta;
     using S = Slot<C, GROUP, GATE, IO, INS>;
@@ -972,17 +1033,18 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE) * 32, 1)
             for (int pc = 0; pc < P; ++pc) {
                 const float2 sc = *reinterpret_cast<const float2*>(ss + 2 * pc);
                 const uint32_t j0 = static_cast<uint32_t>(lane * C + 2 * pc);
-                if constexpr (stage_x(MODE)) {
+                if constexpr (MODE != kRTN) {
+                    constexpr bool ST = stage_x(MODE, UPD);
                     if (int8g)
-                        pair_step_xs<GROUP, GATE, MODE, 8, IOR>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs,
-                                                           ks, gs, gscalar, wp, op, gcodes,
-                                                           gscale + 2 * pc, hkey, g * GROUP, j0,
-                                                           lane, xs);
+                        pair_step_xs<GROUP, GATE, MODE, 8, IOR, ST>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc,
+                                                               qs, ks, gs, gscalar, wp, op, gcodes,
+                                                               gscale + 2 * pc, hkey, g * GROUP, j0,
+                                                               lane, xs);
                     else
-                        pair_step_xs<GROUP, GATE, MODE, 4, IOR>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs,
-                                                           ks, gs, gscalar, wp, op, gcodes,
-                                                           gscale + 2 * pc, hkey, g * GROUP, j0,
-                                                           lane, xs);
+                        pair_step_xs<GROUP, GATE, MODE, 4, IOR, ST>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc,
+                                                               qs, ks, gs, gscalar, wp, op, gcodes,
+                                                               gscale + 2 * pc, hkey, g * GROUP, j0,
+                                                               lane, xs);
                 } else {
                     if (int8g)
                         pair_step<GROUP, GATE, MODE, 8, IOR>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs, ks,
