@@ -61,11 +61,12 @@ lrs_status lrb_ctas_per_sm(const lrs::ChunkKernel& k, int threads, int* per_sm) 
     return LRS_OK;
 }
 
-const void* find_lrb_stream(int C, int group, int update_kind, int gate_kind, int mode) {
+const void* find_lrb_stream(int C, int group, int update_kind, int gate_kind, int mode,
+                            bool merge) {
     switch (mode) {
-        case LRS_ROUND_RTN: return lrs::find_lrb_stream_rtn(C, group, update_kind, gate_kind);
-        case LRS_ROUND_SR: return lrs::find_lrb_stream_sr(C, group, update_kind, gate_kind);
-        case LRS_ROUND_BDR: return lrs::find_lrb_stream_bdr(C, group, update_kind, gate_kind);
+        case LRS_ROUND_RTN: return lrs::find_lrb_stream_rtn(C, group, update_kind, gate_kind, merge);
+        case LRS_ROUND_SR: return lrs::find_lrb_stream_sr(C, group, update_kind, gate_kind, merge);
+        case LRS_ROUND_BDR: return lrs::find_lrb_stream_bdr(C, group, update_kind, gate_kind, merge);
         default: return nullptr;
     }
 }
@@ -95,14 +96,17 @@ lrs_status launch_lrb_stream(const lrs_state* st, void* state_codes, float* scal
                              int32_t mode, unsigned* err, int sms, void* stream) {
     const lrs_shape& sh = st->shape;
     const int C = sh.d_v / 32, G = sh.d_k / sh.group;
-    const void* fn = find_lrb_stream(C, sh.group, sh.update_kind, sh.gate_kind, mode);
-    if (!fn || rank > lrs::kLrbStreamMaxRank) return LRS_ERR_UNSUPPORTED;
+    if (rank > lrs::kLrbStreamMaxRank) return LRS_ERR_UNSUPPORTED;
+    const int m = static_cast<int>(step % static_cast<uint64_t>(rank));   // components filled
+    const bool merge = m + 1 == rank;
+    const void* fn = find_lrb_stream(C, sh.group, sh.update_kind, sh.gate_kind, mode, merge);
+    if (!fn) return LRS_ERR_UNSUPPORTED;
     int slots = sh.update_kind == LRS_UPDATE_DELTA ? G : std::min(2, G);
     slots = std::max(1, std::min(slots, lrs::kMaxSlots));
     const int warp_smem =
         lrb_stream_warp_smem(C, sh.group, sh.gate_kind, slots, sh.d_k, mode != LRS_ROUND_RTN);
     constexpr int kSmemLimit = 227 * 1024;
-    const int warps = std::min(lrs::lrb_max_warps(mode), kSmemLimit / warp_smem);
+    const int warps = std::min(lrs::lrb_max_warps(mode, merge, sh.group), kSmemLimit / warp_smem);
     if (warps < 1) return LRS_ERR_UNSUPPORTED;
     const int smem = warps * warp_smem;
     static std::mutex mu;
@@ -158,7 +162,7 @@ lrs_status launch_lrb_stream(const lrs_state* st, void* state_codes, float* scal
     lp.U = U;
     lp.V = V;
     lp.rank = rank;
-    lp.m = static_cast<int32_t>(step % static_cast<uint64_t>(rank));
+    lp.m = m;
     void* args[] = {&lp};
     e = cudaLaunchKernel(fn, dim3(grid), dim3(warps * 32), args, smem,
                          static_cast<cudaStream_t>(stream));

@@ -148,7 +148,10 @@ __device__ __forceinline__ void pair_step_lrb(const uint8_t* __restrict__ cs, in
                 o.y = __fmaf_rn(qr.x, x1.x, o.y);
                 o.y = __fmaf_rn(qr.y, x1.y, o.y);
                 if (merge) {
-                    // M = sum_l U'_l,i V'_l,j (fma chain in component order)
+                    // M = sum_l U'_l,i V'_l,j (fma chain in component order),
+                    // added where |M| >= RN(s_old / 2). The rule's M != 0 is
+                    // not tested: adding a zero M changes at most the sign of
+                    // a zero x, which no code, scale or later output sees.
                     const int r = un * G::RPU + rl;
                     float2 m0 = f2(0.0f), m1 = f2(0.0f);
 #pragma unroll
@@ -160,10 +163,10 @@ __device__ __forceinline__ void pair_step_lrb(const uint8_t* __restrict__ cs, in
                         }
                     }
                     const float2 y0 = add2(x0, m0), y1 = add2(x1, m1);
-                    x0.x = (m0.x != 0.0f && fabsf(m0.x) >= half0) ? y0.x : x0.x;
-                    x0.y = (m0.y != 0.0f && fabsf(m0.y) >= half0) ? y0.y : x0.y;
-                    x1.x = (m1.x != 0.0f && fabsf(m1.x) >= half1) ? y1.x : x1.x;
-                    x1.y = (m1.y != 0.0f && fabsf(m1.y) >= half1) ? y1.y : x1.y;
+                    x0.x = fabsf(m0.x) >= half0 ? y0.x : x0.x;
+                    x0.y = fabsf(m0.y) >= half0 ? y0.y : x0.y;
+                    x1.x = fabsf(m1.x) >= half1 ? y1.x : x1.x;
+                    x1.y = fabsf(m1.y) >= half1 ? y1.y : x1.y;
                 }
                 a0 = max_abs3(a0, x0.x, x0.y);
                 b0 = max_abs3(b0, x1.x, x1.y);
@@ -283,10 +286,10 @@ __device__ __forceinline__ void pair_step_lrb_rtn(const uint8_t* __restrict__ cs
             }
             const float2 x0 = x[rp][0], x1 = x[rp][1];
             const float2 y0 = add2(x0, m0), y1 = add2(x1, m1);
-            x[rp][0].x = (m0.x != 0.0f && fabsf(m0.x) >= half0) ? y0.x : x0.x;
-            x[rp][0].y = (m0.y != 0.0f && fabsf(m0.y) >= half0) ? y0.y : x0.y;
-            x[rp][1].x = (m1.x != 0.0f && fabsf(m1.x) >= half1) ? y1.x : x1.x;
-            x[rp][1].y = (m1.y != 0.0f && fabsf(m1.y) >= half1) ? y1.y : x1.y;
+            x[rp][0].x = fabsf(m0.x) >= half0 ? y0.x : x0.x;
+            x[rp][0].y = fabsf(m0.y) >= half0 ? y0.y : x0.y;
+            x[rp][1].x = fabsf(m1.x) >= half1 ? y1.x : x1.x;
+            x[rp][1].y = fabsf(m1.y) >= half1 ? y1.y : x1.y;
         }
     }
     float a0 = 0.0f, a1 = 0.0f, b0 = 0.0f, b1 = 0.0f;
@@ -351,12 +354,18 @@ __device__ __forceinline__ float lrb_chain(const float* a, const float* b, const
 }
 
 // The warp's items are (tile, group) pairs as in step_kernel.
-// Launch bound in warps: 8, so up to 255 registers (the bypass's extra
-// per-tile values do not fit beside a register-resident group in 168).
-__host__ __device__ constexpr int lrb_max_warps(int) { return 8; }
+// Launch bound in warps. A merge step (MERGE: step mod rank = rank - 1) and
+// the staged rounding modes take 8, so up to 255 registers: the merge's
+// buffer rows do not fit beside a register-resident group in 168. The other
+// RTN steps with groups of up to 32 rows are compiled without the merge code
+// and take up to 12 (shared memory leaves 10 for d_k = d_v = 128).
+__host__ __device__ constexpr int lrb_max_warps(int mode, bool merge, int group) {
+    return (mode == kRTN && !merge && group <= 32) ? 12 : 8;
+}
 
-template <int C, int GROUP, int UPD, int GATE, int MODE>
-__global__ void __launch_bounds__(lrb_max_warps(MODE) * 32, 1) lrb_step_kernel(const LrbStreamParams lp) {
+template <int C, int GROUP, int UPD, int GATE, int MODE, bool MERGE>
+__global__ void __launch_bounds__(lrb_max_warps(MODE, MERGE, GROUP) * 32, 1)
+    lrb_step_kernel(const LrbStreamParams lp) {
     using S = LrbSlot<C, GROUP, GATE>;
     constexpr int DV = 32 * C;
     constexpr int P = C / 2;
@@ -379,7 +388,7 @@ __global__ void __launch_bounds__(lrb_max_warps(MODE) * 32, 1) lrb_step_kernel(c
     const int ntw = gw < p.ntiles ? (p.ntiles - gw + W - 1) / W : 0;
     const int64_t K = static_cast<int64_t>(ntw) * G;
     const int R = lp.rank, m = lp.m;
-    const bool merge = m + 1 == R;
+    constexpr bool merge = MERGE;   // the host launches this variant when m + 1 == R
 
     if (lane == 0) {
         for (int s = 0; s < NS; ++s) mbar_init(&bars[s], 1);
@@ -661,22 +670,27 @@ __global__ void __launch_bounds__(lrb_max_warps(MODE) * 32, 1) lrb_step_kernel(c
     }
 }
 
-// Defines `ChunkKernel NAME(C, group, update_kind, gate_kind)`: the streaming
-// bypass kernel with rounding MODE; smem is the per-warp bytes for d_k = 128
-// (the host recomputes it for the actual d_k).
+// Defines `const void* NAME(C, group, update_kind, gate_kind, merge)`: the
+// streaming bypass kernel with rounding MODE for a merge step or another step,
+// or nullptr when that shape is not compiled.
+#define LRS_LRB_STREAM_PICK2(MODE, CC, GG, MG)                                                 \
+    if (update_kind == kGated && gate_kind == kGatePerKey)                                     \
+        return reinterpret_cast<const void*>(                                                  \
+            &lrb_step_kernel<CC, GG, kGated, kGatePerKey, MODE, MG>);                          \
+    if (update_kind == kGated && gate_kind == kGate)                                           \
+        return reinterpret_cast<const void*>(&lrb_step_kernel<CC, GG, kGated, kGate, MODE, MG>); \
+    if (update_kind == kDelta && gate_kind == kGate)                                           \
+        return reinterpret_cast<const void*>(&lrb_step_kernel<CC, GG, kDelta, kGate, MODE, MG>); \
+    return nullptr;
 #define LRS_LRB_STREAM_PICK1(MODE, CC, GG)                                                     \
     if (C == CC && group == GG) {                                                              \
-        if (update_kind == kGated && gate_kind == kGatePerKey)                                 \
-            return reinterpret_cast<const void*>(                                              \
-                &lrb_step_kernel<CC, GG, kGated, kGatePerKey, MODE>);                          \
-        if (update_kind == kGated && gate_kind == kGate)                                       \
-            return reinterpret_cast<const void*>(&lrb_step_kernel<CC, GG, kGated, kGate, MODE>); \
-        if (update_kind == kDelta && gate_kind == kGate)                                       \
-            return reinterpret_cast<const void*>(&lrb_step_kernel<CC, GG, kDelta, kGate, MODE>); \
-        return nullptr;                                                                        \
+        if (merge) {                                                                           \
+            LRS_LRB_STREAM_PICK2(MODE, CC, GG, true)                                           \
+        }                                                                                      \
+        LRS_LRB_STREAM_PICK2(MODE, CC, GG, false)                                              \
     }
 #define LRS_LRB_STREAM_VARIANTS(NAME, MODE)                                                    \
-    const void* NAME(int C, int group, int update_kind, int gate_kind) {                       \
+    const void* NAME(int C, int group, int update_kind, int gate_kind, bool merge) {           \
         LRS_LRB_STREAM_PICK1(MODE, 4, 16)                                                      \
         LRS_LRB_STREAM_PICK1(MODE, 4, 32)                                                      \
         LRS_LRB_STREAM_PICK1(MODE, 2, 16)                                                      \

@@ -44,9 +44,12 @@ ChunkKernel find_lrb_kernel_bdr(int d_k, int d_v, int group, int update_kind, in
 
 // The streaming bypass kernels (ranks up to 4), by (C = d_v/32, group,
 // update kind, gate kind); nullptr when not compiled.
-const void* find_lrb_stream_rtn(int C, int group, int update_kind, int gate_kind);
-const void* find_lrb_stream_sr(int C, int group, int update_kind, int gate_kind);
-const void* find_lrb_stream_bdr(int C, int group, int update_kind, int gate_kind);
+const void* find_lrb_stream_rtn(int C, int group, int update_kind, int gate_kind,
+                                 bool merge);
+const void* find_lrb_stream_sr(int C, int group, int update_kind, int gate_kind,
+                                 bool merge);
+const void* find_lrb_stream_bdr(int C, int group, int update_kind, int gate_kind,
+                                 bool merge);
 
 struct LayoutArgs {
     uint8_t* codes;

@@ -298,8 +298,9 @@ __device__ __forceinline__ void new_scales(float A0, float A1, float2& snew, flo
 // as the floats kb + code (kb: word_bias of the two elements' word positions)
 // whose low bits are the stored byte (nibble). inv, s_new: the column's values
 // in both halves. The value rounded is the exact product x*inv: one fused
-// multiply-add rounds it straight to an integer.
-template <int MODE, int BITS>
+// multiply-add rounds it straight to an integer. HASH64 selects the 64-bit
+// form of the SR draw (identical bits).
+template <int MODE, int BITS, bool HASH64 = false>
 __device__ __forceinline__ float2 round_rows(float2 x, float2 inv, float2 deq, float2 s_new,
                                              float2 kb, uint64_t hkey, uint32_t i, uint32_t j) {
     constexpr float QMAX = Q<BITS>::kMax;
@@ -315,10 +316,16 @@ __device__ __forceinline__ float2 round_rows(float2 x, float2 inv, float2 deq, f
             const float2 f = add2(fma2_rm(x, inv, f2(kRound)), f2(-kRound));
             const float2 fr = fma2(x, inv, neg2(f));                      // fraction, rounded once
             const float2 f1 = add2(f, f2(1.0f));
-            const HashColumn hc = hash_column(hkey, j);
-            const uint32_t khi = static_cast<uint32_t>(hkey >> 32) ^ i;
-            const float u0 = hash_uniform(khi, hc);
-            const float u1 = hash_uniform(khi ^ 1u, hc);                 // row i + 1 (i even)
+            float u0, u1;
+            if constexpr (HASH64) {
+                u0 = element_uniform_u64(hkey, i, j);
+                u1 = element_uniform_u64(hkey, i + 1, j);
+            } else {
+                const HashColumn hc = hash_column(hkey, j);
+                const uint32_t khi = static_cast<uint32_t>(hkey >> 32) ^ i;
+                u0 = hash_uniform(khi, hc);
+                u1 = hash_uniform(khi ^ 1u, hc);                         // row i + 1 (i even)
+            }
             c.x = u0 < fr.x ? f1.x : f.x;
             c.y = u1 < fr.y ? f1.y : f.y;
         } else {
