@@ -1,6 +1,6 @@
 // chunk_bdr.cu -- compiled variants of the chunked (multi-token) update with
 // BDR rounding at the chunk's end.
-#include "chunk_kernel.cuh"
+#include "chunk_gated.cuh"
 
 namespace lrs {
 LRS_CHUNK_VARIANTS(find_chunk_kernel_bdr, kBDR)

@@ -48,7 +48,9 @@ struct ChunkParams {
 };
 
 // Shared memory of one CTA: barriers | codes (int8 capacity) | scales |
-// token slots (q, k, [gate], v as fp32).
+// token slots (q, k, [gate], v as fp32). A slot is padded by 16 bytes so that
+// the same row of two adjacent slots falls in different shared-memory banks
+// (chunk_gated_kernel reads two tokens' rows at once).
 template <int DK, int DV, int GROUP, int GATE>
 struct ChunkSmem {
     static constexpr int G = DK / GROUP;
@@ -57,7 +59,7 @@ struct ChunkSmem {
     static constexpr int kRing = kScales + G * DV * 4;
     static constexpr int kQ = 0, kK = DK * 4, kG = 2 * DK * 4;
     static constexpr int kV = kG + (GATE == kGatePerKey ? DK * 4 : 0);
-    static constexpr int kTok = kV + DV * 4;
+    static constexpr int kTok = kV + DV * 4 + 16;
     static constexpr int kBytes = kRing + kChunkSlots * kTok;
     static_assert(kTok % 16 == 0 && kRing % 16 == 0, "alignment");
 };
@@ -441,19 +443,17 @@ __global__ void __launch_bounds__(DV, (3 * 128) / DV) chunk_kernel(const ChunkPa
 
 // Defines `ChunkKernel NAME(int d_k, int d_v, int group, int update_kind,
 // int gate_kind)`: the chunk kernel with rounding MODE for that shape, with its
-// shared-memory bytes, or {nullptr, 0} when it is not compiled.
+// shared-memory bytes, or {nullptr, 0} when it is not compiled. The gated
+// forms take chunk_gated_kernel (chunk_gated.cuh, which the compiling file
+// includes) where a scale group fits in half the key rows.
 #define LRS_CHUNK_PICK(NAME, MODE, DK, DV, GROUP)                                              \
     if (d_k == DK && d_v == DV && group == GROUP) {                                            \
         using S = ChunkSmem<DK, DV, GROUP, kGatePerKey>;                                       \
         using S1 = ChunkSmem<DK, DV, GROUP, kGate>;                                            \
         if (update_kind == kGated && gate_kind == kGatePerKey)                                 \
-            return {reinterpret_cast<const void*>(                                             \
-                        &chunk_kernel<DK, DV, GROUP, kGated, kGatePerKey, MODE>),              \
-                    S::kBytes};                                                                \
+            return {chunk_gated_pick<DK, DV, GROUP, kGatePerKey, MODE>(), S::kBytes};          \
         if (update_kind == kGated && gate_kind == kGate)                                       \
-            return {reinterpret_cast<const void*>(                                             \
-                        &chunk_kernel<DK, DV, GROUP, kGated, kGate, MODE>),                    \
-                    S1::kBytes};                                                               \
+            return {chunk_gated_pick<DK, DV, GROUP, kGate, MODE>(), S1::kBytes};               \
         if (update_kind == kDelta && gate_kind == kGate)                                       \
             return {reinterpret_cast<const void*>(                                             \
                         &chunk_kernel<DK, DV, GROUP, kDelta, kGate, MODE>),                    \

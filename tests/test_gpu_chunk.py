@@ -63,6 +63,16 @@ def test_chunk_lengths(T):
     run_chunks(w, T=T, n_chunks=2)
 
 
+@pytest.mark.parametrize("T", [1, 2, 3, 8, 9, 17])
+@pytest.mark.parametrize("fam,mode", [("gla", I.ROUND_BDR), ("mamba2", I.ROUND_SR)])
+def test_chunk_lengths_gated(fam, mode, T):
+    """The gated forms' kernel skews its two row halves by one token: chunks
+    of one token, of fewer tokens than ring slots, and of more."""
+    d_v = 64 if fam == "mamba2" else 128
+    w = _small(fam, 2, 3, 128, d_v, 32, mode, "mixed", steps=2)
+    run_chunks(w, T=T, n_chunks=2)
+
+
 @pytest.mark.parametrize("d_k,d_v,group", [(64, 64, 16), (64, 128, 32), (128, 64, 32),
                                            (64, 64, 64)])
 def test_chunk_shapes(d_k, d_v, group):
