@@ -3,10 +3,12 @@
 //
 // What it computes is chunk_kernel.cuh's: T tokens applied in order to the
 // dequantized state in fp32, one output per token, one requantization at the
-// end. The mapping differs. Thread (column pair cp, half h) holds columns
-// 2cp and 2cp + 1 over key rows [h*d_k/2, (h+1)*d_k/2) in registers, so one
-// broadcast shared-memory load of q, k or the gates feeds two columns, and
-// each thread runs two independent output chains.
+// end. The mapping differs. The key rows are cut into SEG segments (2 in the
+// compiled variants); a thread holds SEG/2 column pairs over one segment's rows
+// in registers, so one broadcast shared-memory load of q, k or the gates
+// feeds SEG columns, and each thread runs SEG independent output chains. The
+// description below is for SEG = 2; with more segments each passes its
+// partial sums to the next, one token later.
 //
 // The output o_j = sum_i q_i x_ij is one chain in key order: the lower half
 // computes its rows' part and the upper half continues from it. The halves
@@ -113,25 +115,33 @@ __device__ __forceinline__ float2 gated_requantize_group(uint8_t* cs, const floa
     return snew;
 }
 
-template <int DK, int DV, int GROUP, int GATE, int MODE>
+template <int DK, int DV, int GROUP, int GATE, int MODE, int SEG>
 __global__ void __launch_bounds__(DV, (3 * 128) / DV) chunk_gated_kernel(const ChunkParams p) {
     using S = ChunkSmem<DK, DV, GROUP, GATE>;
     constexpr int G = DK / GROUP;
     constexpr int C = DV / 32;
-    constexpr int HK = DK / 2;                   // rows per half
-    constexpr int GH = HK / GROUP;               // scale groups per half
-    static_assert(GROUP <= HK && HK % GROUP == 0, "a scale group must lie in one half");
+    constexpr int NP = SEG / 2;                  // column pairs per thread
+    constexpr int CPL = 2 * NP;                  // columns per thread
+    constexpr int LPS = 32 / SEG;                // lanes per row segment
+    constexpr int RS = DK / SEG;                 // key rows per segment
+    constexpr int GS = RS / GROUP;               // scale groups per segment
+    static_assert(SEG == 2 || SEG == 4, "two or four row segments");
+    static_assert(GROUP <= RS && RS % GROUP == 0 && RS % 4 == 0, "a scale group must lie in one segment");
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* bar_state = reinterpret_cast<uint64_t*>(smem);
     uint64_t* bar_tok = bar_state + 1;
     uint8_t* cs = smem + S::kCodes;
     float* ss = reinterpret_cast<float*>(smem + S::kScales);
     const int lane = threadIdx.x & 31;
-    const int h = lane >> 4;                     // 0: lower rows, 1: upper rows
-    const int cp = (threadIdx.x >> 5) * 16 + (lane & 15);
-    const int c0 = 2 * cp;                       // the pair's first column
-    const int own = c0 / C, pc = (c0 % C) / 2;   // its place in the state layout
-    const int rbase = h * HK;
+    const int seg = lane / LPS;                  // this thread's row segment
+    const int cbase = (threadIdx.x >> 5) * 32 + (lane % LPS) * CPL;   // its first column
+    const int rbase = seg * RS;
+    int own[NP], pc[NP];                         // each pair's place in the state layout
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+        own[q] = (cbase + 2 * q) / C;
+        pc[q] = ((cbase + 2 * q) % C) / 2;
+    }
 
     if (threadIdx.x == 0) {
         mbar_init(bar_state, 1);
@@ -178,51 +188,69 @@ __global__ void __launch_bounds__(DV, (3 * 128) / DV) chunk_gated_kernel(const C
         }
         par_state ^= 1u;
 
-        // the thread's rows of both columns, as row pairs
-        float2 xa[HK / 2], xb[HK / 2];
+        // the thread's rows of its columns, as row pairs: x[pair][column][row pair]
+        float2 x[NP][2][RS / 2];
 #pragma unroll
-        for (int gh = 0; gh < GH; ++gh) {
-            const int g = h * GH + gh;
+        for (int gs = 0; gs < GS; ++gs) {
+            const int g = seg * GS + gs;
             const int gbase = static_cast<int>(tl.goff(g, GROUP * DV / 2));
-            float2 ya[GROUP / 2], yb[GROUP / 2];
-            if (tl.bits(g) == 8)
-                gated_decode_group<DV, GROUP, 8>(cs, ss, gbase, g, pc, own, c0, ya, yb);
-            else
-                gated_decode_group<DV, GROUP, 4>(cs, ss, gbase, g, pc, own, c0, ya, yb);
 #pragma unroll
-            for (int r2 = 0; r2 < GROUP / 2; ++r2) {
-                xa[gh * GROUP / 2 + r2] = ya[r2];
-                xb[gh * GROUP / 2 + r2] = yb[r2];
+            for (int q = 0; q < NP; ++q) {
+                float2 ya[GROUP / 2], yb[GROUP / 2];
+                if (tl.bits(g) == 8)
+                    gated_decode_group<DV, GROUP, 8>(cs, ss, gbase, g, pc[q], own[q], cbase + 2 * q,
+                                                     ya, yb);
+                else
+                    gated_decode_group<DV, GROUP, 4>(cs, ss, gbase, g, pc[q], own[q], cbase + 2 * q,
+                                                     ya, yb);
+#pragma unroll
+                for (int r2 = 0; r2 < GROUP / 2; ++r2) {
+                    x[q][0][gs * GROUP / 2 + r2] = ya[r2];
+                    x[q][1][gs * GROUP / 2 + r2] = yb[r2];
+                }
             }
         }
 
-        float2 carry = f2(0.0f);     // upper half: the lower half's partial sums
+        float carry[CPL];            // the previous segment's partial sums
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) carry[c] = 0.0f;
 #pragma unroll 1
-        for (int n = 0; n <= T; ++n) {
+        for (int n = 0; n < T + SEG - 1; ++n) {
+            // Token n: every thread waits on its barrier itself; a thread whose
+            // wait runs out skips the work, and the one CTA barrier of the
+            // iteration (below) ends the loop for all. The tokens of the other
+            // segments passed that barrier in earlier iterations.
+            bool good = true;
             if (n < T) {
                 const int64_t u = tok_base + n;
-                const bool good = mbar_wait_bounded(&bar_tok[u % NS],
-                                                    static_cast<uint32_t>((u / NS) & 1), p.timeout_ns);
-                if (__syncthreads_or(!good)) {
-                    ok = false;
-                    drain_lo = u;
-                    break;
-                }
+                good = mbar_wait_bounded(&bar_tok[u % NS], static_cast<uint32_t>((u / NS) & 1),
+                                         p.timeout_ns);
             }
-            const int t = n - h;                 // this half's token
-            float2 o = h ? carry : f2(0.0f);
-            if (t >= 0 && t < T) {
+            const int t = n - seg;               // this segment's token
+            float o[CPL];
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) o[c] = seg ? carry[c] : 0.0f;
+            if (good && t >= 0 && t < T) {
                 const int slot = static_cast<int>((tok_base + t) % NS);
                 const uint8_t* tb = smem + S::kRing + slot * S::kTok;
                 const float* tq = reinterpret_cast<const float*>(tb + S::kQ) + rbase;
                 const float* tkk = reinterpret_cast<const float*>(tb + S::kK) + rbase;
                 const float* tg = reinterpret_cast<const float*>(tb + S::kG) + rbase;
-                const float2 wv = *reinterpret_cast<const float2*>(tb + S::kV + c0 * 4);
-                const float2 w0 = f2(wv.x), w1 = f2(wv.y);
+                float2 wc[CPL];                  // w of each column, both halves
+                {
+                    const float* tv = reinterpret_cast<const float*>(tb + S::kV) + cbase;
+                    if constexpr (CPL == 2) {
+                        const float2 v2 = *reinterpret_cast<const float2*>(tv);
+                        wc[0] = f2(v2.x); wc[1] = f2(v2.y);
+                    } else {
+                        const float4 v4 = *reinterpret_cast<const float4*>(tv);
+                        wc[0] = f2(v4.x); wc[1] = f2(v4.y); wc[2] = f2(v4.z); wc[3] = f2(v4.w);
+                    }
+                }
                 const int64_t row = static_cast<int64_t>(t) * p.ntiles + tile;
                 const float2 gs2 = GATE == kGate ? f2(__ldg(p.gates + row)) : f2(0.0f);
 #pragma unroll
-                for (int r = 0; r < HK; r += 4) {
+                for (int r = 0; r < RS; r += 4) {
                     if (r % 16 == 0) asm volatile("" ::: "memory");   // bound the load hoisting
                     const float4 kv = lds4(tkk + r);
                     const float4 qv = lds4(tq + r);
@@ -233,67 +261,86 @@ __global__ void __launch_bounds__(DV, (3 * 128) / DV) chunk_gated_kernel(const C
                         g1 = make_float2(gv.z, gv.w);
                     }
                     const float2 k0 = make_float2(kv.x, kv.y), k1 = make_float2(kv.z, kv.w);
-                    // x = g * x + RN(k w), per column, row pairs
-                    const float2 a0 = fma2(g0, xa[r / 2], mul2(k0, w0));
-                    const float2 a1 = fma2(g1, xa[r / 2 + 1], mul2(k1, w0));
-                    const float2 b0 = fma2(g0, xb[r / 2], mul2(k0, w1));
-                    const float2 b1 = fma2(g1, xb[r / 2 + 1], mul2(k1, w1));
-                    xa[r / 2] = a0; xa[r / 2 + 1] = a1;
-                    xb[r / 2] = b0; xb[r / 2 + 1] = b1;
-                    // the two output chains, key order
-                    o.x = __fmaf_rn(qv.x, a0.x, o.x);
-                    o.y = __fmaf_rn(qv.x, b0.x, o.y);
-                    o.x = __fmaf_rn(qv.y, a0.y, o.x);
-                    o.y = __fmaf_rn(qv.y, b0.y, o.y);
-                    o.x = __fmaf_rn(qv.z, a1.x, o.x);
-                    o.y = __fmaf_rn(qv.z, b1.x, o.y);
-                    o.x = __fmaf_rn(qv.w, a1.y, o.x);
-                    o.y = __fmaf_rn(qv.w, b1.y, o.y);
+#pragma unroll
+                    for (int q = 0; q < NP; ++q) {
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc) {
+                            const int c = 2 * q + cc;
+                            // x = g * x + RN(k w), row pairs
+                            const float2 a = fma2(g0, x[q][cc][r / 2], mul2(k0, wc[c]));
+                            const float2 b = fma2(g1, x[q][cc][r / 2 + 1], mul2(k1, wc[c]));
+                            x[q][cc][r / 2] = a;
+                            x[q][cc][r / 2 + 1] = b;
+                            // this column's output chain, key order
+                            o[c] = __fmaf_rn(qv.x, a.x, o[c]);
+                            o[c] = __fmaf_rn(qv.y, a.y, o[c]);
+                            o[c] = __fmaf_rn(qv.z, b.x, o[c]);
+                            o[c] = __fmaf_rn(qv.w, b.y, o[c]);
+                        }
+                    }
                 }
-                if (h == 1) *reinterpret_cast<float2*>(p.out + row * DV + c0) = o;
+                if (seg == SEG - 1) {
+                    float* op = p.out + row * DV + cbase;
+                    if constexpr (CPL == 2)
+                        *reinterpret_cast<float2*>(op) = make_float2(o[0], o[1]);
+                    else
+                        *reinterpret_cast<float4*>(op) = make_float4(o[0], o[1], o[2], o[3]);
+                }
             }
-            // the lower half's partial sums of token n go to the upper half
-            const float ox = __shfl_up_sync(0xffffffffu, o.x, 16);
-            const float oy = __shfl_up_sync(0xffffffffu, o.y, 16);
-            carry = make_float2(ox, oy);
-            __syncthreads();                     // every thread is done with token n - 1
-            if (threadIdx.x == 0 && n >= 1 && n - 1 + NS < T) {
-                const int64_t u = tok_base + n - 1;
+            // each segment's partial sums go to the next segment
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) carry[c] = __shfl_up_sync(0xffffffffu, o[c], LPS);
+            // every thread is done with token n - SEG + 1; any wait that ran out
+            if (__syncthreads_or(!good)) {
+                ok = false;
+                drain_lo = tok_base + n;
+                break;
+            }
+            const int done = n - SEG + 1;        // the token no segment reads again
+            if (threadIdx.x == 0 && done >= 0 && done + NS < T) {
+                const int64_t u = tok_base + done;
                 fence_proxy_async_smem();
-                issue_token<DK, DV, GROUP, GATE>(p, smem, static_cast<int>(u % NS), tile,
-                                                 n - 1 + NS);
+                issue_token<DK, DV, GROUP, GATE>(p, smem, static_cast<int>(u % NS), tile, done + NS);
                 issued_hi = u + NS + 1;
             }
         }
         if (!ok) break;
         tok_base += T;
 
-        // one requantization at the chunk's end, per thread and scale group
+        // one requantization at the chunk's end, per thread, pair and scale group
         const int b = tile / p.H, hh = tile - b * p.H;
         const uint64_t hkey = MODE == kSR ? tile_hash_key(p.seed, p.step,
                                                           static_cast<uint32_t>(b),
                                                           static_cast<uint32_t>(hh))
                                           : 0ull;
-        float2 snew[GH];
+        float2 snew[GS][NP];
 #pragma unroll
-        for (int gh = 0; gh < GH; ++gh) {
-            const int g = h * GH + gh;
+        for (int gs = 0; gs < GS; ++gs) {
+            const int g = seg * GS + gs;
             const int gbase = static_cast<int>(tl.goff(g, GROUP * DV / 2));
-            float2 ya[GROUP / 2], yb[GROUP / 2];
 #pragma unroll
-            for (int r2 = 0; r2 < GROUP / 2; ++r2) {
-                ya[r2] = xa[gh * GROUP / 2 + r2];
-                yb[r2] = xb[gh * GROUP / 2 + r2];
+            for (int q = 0; q < NP; ++q) {
+                float2 ya[GROUP / 2], yb[GROUP / 2];
+#pragma unroll
+                for (int r2 = 0; r2 < GROUP / 2; ++r2) {
+                    ya[r2] = x[q][0][gs * GROUP / 2 + r2];
+                    yb[r2] = x[q][1][gs * GROUP / 2 + r2];
+                }
+                snew[gs][q] =
+                    tl.bits(g) == 8
+                        ? gated_requantize_group<DV, GROUP, MODE, 8>(cs, ss, gbase, g, pc[q], own[q],
+                                                                     cbase + 2 * q, g * GROUP, ya,
+                                                                     yb, hkey)
+                        : gated_requantize_group<DV, GROUP, MODE, 4>(cs, ss, gbase, g, pc[q], own[q],
+                                                                     cbase + 2 * q, g * GROUP, ya,
+                                                                     yb, hkey);
             }
-            snew[gh] = tl.bits(g) == 8
-                           ? gated_requantize_group<DV, GROUP, MODE, 8>(cs, ss, gbase, g, pc, own,
-                                                                        c0, g * GROUP, ya, yb, hkey)
-                           : gated_requantize_group<DV, GROUP, MODE, 4>(cs, ss, gbase, g, pc, own,
-                                                                        c0, g * GROUP, ya, yb, hkey);
         }
 #pragma unroll
-        for (int gh = 0; gh < GH; ++gh)
-            *reinterpret_cast<float2*>(ss + (h * GH + gh) * DV + c0) = snew[gh];
+        for (int gs = 0; gs < GS; ++gs)
+#pragma unroll
+            for (int q = 0; q < NP; ++q)
+                *reinterpret_cast<float2*>(ss + (seg * GS + gs) * DV + cbase + 2 * q) = snew[gs][q];
         __syncthreads();
         // write the tile back: 16-byte streaming stores
         uint8_t* gc = p.codes + code_off;
@@ -319,10 +366,13 @@ __global__ void __launch_bounds__(DV, (3 * 128) / DV) chunk_gated_kernel(const C
 
 // The gated form's chunk kernel for a shape: this one where a scale group
 // fits in half the key rows, chunk_kernel otherwise.
+// (Four segments, each thread holding two pairs over a quarter of the rows,
+// measured 3-5% slower than two on the throughput and int4 workloads: the
+// three-token skew costs more than the extra chains per thread save.)
 template <int DK, int DV, int GROUP, int GATE, int MODE>
 inline const void* chunk_gated_pick() {
     if constexpr (GROUP <= DK / 2)
-        return reinterpret_cast<const void*>(&chunk_gated_kernel<DK, DV, GROUP, GATE, MODE>);
+        return reinterpret_cast<const void*>(&chunk_gated_kernel<DK, DV, GROUP, GATE, MODE, 2>);
     else
         return reinterpret_cast<const void*>(&chunk_kernel<DK, DV, GROUP, kGated, GATE, MODE>);
 }
