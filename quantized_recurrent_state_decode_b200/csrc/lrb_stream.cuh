@@ -16,7 +16,9 @@
 //     quantization step;
 //   - the output adds sum_l f_l V'_l,j after the key-order chain;
 //   - U' and V' (or zeros after a merge) go back to global memory.
-// All modes use the staged pair code (updated values in shared memory).
+// SR and BDR use the staged pair code (updated values in shared memory), RTN
+// keeps a group's values in registers. Merge steps and the other steps are
+// separate instantiations (MERGE), so the others carry no merge code.
 #pragma once
 
 #include "step_kernel.cuh"
