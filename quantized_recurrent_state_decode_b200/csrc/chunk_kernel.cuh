@@ -187,7 +187,7 @@ __device__ __forceinline__ float requantize_group(float (&x)[DK], int g, const u
     for (int r = g * GROUP; r < (g + 1) * GROUP; r += 2) {
         const int rl = r - g * GROUP;
         const float2 d0 = MODE == kBDR ? make_float2(deq0[rl], deq0[rl + 1]) : f2(0.0f);
-        const float2 tv = round_rows<MODE, BITS, true>(make_float2(x[r], x[r + 1]), inv2, d0, s2, kb,
+        const float2 tv = round_rows<MODE, BITS, false>(make_float2(x[r], x[r + 1]), inv2, d0, s2, kb,
                                                  hkey, static_cast<uint32_t>(r),
                                                  static_cast<uint32_t>(j));
         x[r] = tv.x;

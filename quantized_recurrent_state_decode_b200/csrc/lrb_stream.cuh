@@ -274,24 +274,39 @@ __device__ __forceinline__ void pair_step_lrb_rtn(const uint8_t* __restrict__ cs
     }
     if (merge) {
         // a separate pass over the group, so the merge's values are not live
-        // beside the decode's
+        // beside the decode's; four rows of each component per 16-byte load,
+        // the columns' V' values broadcast into pairs once
+        float2 v0b[kLrbStreamMaxRank], v1b[kLrbStreamMaxRank];
 #pragma unroll
-        for (int rp = 0; rp < GROUP / 2; ++rp) {
-            float2 m0 = f2(0.0f), m1 = f2(0.0f);
+        for (int l = 0; l < kLrbStreamMaxRank; ++l) {
+            v0b[l] = f2(vc0[l]);
+            v1b[l] = f2(vc1[l]);
+        }
+#pragma unroll
+        for (int rq = 0; rq < GROUP / 4; ++rq) {
+            float2 m00 = f2(0.0f), m01 = f2(0.0f), m10 = f2(0.0f), m11 = f2(0.0f);
 #pragma unroll
             for (int l = 0; l < kLrbStreamMaxRank; ++l) {
                 if (l < R) {
-                    const float2 u = *reinterpret_cast<const float2*>(Ut + l * dk + 2 * rp);
-                    m0 = fma2(u, f2(vc0[l]), m0);
-                    m1 = fma2(u, f2(vc1[l]), m1);
+                    const float4 u = *reinterpret_cast<const float4*>(Ut + l * dk + 4 * rq);
+                    const float2 ua = make_float2(u.x, u.y), ub = make_float2(u.z, u.w);
+                    m00 = fma2(ua, v0b[l], m00);
+                    m01 = fma2(ua, v1b[l], m01);
+                    m10 = fma2(ub, v0b[l], m10);
+                    m11 = fma2(ub, v1b[l], m11);
                 }
             }
-            const float2 x0 = x[rp][0], x1 = x[rp][1];
-            const float2 y0 = add2(x0, m0), y1 = add2(x1, m1);
-            x[rp][0].x = fabsf(m0.x) >= half0 ? y0.x : x0.x;
-            x[rp][0].y = fabsf(m0.y) >= half0 ? y0.y : x0.y;
-            x[rp][1].x = fabsf(m1.x) >= half1 ? y1.x : x1.x;
-            x[rp][1].y = fabsf(m1.y) >= half1 ? y1.y : x1.y;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int rp = 2 * rq + h;
+                const float2 m0 = h ? m10 : m00, m1 = h ? m11 : m01;
+                const float2 x0 = x[rp][0], x1 = x[rp][1];
+                const float2 y0 = add2(x0, m0), y1 = add2(x1, m1);
+                x[rp][0].x = fabsf(m0.x) >= half0 ? y0.x : x0.x;
+                x[rp][0].y = fabsf(m0.y) >= half0 ? y0.y : x0.y;
+                x[rp][1].x = fabsf(m1.x) >= half1 ? y1.x : x1.x;
+                x[rp][1].y = fabsf(m1.y) >= half1 ? y1.y : x1.y;
+            }
         }
     }
     float a0 = 0.0f, a1 = 0.0f, b0 = 0.0f, b1 = 0.0f;
