@@ -122,6 +122,12 @@ __device__ __forceinline__ void pair_step_lrb(const uint8_t* __restrict__ cs, in
     const float2 gsc = f2(gscalar);
     const float half0 = __fmul_rn(0.5f, sc.x), half1 = __fmul_rn(0.5f, sc.y);
     float a0 = 0.0f, b0 = 0.0f;
+    float2 v0b[kLrbStreamMaxRank], v1b[kLrbStreamMaxRank];   // V' broadcast into pairs once
+#pragma unroll
+    for (int l = 0; l < kLrbStreamMaxRank; ++l) {
+        v0b[l] = f2(vc0[l]);
+        v1b[l] = f2(vc1[l]);
+    }
 
 #pragma unroll 1
     for (int un = 0; un < G::UNITS; ++un) {
@@ -160,8 +166,8 @@ __device__ __forceinline__ void pair_step_lrb(const uint8_t* __restrict__ cs, in
                     for (int l = 0; l < kLrbStreamMaxRank; ++l) {
                         if (l < R) {
                             const float2 u = *reinterpret_cast<const float2*>(Ut + l * dk + r);
-                            m0 = fma2(u, f2(vc0[l]), m0);
-                            m1 = fma2(u, f2(vc1[l]), m1);
+                            m0 = fma2(u, v0b[l], m0);
+                            m1 = fma2(u, v1b[l], m1);
                         }
                     }
                     const float2 y0 = add2(x0, m0), y1 = add2(x1, m1);

@@ -68,8 +68,11 @@ def test_lrb_family_mode_grid(fam, mode, prec, rank):
 
 
 @pytest.mark.parametrize("rank", [1, 2, 3, 8])
-def test_lrb_ranks(rank):
-    w = _small("gla", 2, 3, 128, 128, 32, I.ROUND_SR, "mixed", steps=2 * rank + 1)
+@pytest.mark.parametrize("mode", [I.ROUND_RTN, I.ROUND_SR])
+def test_lrb_ranks(rank, mode):
+    """Every rank through two merge cycles, on the register (RTN) and the
+    staged (SR) pair code."""
+    w = _small("gla", 2, 3, 128, 128, 32, mode, "mixed", steps=2 * rank + 1)
     run_lrb(w, rank=rank, steps=2 * rank + 1)
 
 
