@@ -104,7 +104,7 @@ lrs_status launch_lrb_stream(const lrs_state* st, void* state_codes, float* scal
     int slots = sh.update_kind == LRS_UPDATE_DELTA ? G : std::min(2, G);
     slots = std::max(1, std::min(slots, lrs::kMaxSlots));
     const int warp_smem =
-        lrb_stream_warp_smem(C, sh.group, sh.gate_kind, slots, sh.d_k, mode != LRS_ROUND_RTN);
+        lrb_stream_warp_smem(C, sh.group, sh.gate_kind, slots, sh.d_k, lrs::lrb_staged(mode, merge));
     constexpr int kSmemLimit = 227 * 1024;
     const int warps = std::min(lrs::lrb_max_warps(mode, merge, sh.group), kSmemLimit / warp_smem);
     if (warps < 1) return LRS_ERR_UNSUPPORTED;

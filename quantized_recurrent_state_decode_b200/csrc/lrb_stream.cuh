@@ -105,7 +105,7 @@ __device__ __forceinline__ void lrb_issue_item(const LrbStreamParams& lp, uint8_
 // step; then the output chain, new scales and codes as pair_step_xs.
 // Ut: U' (decayed, appended; component-major, d_k floats per component) at
 // the group's first row. vc0, vc1: V'[l] of the pair's two columns.
-template <int GROUP, int GATE, int MODE, int BITS>
+template <int GROUP, int GATE, int MODE, int BITS, bool STAGE>
 __device__ __forceinline__ void pair_step_lrb(const uint8_t* __restrict__ cs, int ubase, float2 sc,
                                               const float* __restrict__ qs,
                                               const float* __restrict__ gs, float gscalar,
@@ -178,7 +178,8 @@ __device__ __forceinline__ void pair_step_lrb(const uint8_t* __restrict__ cs, in
                 }
                 a0 = max_abs3(a0, x0.x, x0.y);
                 b0 = max_abs3(b0, x1.x, x1.y);
-                xs[(un * RPUH + rl / 2) * 32 + lane] = make_float4(x0.x, x0.y, x1.x, x1.y);
+                if constexpr (STAGE)
+                    xs[(un * RPUH + rl / 2) * 32 + lane] = make_float4(x0.x, x0.y, x1.x, x1.y);
             }
         }
     }
@@ -189,6 +190,9 @@ __device__ __forceinline__ void pair_step_lrb(const uint8_t* __restrict__ cs, in
     const float2 inv0 = f2(inv.x), inv1 = f2(inv.y);
     const float2 sn0 = f2(snew.x), sn1 = f2(snew.y);
 
+    // Without a merge (STAGE false, BDR), x = RN(g deq) is recomputed from
+    // the old codes the rounding decodes anyway, by the same operations.
+    static_assert(STAGE || MODE == kBDR, "only BDR recomputes x");
 #pragma unroll 1
     for (int un = 0; un < G::UNITS; ++un) {
         uint32_t ow[4];
@@ -197,6 +201,8 @@ __device__ __forceinline__ void pair_step_lrb(const uint8_t* __restrict__ cs, in
             const uint4 raw = lds_unit(cs, ubase + un, lane);
             wd[0] = raw.x; wd[1] = raw.y; wd[2] = raw.z; wd[3] = raw.w;
         }
+        float gg[STAGE || GATE != kGatePerKey ? 1 : G::RPU];
+        if constexpr (!STAGE && GATE == kGatePerKey) ld_smem_rows<G::RPU>(gs + un * G::RPU, gg);
 #pragma unroll
         for (int wi = 0; wi < 4; ++wi) {
             float f[G::EPW];
@@ -205,11 +211,18 @@ __device__ __forceinline__ void pair_step_lrb(const uint8_t* __restrict__ cs, in
 #pragma unroll
             for (int rp = 0; rp < G::RPW / 2; ++rp) {
                 const int rl = wi * G::RPW + 2 * rp;
-                const float4 xv = xs[(un * RPUH + rl / 2) * 32 + lane];
                 float2 dq0 = f2(0.0f), dq1 = f2(0.0f);
                 if constexpr (MODE == kBDR) {
                     dq0 = mul2(add2(make_float2(f[4 * rp], f[4 * rp + 2]), f2(-(kTwo23 + BIAS))), s0);
                     dq1 = mul2(add2(make_float2(f[4 * rp + 1], f[4 * rp + 3]), f2(-(kTwo23 + BIAS))), s1);
+                }
+                float4 xv;
+                if constexpr (STAGE) {
+                    xv = xs[(un * RPUH + rl / 2) * 32 + lane];
+                } else {
+                    const float2 gr = GATE == kGatePerKey ? make_float2(gg[rl], gg[rl + 1]) : gsc;
+                    const float2 x0 = mul2(gr, dq0), x1 = mul2(gr, dq1);
+                    xv = make_float4(x0.x, x0.y, x1.x, x1.y);
                 }
                 const uint32_t i = static_cast<uint32_t>(row0 + un * G::RPU + rl);
                 const float2 kb0 = make_float2(word_bias<BITS>(4 * rp), word_bias<BITS>(4 * rp + 2));
@@ -380,10 +393,15 @@ __device__ __forceinline__ float lrb_chain(const float* a, const float* b, const
 // Launch bound in warps. A merge step (MERGE: step mod rank = rank - 1) and
 // the staged rounding modes take 8, so up to 255 registers: the merge's
 // buffer rows do not fit beside a register-resident group in 168. The other
-// RTN steps with groups of up to 32 rows are compiled without the merge code
-// and take up to 12 (shared memory leaves 10 for d_k = d_v = 128).
+// RTN and BDR steps with groups of up to 32 rows are compiled without the merge
+// code and take up to 12 (shared memory leaves 10 for d_k = d_v = 128).
 __host__ __device__ constexpr int lrb_max_warps(int mode, bool merge, int group) {
-    return (mode == kRTN && !merge && group <= 32) ? 12 : 8;
+    return (mode != kSR && !merge && group <= 32) ? 12 : 8;
+}
+// Whether the pair code stages the updated values in shared memory: SR, and
+// every merge step. A non-merge BDR step recomputes them (more warps fit).
+__host__ __device__ constexpr bool lrb_staged(int mode, bool merge) {
+    return mode == kSR || (mode == kBDR && merge);
 }
 
 template <int C, int GROUP, int UPD, int GATE, int MODE, bool MERGE>
@@ -630,12 +648,12 @@ __global__ void __launch_bounds__(lrb_max_warps(MODE, MERGE, GROUP) * 32, 1)
                                                           gs, gscalar, op, gcodes, gscale + 2 * pc,
                                                           lane, merge, R, Ug, dk, vc0, vc1);
                 } else if (int8g)
-                    pair_step_lrb<GROUP, GATE, MODE, 8>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs, gs,
+                    pair_step_lrb<GROUP, GATE, MODE, 8, lrb_staged(MODE, MERGE)>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs, gs,
                                                         gscalar, op, gcodes, gscale + 2 * pc, hkey,
                                                         g * GROUP, j0, lane, xs, merge, R, Ug, dk,
                                                         vc0, vc1);
                 else
-                    pair_step_lrb<GROUP, GATE, MODE, 4>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs, gs,
+                    pair_step_lrb<GROUP, GATE, MODE, 4, lrb_staged(MODE, MERGE)>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs, gs,
                                                         gscalar, op, gcodes, gscale + 2 * pc, hkey,
                                                         g * GROUP, j0, lane, xs, merge, R, Ug, dk,
                                                         vc0, vc1);
