@@ -47,6 +47,8 @@ def lib():
         L.orc_lrb_step.argtypes = [i32, P, P, i32, i32, i32, i32, i32, i32, P, P, P, i32, P, P,
                                    P, P, P, P, P, P, u64, u64, P]
         L.orc_lrb_step.restype = i32
+        L.orc_lrb_step_pg.argtypes = L.orc_lrb_step.argtypes
+        L.orc_lrb_step_pg.restype = i32
         L.orc_bf16_rne.argtypes = [ctypes.c_float]
         L.orc_bf16_rne.restype = ctypes.c_uint16
         L.orc_bf16_rne_array.argtypes = [i64, P, P]
@@ -157,7 +159,8 @@ def chunk_step(codes, scales, q, k, v, gates, beta, prec_map, tile_b, tile_h, *,
 def lrb_step(codes, scales, U, V, q, k, v, gates, beta, prec_map, tile_b, tile_h, *, group,
              update_kind, gate_kind, mode, rank, seed=0, step=0, want_x=False):
     """Decode step with Low-Rank Bypass; codes, scales, U [n][rank][d_k] and V
-    [n][rank][d_v] (float32) updated in place. Returns out [n][d_v] (and the
+    [n][rank][d_v] (float32) updated in place. prec_map is [H] (per head) or
+    [H][d_k/group] (per head and scale group). Returns out [n][d_v] (and the
     values before rounding [n][d_k][d_v] with want_x)."""
     n, d_k, d_v = codes.shape
     assert codes.dtype == np.int8 and scales.dtype == np.float32
@@ -169,9 +172,10 @@ def lrb_step(codes, scales, U, V, q, k, v, gates, beta, prec_map, tile_b, tile_h
     tile_h = np.ascontiguousarray(tile_h, dtype=np.int32)
     out = np.zeros((n, d_v), np.float32)
     x = np.zeros((n, d_k, d_v), np.float32) if want_x else None
-    rc = lib().orc_lrb_step(n, _p(tile_b), _p(tile_h), d_k, d_v, group, update_kind, gate_kind,
-                            mode, _p(prec_map), _p(codes), _p(scales), rank, _p(U), _p(V), _p(q),
-                            _p(k), _p(v), _p(gates), _p(beta), _p(out), seed, step, _p(x))
+    fn = _per_group(prec_map, d_k, group, lib().orc_lrb_step, lib().orc_lrb_step_pg)
+    rc = fn(n, _p(tile_b), _p(tile_h), d_k, d_v, group, update_kind, gate_kind, mode,
+            _p(prec_map), _p(codes), _p(scales), rank, _p(U), _p(V), _p(q), _p(k), _p(v),
+            _p(gates), _p(beta), _p(out), seed, step, _p(x))
     if rc != 0:
         raise ValueError("orc_lrb_step rejected its arguments (%d)" % rc)
     return (out, x) if want_x else out

@@ -512,11 +512,11 @@ static void lrb_tile(int d_k, int d_v, int group, const int *qmaxs, int update_k
     requantize_tile(d_k, d_v, group, qmaxs, mode, x, deq, c, s, seed, step, b, h);
 }
 
-int orc_lrb_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int d_k, int d_v,
-                 int group, int update_kind, int gate_kind, int mode, const uint8_t *prec_map,
-                 int8_t *codes, float *scales, int rank, float *U, float *V, const float *q,
-                 const float *k, const float *v, const float *gates, const float *beta,
-                 float *out, uint64_t seed, uint64_t step, float *x_out)
+static int lrb_impl(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int d_k, int d_v,
+                    int group, int update_kind, int gate_kind, int mode, const uint8_t *prec_map,
+                    int prec_groups, int8_t *codes, float *scales, int rank, float *U, float *V,
+                    const float *q, const float *k, const float *v, const float *gates,
+                    const float *beta, float *out, uint64_t seed, uint64_t step, float *x_out)
 {
     if (ntiles < 0 || check_shape(d_k, d_v, group, update_kind, gate_kind) != 0) return -1;
     if (mode != ORC_ROUND_RTN && mode != ORC_ROUND_SR && mode != ORC_ROUND_BDR) return -1;
@@ -527,7 +527,7 @@ int orc_lrb_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int d
         return -1;
     if (update_kind == ORC_UPDATE_DELTA && !beta) return -1;
     int G = d_k / group;
-    int rc = check_prec(ntiles, tile_h, prec_map, 1, G);
+    int rc = check_prec(ntiles, tile_h, prec_map, prec_groups, G);
     if (rc != 0) return rc;
     size_t n = (size_t)d_k * d_v;
     float *deq = (float *)malloc(n * sizeof(float));
@@ -542,7 +542,7 @@ int orc_lrb_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int d
     int m = (int)(step % (uint64_t)rank);
     size_t gate_len = (gate_kind == ORC_GATE_PER_KEY) ? (size_t)d_k : 1;
     for (int t = 0; t < ntiles; ++t) {
-        head_qmaxs(prec_map, 1, G, tile_h[t], qm);
+        head_qmaxs(prec_map, prec_groups, G, tile_h[t], qm);
         lrb_tile(d_k, d_v, group, qm, update_kind, gate_kind, mode, rank, m, codes + t * n,
                  scales + (size_t)t * G * d_v, U + (size_t)t * rank * d_k,
                  V + (size_t)t * rank * d_v, q + (size_t)t * d_k, k + (size_t)t * d_k,
@@ -552,6 +552,29 @@ int orc_lrb_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int d
     }
     free(deq); free(x); free(M); free(w); free(qm);
     return 0;
+}
+
+int orc_lrb_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int d_k, int d_v,
+                 int group, int update_kind, int gate_kind, int mode, const uint8_t *prec_map,
+                 int8_t *codes, float *scales, int rank, float *U, float *V, const float *q,
+                 const float *k, const float *v, const float *gates, const float *beta,
+                 float *out, uint64_t seed, uint64_t step, float *x_out)
+{
+    return lrb_impl(ntiles, tile_b, tile_h, d_k, d_v, group, update_kind, gate_kind, mode,
+                    prec_map, 1, codes, scales, rank, U, V, q, k, v, gates, beta, out, seed, step,
+                    x_out);
+}
+
+int orc_lrb_step_pg(int ntiles, const int32_t *tile_b, const int32_t *tile_h, int d_k, int d_v,
+                    int group, int update_kind, int gate_kind, int mode, const uint8_t *prec_map,
+                    int8_t *codes, float *scales, int rank, float *U, float *V, const float *q,
+                    const float *k, const float *v, const float *gates, const float *beta,
+                    float *out, uint64_t seed, uint64_t step, float *x_out)
+{
+    if (d_k <= 0 || group <= 0 || d_k % group != 0) return -1;
+    return lrb_impl(ntiles, tile_b, tile_h, d_k, d_v, group, update_kind, gate_kind, mode,
+                    prec_map, d_k / group, codes, scales, rank, U, V, q, k, v, gates, beta, out,
+                    seed, step, x_out);
 }
 
 uint16_t orc_bf16_rne(float x)

@@ -126,6 +126,14 @@ int orc_lrb_step(int ntiles, const int32_t *tile_b, const int32_t *tile_h,
                  float *V, const float *q, const float *k, const float *v, const float *gates,
                  const float *beta, float *out, uint64_t seed, uint64_t step, float *x_out);
 
+/* orc_lrb_step with one width per (head, scale group): prec_map [H][d_k/group]. */
+int orc_lrb_step_pg(int ntiles, const int32_t *tile_b, const int32_t *tile_h,
+                    int d_k, int d_v, int group, int update_kind, int gate_kind, int mode,
+                    const uint8_t *prec_map, int8_t *codes, float *scales, int rank, float *U,
+                    float *V, const float *q, const float *k, const float *v,
+                    const float *gates, const float *beta, float *out, uint64_t seed,
+                    uint64_t step, float *x_out);
+
 /* bfloat16 (the upper half of binary32: sign, 8 exponent bits, 7 fraction
  * bits) nearest to x, ties to the even fraction; NaN becomes a quiet NaN of the
  * same sign. Returns the 16-bit pattern. */

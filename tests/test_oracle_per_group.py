@@ -76,6 +76,55 @@ def test_mixed_groups_are_groupwise_head_runs(mode, delta, T):
         np.testing.assert_array_equal(runs["pg"][1][:, gi], ref[1][:, gi])
 
 
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("delta", [False, True])
+@pytest.mark.parametrize("step", [4, 7])                 # rank 4: step 7 merges, step 4 does not
+def test_lrb_mixed_groups_are_groupwise_head_runs(mode, delta, step):
+    """The same pins for the decode step with a Low-Rank Bypass buffer: with
+    codes valid at both widths, a per-group map gives the outputs and buffer
+    of both per-head runs, and each group the codes and scales of the run at
+    its width; a uniform per-group map is the per-head map."""
+    rng = np.random.default_rng(40 + 7 * mode + 3 * delta + step)
+    n, d_k, d_v, group, rank = 3, 32, 16, 8, 4
+    G = d_k // group
+    pm = np.array([[4, 8, 8, 4]], np.uint8)
+    codes8, scales = _state(rng, n, d_k, d_v, group, 8)
+    codes = codes8.copy()
+    for gi in range(G):
+        if pm[0, gi] == 4:
+            rows = slice(gi * group, (gi + 1) * group)
+            codes[:, rows] = np.clip(codes[:, rows] // 18, -7, 7)
+    q, k, v, g, beta = _chunk_inputs(rng, 1, n, d_k, d_v, per_key=not delta, delta=delta)
+    m = step % rank
+    U0 = np.zeros((n, rank, d_k), F32)
+    V0 = np.zeros((n, rank, d_v), F32)
+    U0[:, :m] = 0.3 * rng.standard_normal((n, m, d_k)).astype(F32)
+    V0[:, :m] = 0.3 * rng.standard_normal((n, m, d_v)).astype(F32)
+    kw = dict(group=group, update_kind=oracle.UPDATE_DELTA if delta else oracle.UPDATE_GATED,
+              gate_kind=oracle.GATE_SCALAR if delta else oracle.GATE_PER_KEY, mode=mode,
+              rank=rank, seed=13, step=step)
+    runs = {}
+    maps = (("pg", pm), ("8", np.array([8], np.uint8)), ("4", np.array([4], np.uint8)),
+            ("pg8", np.full((1, G), 8, np.uint8)))
+    for name, mp in maps:
+        c, sc, U, V = codes.copy(), scales.copy(), U0.copy(), V0.copy()
+        o = oracle.lrb_step(c, sc, U, V, q[0], k[0], v[0], g[0], None if beta is None else beta[0],
+                            mp, np.arange(n), np.zeros(n), **kw)
+        runs[name] = (c, sc, o, U, V)
+    for other in ("8", "4"):
+        for idx in (2, 3, 4):                      # output, U, V
+            np.testing.assert_array_equal(runs["pg"][idx], runs[other][idx])
+    for idx in range(5):
+        np.testing.assert_array_equal(runs["pg8"][idx], runs["8"][idx])
+    for gi in range(G):
+        ref = runs[str(pm[0, gi])]
+        rows = slice(gi * group, (gi + 1) * group)
+        np.testing.assert_array_equal(runs["pg"][0][:, rows], ref[0][:, rows])
+        np.testing.assert_array_equal(runs["pg"][1][:, gi], ref[1][:, gi])
+    if m + 1 == rank:
+        assert not runs["pg"][3].any() and not runs["pg"][4].any()     # emptied by the merge
+
+
 def test_import_per_group_widths():
     rng = np.random.default_rng(2)
     n, d_k, d_v, group = 2, 16, 8, 4
