@@ -237,9 +237,9 @@ lrs_status lrs_chunk_step(const lrs_state *st, void *state_codes, float *scales,
  *   - at the step that fills the buffer, every element of U V^T whose
  *     magnitude is at least half of its quantization step (old scale / 2) is
  *     added to x before the requantization, and the buffer is emptied.
- * Other arguments, layouts, errors and asynchrony as lrs_decode_step; states
- * with per-group widths are not supported (LRS_ERR_UNSUPPORTED); d_k and d_v
- * in {64, 128}. */
+ * Other arguments, layouts, errors and asynchrony as lrs_decode_step, including
+ * states with one width per (head, scale group) (lrs_state_alloc_groups); d_k
+ * and d_v in {64, 128}. */
 lrs_status lrs_lrb_step(const lrs_state *st, void *state_codes, float *scales,
                         const uint8_t *prec_map, int32_t rank, float *U, float *V,
                         const float *q, const float *k, const float *v, const float *gates,

@@ -188,8 +188,6 @@ lrs_status lrs_lrb_step(const lrs_state* st, void* state_codes, float* scales,
         return lrs::api_fail(LRS_ERR_INVALID_ARG, "rank must be in [1, 8]");
     if (mode != LRS_ROUND_RTN && mode != LRS_ROUND_SR && mode != LRS_ROUND_BDR)
         return lrs::api_fail(LRS_ERR_INVALID_ARG, "mode is not an lrs_round_mode");
-    if (lrs::state_prec_groups(st) != 1)
-        return lrs::api_fail(LRS_ERR_UNSUPPORTED, "the bypass step takes per-head widths");
     const void* ptrs[] = {state_codes, scales, U, V, q, k, v, gates, out};
     for (const void* p : ptrs) {
         if (!p) return lrs::api_fail(LRS_ERR_INVALID_ARG, "a buffer is NULL");
@@ -245,7 +243,7 @@ lrs_status lrs_lrb_step(const lrs_state* st, void* state_codes, float* scales,
     p.H = sh.heads;
     p.ntiles = static_cast<int32_t>(ntiles);
     p.rank = rank;
-    p.pgroups = 1;
+    p.pgroups = lrs::state_prec_groups(st);
     p.inject = lrs::take_injected_timeout(&p.timeout_ns) ? 1 : 0;
     const int grid = static_cast<int>(std::min<int64_t>(ntiles, int64_t(sms) * per_sm));
     void* args[] = {&p};

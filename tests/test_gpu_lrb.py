@@ -14,9 +14,9 @@ from tests.test_gpu_parity import _small
 pytestmark = pytest.mark.gpu
 
 
-def run_lrb(w, rank, steps, tiles=None, mode=None, v_scale=None):
+def run_lrb(w, rank, steps, tiles=None, mode=None, v_scale=None, pm=None):
     mode = w.mode if mode is None else mode
-    pm = P.prec_map_for(w)
+    pm = P.prec_map_for(w) if pm is None else pm
     if tiles == "sample":
         tiles = P.sample_tiles(w, pm)
     pair = P.Pair(w, pm, tiles=tiles, mode=mode)
@@ -94,7 +94,21 @@ def test_lrb_many_tiles_per_cta_sampled():
     run_lrb(w, rank=4, steps=5, tiles="sample")
 
 
-def test_lrb_rejects_bad_rank_and_group_widths():
+@pytest.mark.parametrize("rank", [4, 6])
+@pytest.mark.parametrize("fam,mode", [("gla", I.ROUND_RTN), ("gla", I.ROUND_BDR),
+                                      ("gdn", I.ROUND_SR), ("mamba2", I.ROUND_SR)])
+def test_lrb_group_widths(fam, mode, rank):
+    """One width per (head, scale group): both bypass kernels (rank 4
+    streaming, rank 6 one CTA per tile) against the oracle's per-group entry,
+    through a merge."""
+    d_v = 64 if fam == "mamba2" else 128
+    w = _small(fam, 2, 5, 128, d_v, 32, mode, "mixed", steps=rank + 2)
+    rng = np.random.default_rng(rank + 3 * mode)
+    pm = rng.choice(np.array([4, 8], np.uint8), size=(w.heads, w.d_k // w.group))
+    run_lrb(w, rank=rank, steps=rank + 2, pm=pm)
+
+
+def test_lrb_rejects_bad_rank():
     w = _small("gla", 1, 2, 128, 128, 32, I.ROUND_RTN, "int8", steps=1)
     e = torch.zeros(1 << 16, device="cuda")
     st = lrs.lrs_state_alloc(P.make_shape(w), np.full(2, 8, np.uint8))
@@ -104,14 +118,6 @@ def test_lrb_rejects_bad_rank_and_group_widths():
                 lrs.lrs_lrb_step(st, st.state_codes, st.scales, st.prec_map, r, e, e, e, e, e, e,
                                  None, e, 0, 0, 0)
             assert ei.value.status == lrs.LRS_ERR_INVALID_ARG
-    finally:
-        lrs.lrs_state_free(st)
-    st = lrs.lrs_state_alloc(P.make_shape(w), np.full((2, 4), 8, np.uint8))
-    try:
-        with pytest.raises(lrs.LrsError) as ei:
-            lrs.lrs_lrb_step(st, st.state_codes, st.scales, st.prec_map, 2, e, e, e, e, e, e,
-                             None, e, 0, 0, 0)
-        assert ei.value.status == lrs.LRS_ERR_UNSUPPORTED
     finally:
         lrs.lrs_state_free(st)
 
