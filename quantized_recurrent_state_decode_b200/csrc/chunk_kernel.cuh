@@ -325,11 +325,9 @@ __global__ void __launch_bounds__(DV, (3 * 128) / DV) chunk_kernel(const ChunkPa
                 good = good && mbar_wait_bounded(&bar_tok[nslot],
                                                  static_cast<uint32_t>(((u + 1) / NS) & 1),
                                                  p.timeout_ns);
-            if (__syncthreads_or(!good)) {
-                ok = false;
-                drain_lo = u;
-                break;
-            }
+            // A thread whose wait ran out skips the token; the one CTA barrier
+            // of the iteration (below) ends the loop for all.
+            if (good) {
             const uint8_t* tk = smem + S::kRing + slot * S::kTok;
             const float* tq = reinterpret_cast<const float*>(tk + S::kQ);
             const float* tkk = reinterpret_cast<const float*>(tk + S::kK);
@@ -382,7 +380,13 @@ __global__ void __launch_bounds__(DV, (3 * 128) / DV) chunk_kernel(const ChunkPa
             }
             unext = un;
             p.out[row * DV + j] = o;
-            __syncthreads();                 // every thread is done with the slot
+            }
+            // every thread is done with the slot; any wait that ran out
+            if (__syncthreads_or(!good)) {
+                ok = false;
+                drain_lo = u;
+                break;
+            }
             if (j == 0 && t + NS < T) {
                 fence_proxy_async_smem();
                 issue_token<DK, DV, GROUP, GATE>(p, smem, slot, tile, t + NS);
