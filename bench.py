@@ -133,73 +133,112 @@ class ClockSampler:
 
 # --------------------------------------------------------------- reference ---
 
-def run_reference(args, w):
-    """The CPU oracle on the host cores: each step runs a bounded sample of
-    tiles, and the metric is scaled to the whole workload."""
-    import numpy as np
-    import oracle
-    from quantized_recurrent_state_decode_b200 import inputs as I
+class OracleSampler:
+    """The CPU oracle on the host cores over a fixed, seeded sample of tiles of
+    the workload. A pool of one thread per core is created once; each step
+    hands every thread one contiguous slice of the sample (the oracle's C code
+    runs single-threaded per call, outside the interpreter lock). Both CPU
+    legs of the benchmark -- `--impl reference` and the GPU arm's
+    `cpu_baseline` -- time through this one sampler, so they report one
+    number for one workload."""
 
-    nthreads = oracle.default_threads()
-    mode = MODES[args.mode] if args.mode else w.mode
-    pm = oracle_precision_map(w)
-    # calibrate: time per tile with all threads
-    ntiles_all = w.batch * w.heads
-    rng = np.random.default_rng(0)
-    per_step = max(nthreads, 8)
-    tiles = rng.choice(ntiles_all, size=per_step, replace=False)
-    tb = (tiles // w.heads).astype(np.int32)
-    th = (tiles % w.heads).astype(np.int32)
-    S0 = I.initial_state(w)[tb, th].numpy()
-    codes, scales = oracle.import_fp32(S0, pm, th, group=w.group)
-    x0 = I.step_inputs(w, 0)
-    sel = {n: (None if v is None else v[tb, th].numpy().reshape(len(tiles), -1))
-           for n, v in x0.items()}
+    def __init__(self, w, mode, ntiles=None, seed=0):
+        import concurrent.futures as cf
+        import numpy as np
+        import oracle
+        from quantized_recurrent_state_decode_b200 import inputs as I
+        self.w, self.mode = w, mode
+        self.nthreads = oracle.default_threads()
+        n_all = w.batch * w.heads
+        n = ntiles if ntiles else max(self.nthreads * 16, 256)
+        n = min(n_all, n)
+        rng = np.random.default_rng(seed)
+        tiles = np.sort(rng.choice(n_all, size=n, replace=False))
+        self.tb = (tiles // w.heads).astype(np.int32)
+        self.th = (tiles % w.heads).astype(np.int32)
+        self.n, self.n_all = n, n_all
+        self.pm = oracle_precision_map(w)
+        S0 = I.initial_state(w)[self.tb, self.th].numpy()
+        self.codes, self.scales = oracle.import_fp32(S0, self.pm, self.th, group=w.group)
+        self.xs = []
+        for t in range(4):
+            x = I.step_inputs(w, t)
+            self.xs.append({k: (None if v is None else v[self.tb, self.th].numpy().reshape(n, -1))
+                            for k, v in x.items()})
+        T = self.nthreads
+        self.slices = [slice(n * i // T, n * (i + 1) // T) for i in range(T)]
+        self.slices = [sl for sl in self.slices if sl.stop > sl.start]
+        self.pool = cf.ThreadPoolExecutor(len(self.slices))
 
-    def one(t):
+    def _part(self, sl, x, t):
+        import numpy as np
+        import oracle
+        w = self.w
+        codes, scales = self.codes[sl], self.scales[sl]      # contiguous views, updated in place
+        sel = {k: (None if v is None else v[sl]) for k, v in x.items()}
         oracle.step(codes, scales, sel["q"], sel["k"], sel["v"], sel["gates"],
-                    None if sel["beta"] is None else sel["beta"].reshape(-1), pm, tb, th,
-                    group=w.group, update_kind=w.update_kind, gate_kind=w.gate_kind, mode=mode,
-                    seed=1, step=t, nthreads=nthreads)
+                    None if sel["beta"] is None else sel["beta"].reshape(-1), self.pm,
+                    self.tb[sl], self.th[sl], group=w.group, update_kind=w.update_kind,
+                    gate_kind=w.gate_kind, mode=self.mode, seed=1, step=t, nthreads=1)
 
-    t0 = time.perf_counter()
-    one(0)
-    t_sample = time.perf_counter() - t0
-    budget = 120.0
-    reps = max(1, int(budget / max(t_sample, 1e-6) / max(args.steps + args.warmup, 1)))
-    reps = min(reps, 64)
+    def step(self, t):
+        """One step over the sample; returns its wall time in seconds."""
+        x = self.xs[t % len(self.xs)]
+        t0 = time.perf_counter()
+        list(self.pool.map(lambda sl: self._part(sl, x, t), self.slices))
+        return time.perf_counter() - t0
+
+    def steps_per_s(self, sec_per_sample_step):
+        """Whole-workload steps/s from the time of one step over the sample."""
+        return 1.0 / (sec_per_sample_step / self.n * self.n_all)
+
+    def describe(self, steps, el):
+        return ("%d of %d tiles per step (seeded sample), %d steps, %.1f s of oracle time on "
+                "%d threads created once, scaled to the whole workload"
+                % (self.n, self.n_all, steps, el, len(self.slices)))
+
+    def close(self):
+        self.pool.shutdown()
+
+
+def run_reference(args, w):
+    """The CPU oracle on the host cores: W untimed and K timed steps, each one
+    step over the seeded tile sample; the metric is scaled to the workload."""
+    mode = MODES[args.mode] if args.mode else w.mode
+    smp = OracleSampler(w, mode)
+    # a bounded sample: at most ~150 s for the whole run
+    t1 = smp.step(0)
+    reps = max(1, min(16, int(150.0 / max(t1, 1e-3) / max(args.steps + args.warmup, 1))))
     for t in range(args.warmup):
         for _ in range(reps):
-            one(t)
-    t0 = time.perf_counter()
+            smp.step(t)
+    el = 0.0
     for t in range(args.steps):
         for _ in range(reps):
-            one(t)
-    el = time.perf_counter() - t0
-    sec_per_tile = el / (args.steps * reps * len(tiles))
-    sec_per_step = sec_per_tile * ntiles_all
-    steps_per_s = 1.0 / sec_per_step
-    sample = ("%d of %d tiles x %d repeats per step, %d threads, extrapolated to the whole "
-              "workload" % (len(tiles), ntiles_all, reps, nthreads))
+            el += smp.step(t)
+    smp.close()
+    steps_per_s = smp.steps_per_s(el / (args.steps * reps))
     line = {"metric": METRIC, "impl": "reference", "value": steps_per_s, "unit": "steps/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": sec_per_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": 1e3 / steps_per_s, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": config_of(w, mode, args.layers, args.gpus),
-            "cpu_baseline": {"value": steps_per_s, "unit": "steps/s", "cores": nthreads,
-                             "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": steps_per_s, "unit": "steps/s", "cores": len(smp.slices),
+                             "kind": "oracle",
+                             "sample": smp.describe(args.steps * reps, el)},
             "e2e": {"value": steps_per_s, "unit": "steps/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
 
 
 def oracle_precision_map(w):
+    """The decay-ranked map of a mixed workload from the whole run's gates."""
     import oracle
     from quantized_recurrent_state_decode_b200 import inputs as I
     pm = I.uniform_prec_map(w)
     if pm is not None:
         return pm.numpy()
-    decay = I.decay_tensor(w, steps=min(w.steps, 16))
+    decay = I.decay_tensor(w)
     return oracle.precision_map(oracle.decay_means(decay.numpy()), I.n_int8_heads(w))
 
 
@@ -219,14 +258,14 @@ def config_of(w, mode, layers, n):
 
 def precision_map(w, lrs, dev):
     """Per-head precision: uniform for int8/int4 workloads; for mixed ones,
-    the library's mean decay per head over the first steps' gates, ranked."""
+    the library's mean decay per head over the whole run's gates, ranked."""
     import numpy as np
     import torch
     from quantized_recurrent_state_decode_b200 import inputs as I
     pm = I.uniform_prec_map(w)
     if pm is not None:
         return pm.numpy()
-    decay = I.decay_tensor(w, steps=min(w.steps, 16), device=dev)
+    decay = I.decay_tensor(w, device=dev)
     outer, H, inner = decay.shape
     means = torch.zeros(H, dtype=torch.float64, device=dev)
     lrs.lrs_decay_head_means(decay, outer, H, inner, means)
@@ -332,8 +371,11 @@ def run_gpu(args, w):
     achieved = bytes_step / launch_s / 1e9
     peak, peak_kind = measured_peaks()
 
-    # end to end: host inputs in pinned memory, copies inside the timed region
-    e2e_steps = min(args.steps, 256)
+    # end to end: host inputs in pinned memory, copies inside the timed region,
+    # over at least 256 steps whatever --steps is (the host step overlaps
+    # consecutive calls through two staging buffers: it needs a long run to
+    # reach its steady state)
+    e2e_steps = max(256, min(args.steps, 1024))
     xh = [{n: (None if v is None else v.cpu().pin_memory()) for n, v in x.items()} for x in xs]
     out_h = torch.empty(nb, w.heads, w.d_v).pin_memory()
     st0 = states[0]
@@ -359,6 +401,8 @@ def run_gpu(args, w):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), device=dev)
     h2d = sum(v.numel() * 4 for v in xh[0].values() if v is not None)
     d2h = out_h.numel() * 4
+    pinned = pinned_copy_rates(h2d, d2h, dev, stream)
+    e2e_sps = world * e2e_steps / (e2e_ms / 1e3)
 
     extras = {}
     if not args.no_extras and rank == 0:
@@ -367,6 +411,8 @@ def run_gpu(args, w):
 
     for st in states:
         lrs.lrs_state_free(st)
+    if args.configs and rank == 0:
+        extras["configs"] = run_configs(dev, stream)
     if not args.no_extras and rank == 0 and args.drift_steps > 0:
         extras["drift"] = run_drift(dev, stream, args.drift_steps)
     if world > 1:
@@ -390,8 +436,10 @@ def run_gpu(args, w):
                          w.d_v // 32, w.group, "delta" if w.update_kind else "gated",
                          "per_key" if w.gate_kind else "scalar",
                          {0: "rtn", 1: "sr", 2: "bdr"}[mode])},
-        "e2e": {"value": world * e2e_steps / (e2e_ms / 1e3), "unit": "steps/s",
+        "e2e": {"value": e2e_sps, "unit": "steps/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "h2d_gbs_achieved": e2e_sps / world * h2d / 1e9,
+                "pinned_copy_gbs_measured": pinned,
                 "api": "lrs_decode_step_host"},
         "gpu_launches": args.steps,
         "clocks": clocks,
@@ -400,6 +448,29 @@ def run_gpu(args, w):
     if args.cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, mode)
     print(json.dumps(line))
+
+
+def pinned_copy_rates(h2d, d2h, dev, stream, reps=32):
+    """Plain pinned-host <-> device copy rates at the step's own sizes (one
+    host-to-device copy of h2d bytes, one device-to-host copy of d2h bytes),
+    the ceiling of the host-buffer step's copies."""
+    import torch
+    hs = torch.empty(h2d // 4).pin_memory()
+    ds = torch.empty(h2d // 4, device=dev)
+    ho = torch.empty(d2h // 4).pin_memory()
+    do = torch.empty(d2h // 4, device=dev)
+    res = {}
+    with torch.cuda.stream(stream):
+        for name, dst, src, nbytes in (("h2d", ds, hs, h2d), ("d2h", ho, do, d2h)):
+            dst.copy_(src, non_blocking=True)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                dst.copy_(src, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            res[name] = nbytes * reps / (e0.elapsed_time(e1) / 1e3) / 1e9
+    return res
 
 
 def _capture_on(stream, n, pick, lrs, out, seed, mode):
@@ -502,6 +573,110 @@ def run_extras(args, w, wl, states, xs, out, seed, stream, L, NI, mode, dev, pm)
                                 "state_gbs": fb / (ms / 1e3) / 1e9, "bytes_per_step": fb}
     del g, Ss
     return res
+
+
+# The five synthetic workloads the step is specified on, each in its stated
+# rounding mode(s): (label, workload, batch override, modes).
+CONFIG_RUNS = [
+    ("C1", "gla_rtn_int8_b2h2_64", None, ("rtn",)),
+    ("C2", "gdn_sr_int8_b64h16_128", None, ("sr",)),
+    ("C3", "mamba2_mixed_sr_b128h64", None, ("sr",)),
+    ("C4", "gla_bdr_int4_b256h32_128", None, ("bdr", "rtn")),
+    ("C5", "gdn_mixed_sr_h32_128", 64, ("sr",)),
+    ("C5", "gdn_mixed_sr_h32_128", 256, ("sr",)),
+    ("C5", "gdn_mixed_sr_h32_128", 1024, ("sr",)),
+]
+L2_BYTES = 126 * 2**20
+
+
+def _time_graph(stream, n, launch):
+    """Device time per launch of n launches captured in one CUDA graph
+    (eager warm-up launches first, one untimed replay)."""
+    import torch
+    for i in range(3):
+        launch(i)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            launch(i)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    del g
+    return ms
+
+
+def run_configs(dev, stream, n=64):
+    """Every specified workload in its rounding mode(s): the quantized step and
+    the fp32-state kernel on the same inputs, each over layer states rotated so
+    that their total is at least 4x the L2 (one state at most where a single
+    state already exceeds that; the tiny first workload stays in L2)."""
+    import torch
+    from quantized_recurrent_state_decode_b200 import inputs as I
+    from quantized_recurrent_state_decode_b200 import lrs
+    peak, peak_kind = measured_peaks()
+    rows = []
+    for label, name, batch, modes in CONFIG_RUNS:
+        w = I.WORKLOADS[name]
+        if batch:
+            w = w.with_batch(batch)
+        pm = precision_map(w, lrs, dev)
+        shp = lrs.shape(w.batch, w.heads, w.d_k, w.d_v, w.group, w.update_kind, w.gate_kind)
+        sb = state_bytes(w, pm)
+        L = max(1, min(64, -(-4 * L2_BYTES // (sb // 2))))
+        states = [lrs.lrs_state_alloc(shp, pm) for _ in range(L)]
+        S0 = I.initial_state(w, device=dev)
+        for st in states:
+            lrs.lrs_state_import_fp32(st, S0)
+        NI = 8
+        xs = [I.step_inputs(w, t, device=dev) for t in range(NI)]
+        out = torch.empty(w.batch, w.heads, w.d_v, device=dev)
+        seed = I.sr_seed(w)
+        fb = w.batch * w.heads * w.d_k * w.d_v * 4 * 2          # fp32 state read + written
+        Lf = max(1, min(16, -(-4 * L2_BYTES // (fb // 2))))
+        Ss = [S0.clone() for _ in range(Lf)]
+        del S0
+        with torch.cuda.stream(stream):
+            def f32(i):
+                x = xs[i % NI]
+                lrs.lrs_fp32_decode_step(shp, Ss[i % Lf], x["q"], x["k"], x["v"], x["gates"],
+                                         x["beta"], out, stream)
+            ms_f = _time_graph(stream, n, f32)
+            for mname in modes:
+                m = MODES[mname]
+
+                def step(i, m=m):
+                    st, x = states[i % L], xs[i % NI]
+                    lrs.lrs_decode_step(st, st.state_codes, st.scales, st.prec_map, x["q"],
+                                        x["k"], x["v"], x["gates"], x["beta"], out, seed, i, m,
+                                        stream)
+                ms = _time_graph(stream, n, step)
+                lrs.lrs_sync(stream)
+                gbs = sb / (ms / 1e3) / 1e9
+                rows.append({
+                    "config": label, "workload": w.name, "family": w.family, "batch": w.batch,
+                    "heads": w.heads, "d_k": w.d_k, "d_v": w.d_v, "group": w.group,
+                    "state": w.precision, "rounding": mname,
+                    "us_per_step": ms * 1e3, "steps_per_s": 1e3 / ms,
+                    "state_bytes_per_step": sb, "state_gbs": gbs, "hbm_frac": gbs / peak,
+                    "layers_rotated": L,
+                    "fp32_state_kernel": {"us_per_step": ms_f * 1e3, "bytes_per_step": fb,
+                                          "state_gbs": fb / (ms_f / 1e3) / 1e9,
+                                          "hbm_frac": fb / (ms_f / 1e3) / 1e9 / peak,
+                                          "layers_rotated": Lf},
+                    "speedup_vs_fp32_state": ms_f / ms})
+        for st in states:
+            lrs.lrs_state_free(st)
+        del Ss, xs, out
+        torch.cuda.empty_cache()
+    return {"peak_gbs": peak, "peak_kind": peak_kind, "timed_launches": n,
+            "timing": "CUDA events around a graph of %d launches; state bytes = codes + "
+                      "scales read and written once" % n, "runs": rows}
 
 
 FP32_LANES_PER_SM = 128      # fp32 fused multiply-add lanes per SM (sm_100)
@@ -683,39 +858,17 @@ def _sm_max_mhz():
 
 
 def cpu_baseline(w, mode):
-    """The oracle on the host cores, a bounded sample of tiles for ~10-20 s."""
-    import numpy as np
-    import oracle
-    from quantized_recurrent_state_decode_b200 import inputs as I
-    nthreads = oracle.default_threads()
-    ntiles_all = w.batch * w.heads
-    n = min(ntiles_all, max(nthreads * 16, 256))
-    rng = np.random.default_rng(1)
-    tiles = np.sort(rng.choice(ntiles_all, size=n, replace=False))
-    tb = (tiles // w.heads).astype(np.int32)
-    th = (tiles % w.heads).astype(np.int32)
-    pm = oracle_precision_map(w)
-    S0 = I.initial_state(w)[tb, th].numpy()
-    codes, scales = oracle.import_fp32(S0, pm, th, group=w.group)
-    xs = []
-    for t in range(4):
-        x = I.step_inputs(w, t)
-        xs.append({k: (None if v is None else v[tb, th].numpy().reshape(n, -1))
-                   for k, v in x.items()})
-    reps, el = 0, 0.0
-    while el < 12.0 or reps == 0:
-        sel = xs[reps % len(xs)]
-        t0 = time.perf_counter()
-        oracle.step(codes, scales, sel["q"], sel["k"], sel["v"], sel["gates"],
-                    None if sel["beta"] is None else sel["beta"].reshape(-1), pm, tb, th,
-                    group=w.group, update_kind=w.update_kind, gate_kind=w.gate_kind, mode=mode,
-                    seed=1, step=reps, nthreads=nthreads)
-        el += time.perf_counter() - t0
-        reps += 1
-    sec_step = el / reps / n * ntiles_all
-    return {"value": 1.0 / sec_step, "unit": "steps/s", "cores": nthreads, "kind": "oracle",
-            "sample": "%d of %d tiles for %d steps (%.1f s of oracle time), scaled to the whole "
-                      "workload" % (n, ntiles_all, reps, el)}
+    """The oracle on the host cores, the same sampler as `--impl reference`,
+    for about 12 s of oracle time."""
+    smp = OracleSampler(w, mode)
+    smp.step(0)
+    el, steps = 0.0, 0
+    while el < 12.0:
+        el += smp.step(steps)
+        steps += 1
+    smp.close()
+    return {"value": smp.steps_per_s(el / steps), "unit": "steps/s", "cores": len(smp.slices),
+            "kind": "oracle", "sample": smp.describe(steps, el)}
 
 
 def main():
@@ -732,6 +885,8 @@ def main():
     ap.add_argument("--drift-steps", type=int, default=1024,
                     help="steps of the int4 output-drift series (0: skip it)")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-configs", dest="configs", action="store_false",
+                    help="skip the per-workload table (the `configs` key)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -264,20 +264,25 @@ lrs_status lrs_decode_step_host(const lrs_state *st, const float *q_host, const 
                                 uint64_t step, int32_t mode, void *stream);
 
 /* lrs_decode_step_host without any device allocation. This entry point has no
- * counterpart in the method's sources; it exists for callers that cannot
- * allocate device memory at the time they step: code running while a stream
- * is captured into a CUDA graph (where cudaMalloc is not allowed), and
- * processes whose device memory belongs to another allocator or a fixed pool.
- * Its scratch -- a device error word and the staging of q, k, v, gates, beta
- * and out -- is a 32 MiB array inside the library's image, which every GPU
- * that loads the library holds until the process exits. It calls no
- * cudaMalloc, cudaFree or other allocating routine.
+ * counterpart in the method's sources. It is for callers that must not
+ * allocate device memory when they step: a process whose device memory is
+ * owned by another allocator or by a fixed pool sized at start-up (an
+ * allocation behind its back can fail for lack of room, or break the pool's
+ * accounting), and code on a latency-critical path that must not pay for a
+ * cudaMalloc, which can synchronize the device. Its scratch -- a device error
+ * word and the staging of q, k, v, gates, beta and out -- is a 32 MiB array
+ * inside the library's image. Each device takes those 32 MiB when the
+ * library's device code is loaded there: at the latest on this entry point's
+ * first call on that device (CUDA loads modules lazily by default), and they
+ * stay taken until the process exits. It calls no cudaMalloc, cudaFree or
+ * other allocating routine.
  *   - Limit: the staging must fit: 256 + 16-byte-padded sizes of q, k
  *     ([B][H][d_k]), v, out ([B][H][d_v]), gates and beta must not exceed
  *     32 MiB; a larger step is rejected with LRS_ERR_UNSUPPORTED and nothing
  *     is launched. (B=256, H=32, 128x128 with per-key gates needs 20 MiB.)
- *   - The first call on a device looks up the array's device address; make
- *     it before any stream capture on that device.
+ *   - The first call on a device looks up the array's device address (and
+ *     may load the library's device code there, taking the 32 MiB): make one
+ *     call on each device before sizing a fixed pool from the free memory.
  *   - Every call shares the one array, which keeps the last call's contents:
  *     calls that overlap on the GPU (other streams, other threads) race and
  *     corrupt each other's inputs and outputs. Serialize them.
@@ -286,7 +291,8 @@ lrs_status lrs_decode_step_host(const lrs_state *st, const float *q_host, const 
  *     wait timed out, bit 1 = the precision map did not fit the layout. The
  *     word is cleared at the start of each call; lrs_sync does not see it.
  * Arguments otherwise as lrs_decode_step_host (the state's own buffers are
- * stepped; host buffers pinned for asynchronous copies). */
+ * stepped; host buffers pinned for asynchronous copies); the launch is the
+ * same as lrs_decode_step's. */
 lrs_status lrs_decode_step_host_noalloc(const lrs_state *st, const float *q_host,
                                         const float *k_host, const float *v_host,
                                         const float *gates_host, const float *beta_host,
@@ -337,7 +343,18 @@ lrs_status lrs_precision_map(int32_t heads, const double *means_host, int32_t n_
                              uint8_t *prec_map_host);
 
 /* Wait for stream, then return and clear the first error recorded on the
- * device by this library's kernels (LRS_ERR_DEVICE_*), or LRS_OK. */
+ * device by this library's kernels (LRS_ERR_DEVICE_*), or LRS_OK.
+ *
+ * State after a device timeout. A kernel records LRS_ERR_DEVICE_TIMEOUT when
+ * a wait for its own copies runs out (2 s in normal operation: far above any
+ * legitimate wait; it means the device stalled). The kernel then stops: tiles
+ * it had not reached keep their old codes and scales, tiles it finished hold
+ * the new ones, and the tile it was working on may hold new codes and scales
+ * in its first scale groups and old ones in the rest (the delta rule reads a
+ * whole tile before writing it, so there a tile is either old or new; the
+ * gated forms write each group as they go). The step's outputs are not
+ * valid. The state as a whole is therefore neither the old nor the new state:
+ * restore it from a checkpoint (lrs_state_copy_raw) before stepping again. */
 lrs_status lrs_sync(void *stream);
 
 /* Fault injection for tests of the error path: when enabled (nonzero), the
@@ -345,6 +362,15 @@ lrs_status lrs_sync(void *stream);
  * timeout_us microseconds, so the kernel records LRS_ERR_DEVICE_TIMEOUT and
  * returns without touching the state. Disarms itself after that launch. */
 lrs_status lrs_debug_inject_timeout(int32_t enable, int32_t timeout_us);
+
+/* The same with a later wait running out: the next lrs_decode_step (or
+ * lrs_decode_step_bf16) copies in only the first items_copied (tile, scale
+ * group) items of each warp of its launch, and the wait for the next item
+ * runs out after timeout_us microseconds. items_copied < 0 disarms. With the
+ * gated update a warp's first tile may then be left part-way: its first
+ * items_copied groups hold the new codes and scales, the rest the old ones
+ * (see "State after a device timeout" at lrs_sync). */
+lrs_status lrs_debug_inject_timeout_after(int32_t items_copied, int32_t timeout_us);
 
 /* Message of the last error returned on this thread ("" if none). */
 const char *lrs_last_error(void);

@@ -75,28 +75,17 @@ lrs_status device_ctx(DeviceCtx** out) {
     return LRS_OK;
 }
 
-// Fault injection (tests of the error path only).
+// Fault injection (tests of the error path only): the next step launch
+// issues copies for only its first g_inject_items items per warp (0: none)
+// and gives its waits g_inject_timeout_ns.
 std::mutex g_inject_mu;
 bool g_inject = false;
+int32_t g_inject_items = 0;
 uint64_t g_inject_timeout_ns = 0;
 
-// Launch shape of the step kernel: warps per CTA and ring slots per warp
-// (0 = the defaults below). LRS_STEP_WARPS / LRS_STEP_SLOTS override them
-// for launch-shape sweeps.
-int env_int(const char* name) {
-    const char* s = getenv(name);
-    return s ? atoi(s) : 0;
-}
-int step_warps_override() {
-    static int v = env_int("LRS_STEP_WARPS");
-    return v;
-}
-int step_slots_override() {
-    static int v = env_int("LRS_STEP_SLOTS");
-    return v;
-}
 constexpr int kDefaultWarps = 12;
 constexpr int kDefaultSlots = 2;
+constexpr int kSmemLimit = 227 * 1024;
 
 struct StatePriv {
     int device = -1;
@@ -247,6 +236,57 @@ int step_warp_smem(int C, int group, int update_kind, int gate_kind, int slots, 
 #undef LRS_SLOT
 #undef LRS_SLOT_IO
     return -1;
+}
+
+// One launch shape per (kernel, device), prepared on its first use: the
+// dynamic shared-memory limit raised once (the attribute belongs to the
+// function and is never lowered again) and the CTAs that fit on an SM.
+lrs_status step_launch_shape(const lrs_shape& sh, int mode, int io, int device, int sms,
+                             StepLaunch* out) {
+    const int C = sh.d_v / 32, G = sh.d_k / sh.group;
+    const void* fn = find_step_kernel(C, sh.group, sh.update_kind, sh.gate_kind, mode, io);
+    if (!fn) return fail(LRS_ERR_UNSUPPORTED, "no compiled kernel for this shape and mode");
+    // ring slots per warp: the delta rule keeps a whole tile resident; the
+    // gated forms stream a few groups ahead (at most G, so that the single v
+    // buffer is never overwritten before it is read)
+    int slots = sh.update_kind == LRS_UPDATE_DELTA ? G : std::min(kDefaultSlots, G);
+    slots = std::max(1, std::min(slots, kMaxSlots));
+    const int warp_smem = step_warp_smem(C, sh.group, sh.update_kind, sh.gate_kind, slots, mode,
+                                         io, sh.d_k);
+    if (warp_smem <= 0) return fail(LRS_ERR_UNSUPPORTED, "no shared-memory layout for this shape");
+    int warps = std::min(kDefaultWarps, std::max(1, kSmemLimit / warp_smem));
+    warps = std::min(warps, step_max_warps(sh.group, mode, sh.update_kind));
+    const int smem = warps * warp_smem;
+
+    struct Prepared { const void* fn; int dev; int smem; int per_sm; };
+    static std::mutex mu;
+    static std::vector<Prepared> prepared;
+    int per_sm = 0;
+    std::lock_guard<std::mutex> lk(mu);
+    bool attr = false;
+    for (const Prepared& c : prepared) {
+        if (c.fn != fn || c.dev != device) continue;
+        attr = true;
+        if (c.smem == smem) per_sm = c.per_sm;
+    }
+    if (per_sm == 0) {
+        cudaError_t e = cudaSuccess;
+        if (!attr)
+            e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return cuda_fail(e, "cudaFuncSetAttribute");
+        }
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, warps * 32, smem);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+        }
+        if (per_sm < 1) return fail(LRS_ERR_UNSUPPORTED, "step kernel does not fit on an SM");
+        prepared.push_back({fn, device, smem, per_sm});
+    }
+    *out = {fn, slots, warps, warp_smem, smem, sms * per_sm};
+    return LRS_OK;
 }
 
 }  // namespace lrs
@@ -412,72 +452,18 @@ static lrs_status decode_step_io(const lrs_state* st, void* state_codes, float* 
     if (sh.update_kind == LRS_UPDATE_DELTA) LRS_REQUIRE_PTR(beta);
     if (mode != LRS_ROUND_RTN && mode != LRS_ROUND_SR && mode != LRS_ROUND_BDR)
         return fail(LRS_ERR_INVALID_ARG, "mode %d", mode);
-    const int C = sh.d_v / 32, G = sh.d_k / sh.group;
-    const void* fn = lrs::find_step_kernel(C, sh.group, sh.update_kind, sh.gate_kind, mode, io);
-    if (!fn) return fail(LRS_ERR_UNSUPPORTED, "no compiled kernel for this shape and mode");
+    const int G = sh.d_k / sh.group;
     DeviceCtx* ctx = nullptr;
     s = device_ctx(&ctx);
     if (s != LRS_OK) return s;
     const int ntiles = sh.batch * sh.heads;
     if (ntiles == 0) return ok();
 
-    // ring slots per warp: the delta rule keeps a whole tile resident; the
-    // gated forms stream a few groups ahead (at most G, so that the single v
-    // buffer is never overwritten before it is read)
-    int slots = G;
-    if (sh.update_kind != LRS_UPDATE_DELTA) {
-        slots = step_slots_override() > 0 ? step_slots_override() : kDefaultSlots;
-        slots = std::min(slots, G);
-    }
-    slots = std::max(1, std::min(slots, lrs::kMaxSlots));
-    const int warp_smem = lrs::step_warp_smem(C, sh.group, sh.update_kind, sh.gate_kind, slots, mode, io,
-                                              sh.d_k);
-    constexpr int kSmemLimit = 227 * 1024;
-    int warps = step_warps_override();
-    if (warps <= 0) warps = kDefaultWarps;
-    warps = std::min(warps, std::max(1, kSmemLimit / warp_smem));
-    warps = std::min(warps, lrs::step_max_warps(sh.group, mode, sh.update_kind));
-    const int smem = warps * warp_smem;
-
-    // Per kernel and device, raise the dynamic shared memory limit once to the
-    // largest launch can ask for (the attribute belongs to the function, so it
-    // is never lowered again); per launch shape, record how many CTAs fit.
-    static std::mutex mu;
-    struct Prepared { const void* fn; int dev; };
-    struct Occupancy { const void* fn; int dev; int smem; int threads; int per_sm; };
-    static std::vector<Prepared> prepared;
-    static std::vector<Occupancy> occupancy;
-    int per_sm = 0;
-    {
-        std::lock_guard<std::mutex> lk(mu);
-        const int dev = static_cast<const StatePriv*>(st->priv)->device;
-        bool ready = false;
-        for (const Prepared& c : prepared) ready = ready || (c.fn == fn && c.dev == dev);
-        if (!ready) {
-            cudaError_t e =
-                cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
-            if (e != cudaSuccess) {
-                cudaGetLastError();
-                return cuda_fail(e, "cudaFuncSetAttribute");
-            }
-            prepared.push_back({fn, dev});
-        }
-        for (const Occupancy& c : occupancy)
-            if (c.fn == fn && c.dev == dev && c.smem == smem && c.threads == warps * 32)
-                per_sm = c.per_sm;
-        if (per_sm == 0) {
-            cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, warps * 32, smem);
-            if (e != cudaSuccess) {
-                cudaGetLastError();
-                return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
-            }
-            if (per_sm < 1) return fail(LRS_ERR_UNSUPPORTED, "step kernel does not fit on an SM");
-            occupancy.push_back({fn, dev, smem, warps * 32, per_sm});
-        }
-    }
-    int grid = ctx->sms * per_sm;
-    grid = std::min(grid, (ntiles + warps - 1) / warps);
-
+    lrs::StepLaunch ls;
+    s = lrs::step_launch_shape(sh, mode, io, static_cast<const StatePriv*>(st->priv)->device,
+                               ctx->sms, &ls);
+    if (s != LRS_OK) return s;
+    const int grid = std::min(ls.grid, (ntiles + ls.warps - 1) / ls.warps);
     lrs::StepParams p;
     p.codes = static_cast<uint8_t*>(state_codes);
     p.scales = scales;
@@ -499,19 +485,19 @@ static lrs_status decode_step_io(const lrs_state* st, void* state_codes, float* 
     p.G = G;
     p.ntiles = ntiles;
     p.pgroups = static_cast<const StatePriv*>(st->priv)->pgroups;
-    p.warp_smem = warp_smem;
-    p.slots = slots;
+    p.warp_smem = ls.warp_smem;
+    p.slots = ls.slots;
     p.inject = 0;
     {
         std::lock_guard<std::mutex> lk(g_inject_mu);
         if (g_inject) {
-            p.inject = 1;
+            p.inject = 1 + g_inject_items;
             p.timeout_ns = g_inject_timeout_ns;
             g_inject = false;
         }
     }
     void* args[] = {&p};
-    cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(warps * 32), args, smem,
+    cudaError_t e = cudaLaunchKernel(ls.fn, dim3(grid), dim3(ls.warps * 32), args, ls.smem,
                                      static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {
         cudaGetLastError();  // a failed launch must not surface again in a later call
@@ -763,9 +749,15 @@ lrs_status lrs_sync(void* stream) {
 }
 
 lrs_status lrs_debug_inject_timeout(int32_t enable, int32_t timeout_us) {
-    if (enable && timeout_us < 1) return fail(LRS_ERR_INVALID_ARG, "timeout_us=%d", timeout_us);
+    return lrs_debug_inject_timeout_after(enable ? 0 : -1, timeout_us);
+}
+
+lrs_status lrs_debug_inject_timeout_after(int32_t items_copied, int32_t timeout_us) {
+    if (items_copied >= 0 && timeout_us < 1)
+        return fail(LRS_ERR_INVALID_ARG, "timeout_us=%d", timeout_us);
     std::lock_guard<std::mutex> lk(g_inject_mu);
-    g_inject = enable != 0;
+    g_inject = items_copied >= 0;
+    g_inject_items = items_copied < 0 ? 0 : items_copied;
     g_inject_timeout_ns = static_cast<uint64_t>(timeout_us) * 1000ull;
     return ok();
 }
@@ -791,6 +783,19 @@ bool take_injected_timeout(uint64_t* timeout_ns) {
     g_inject = false;
     *timeout_ns = g_inject_timeout_ns;
     return true;
+}
+
+int sm_count(int device) {
+    static std::mutex mu;
+    static int sms[kMaxDevices];
+    if (device < 0 || device >= kMaxDevices) return 0;
+    std::lock_guard<std::mutex> lk(mu);
+    if (sms[device] == 0 &&
+        cudaDeviceGetAttribute(&sms[device], cudaDevAttrMultiProcessorCount, device) != cudaSuccess) {
+        cudaGetLastError();
+        sms[device] = 0;
+    }
+    return sms[device];
 }
 
 lrs_status api_fail(lrs_status s, const char* msg) { return fail(s, "%s", msg); }

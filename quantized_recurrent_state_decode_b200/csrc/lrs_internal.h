@@ -28,6 +28,21 @@ const void* find_step_kernel_bdr_bf16(int C, int group, int update_kind, int gat
 int step_warp_smem(int C, int group, int update_kind, int gate_kind, int slots, int mode, int io,
                    int d_k);
 
+// Launch shape of the step kernel for one state shape, rounding mode and I/O
+// type on `device` with `sms` SMs: kernel, ring slots per warp, warps per
+// CTA, shared memory per warp and per CTA, and the grid (CTAs that fit on all
+// SMs; a launch takes at most one warp per tile). Prepared once per (kernel,
+// device). The one launcher of every entry point that runs the step kernel.
+struct StepLaunch {
+    const void* fn;
+    int slots, warps, warp_smem, smem, grid;
+};
+lrs_status step_launch_shape(const lrs_shape& sh, int mode, int io, int device, int sms,
+                             StepLaunch* out);
+
+// SM count of a device (queried once; 0 when the query fails).
+int sm_count(int device);
+
 // The chunked-update kernel for one shape and rounding mode, with the bytes
 // of shared memory it takes per CTA ({nullptr, 0} when not compiled).
 struct ChunkKernel {

@@ -2,14 +2,16 @@
 //
 // lrs_decode_step_host stages the step's inputs and output in device buffers
 // that it allocates on first use, and its kernels record errors in a device
-// word allocated by the library. Some callers cannot allocate device memory
-// when they step: code running while a stream is being captured into a CUDA
-// graph (cudaMalloc is not allowed there), and processes whose device memory
-// is owned by another allocator or a fixed pool that must not grow behind its
-// back. lrs_decode_step_host_noalloc serves them: its scratch (the error word
-// and the staging of inputs and output) is the file-scope array below, part
-// of the library's image, which every GPU that loads the library holds until
-// the process exits.
+// word allocated by the library. Some callers must not allocate device memory
+// when they step: processes whose device memory belongs to another allocator
+// or to a fixed pool sized at start-up (an allocation behind its back can fail
+// or break its accounting), and latency-critical paths that cannot afford a
+// cudaMalloc, which may synchronize the device. lrs_decode_step_host_noalloc
+// serves them: its scratch (the error word and the staging of inputs and
+// output) is the file-scope array below, part of the library's device image.
+// Each device takes it when that image is loaded there -- at the latest on the
+// first call on the device, since CUDA loads modules lazily -- and keeps it
+// until the process exits.
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
@@ -73,9 +75,7 @@ extern "C" lrs_status lrs_decode_step_host_noalloc(const lrs_state* st, const fl
     if (delta && !beta_host) return lrs::api_fail(LRS_ERR_INVALID_ARG, "beta_host is NULL");
     if (mode != LRS_ROUND_RTN && mode != LRS_ROUND_SR && mode != LRS_ROUND_BDR)
         return lrs::api_fail(LRS_ERR_INVALID_ARG, "mode is not an lrs_round_mode");
-    const int C = sh.d_v / 32, G = sh.d_k / sh.group;
-    const void* fn = lrs::find_step_kernel(C, sh.group, sh.update_kind, sh.gate_kind, mode);
-    if (!fn) return lrs::api_fail(LRS_ERR_UNSUPPORTED, "no compiled kernel for this shape and mode");
+    const int G = sh.d_k / sh.group;
 
     const size_t T = static_cast<size_t>(sh.batch) * sh.heads;
     const size_t bq = T * sh.d_k * 4, bv = T * sh.d_v * 4;
@@ -116,29 +116,14 @@ extern "C" lrs_status lrs_decode_step_host_noalloc(const lrs_state* st, const fl
         return lrs::api_cuda_fail(e, "host-to-device copy into the static scratch");
     }
 
-    // launch shape: the same choices as lrs_decode_step (a whole tile resident
-    // for the delta rule, two slots otherwise, up to the variant's warps)
-    int slots = delta ? G : std::min(2, G);
-    slots = std::max(1, std::min(slots, lrs::kMaxSlots));
-    const int warp_smem = lrs::step_warp_smem(C, sh.group, sh.update_kind, sh.gate_kind, slots, mode,
-                                              lrs::kStepIoF32, sh.d_k);
-    constexpr int kSmemLimit = 227 * 1024;
-    int warps = std::min(12, std::max(1, kSmemLimit / warp_smem));
-    warps = std::min(warps, lrs::step_max_warps(sh.group, mode, sh.update_kind));
-    const int smem = warps * warp_smem;
-    int dev = 0, sms = 0, per_sm = 0;
-    cudaGetDevice(&dev);
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
-        (e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit)) !=
-            cudaSuccess ||
-        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, warps * 32, smem)) !=
-            cudaSuccess) {
-        cudaGetLastError();
-        return lrs::api_cuda_fail(e, "preparing the step kernel");
-    }
-    if (per_sm < 1) return lrs::api_fail(LRS_ERR_UNSUPPORTED, "step kernel does not fit on an SM");
+    // the launch shape of lrs_decode_step (one shared, cached helper)
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return lrs::api_cuda_fail(e, "cudaGetDevice");
+    lrs::StepLaunch ls;
+    s = lrs::step_launch_shape(sh, mode, lrs::kStepIoF32, dev, lrs::sm_count(dev), &ls);
+    if (s != LRS_OK) return s;
     const int ntiles = static_cast<int>(T);
-    const int grid = std::min(sms * per_sm, (ntiles + warps - 1) / warps);
+    const int grid = std::min(ls.grid, (ntiles + ls.warps - 1) / ls.warps);
 
     lrs::StepParams p;
     memset(&p, 0, sizeof p);
@@ -162,11 +147,12 @@ extern "C" lrs_status lrs_decode_step_host_noalloc(const lrs_state* st, const fl
     p.G = G;
     p.ntiles = ntiles;
     p.pgroups = lrs::state_prec_groups(st);
-    p.slots = slots;
-    p.warp_smem = warp_smem;
+    p.slots = ls.slots;
+    p.warp_smem = ls.warp_smem;
     p.inject = 0;
     void* args[] = {&p};
-    if ((e = cudaLaunchKernel(fn, dim3(grid), dim3(warps * 32), args, smem, cs)) != cudaSuccess) {
+    if ((e = cudaLaunchKernel(ls.fn, dim3(grid), dim3(ls.warps * 32), args, ls.smem, cs)) !=
+        cudaSuccess) {
         cudaGetLastError();
         return lrs::api_cuda_fail(e, "launch of the step kernel");
     }

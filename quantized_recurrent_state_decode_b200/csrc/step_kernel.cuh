@@ -67,7 +67,7 @@ struct StepParams {
     int32_t pgroups;     // widths in prec_map per head: 1, or one per scale group: G
     int32_t slots;       // ring slots per warp, 1..min(G, 16); the delta rule needs G
     int32_t warp_smem;   // bytes of shared memory per warp
-    int32_t inject;      // fault injection: issue no copies
+    int32_t inject;      // error-path tests: 0, or n + 1 to issue copies for n items per warp
 };
 
 // Shared-memory layout of one warp (ES = bytes of a q, k, v element).
@@ -95,7 +95,10 @@ struct Slot {
     static constexpr int kK = kQ + GROUP * ES;                    // INS only
     static constexpr int kBytes = INS ? kK + GROUP * ES : kQ;
     static_assert(kBytes % 16 == 0, "slot alignment");
-    static constexpr int kXsBytes = GROUP * 256;   // x staging (SR, BDR): 16 B per row pair and lane
+    // x staging (SR, BDR): 16 B per row pair and lane; then, for SR, the
+    // group's row table of the element hash (8 B per key row)
+    static constexpr int kTabOff = GROUP * 256;
+    static constexpr int kXsBytes = kTabOff + GROUP * 8;
     // offsets inside a tile-input buffer (!INS)
     __host__ __device__ static int in_k(int d_k) { return d_k * ES; }
     __host__ __device__ static int in_g(int d_k) { return 2 * d_k * ES; }
@@ -157,6 +160,39 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
         "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
         : "=f"(r.x), "=f"(r.y)
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return r;
+}
+
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+// a + b rounded toward plus infinity, two-wide.
+__device__ __forceinline__ float2 add2_rp(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rp.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+// 1.0f when a < b (a > b), else 0.0f: one comparison that writes a float.
+__device__ __forceinline__ float set_lt(float a, float b) {
+    float r;
+    asm("set.lt.f32.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float set_gt(float a, float b) {
+    float r;
+    asm("set.gt.f32.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
     return r;
 }
 
@@ -294,6 +330,78 @@ __device__ __forceinline__ void new_scales(float A0, float A1, float2& snew, flo
     inv = make_float2(A0 < kTiny ? 0.0f : iv.x, A1 < kTiny ? 0.0f : iv.y);
 }
 
+// Stochastic rounding of two elements (key rows i, i+1 of one column), from
+// their draws' `top` words (see hash_top). Returned as the floats kb + code
+// (kb: word_bias of the elements' word positions).
+//
+// The floor comes straight out as kb + floor(y) from one fused multiply-add
+// rounded toward minus infinity (y = x*inv exact inside it; kb is an integer
+// in [2^23, 2^24), where the float spacing is 1). The floor is clamped to
+// [-qmax, qmax - 1] first: the clamped cases then decide themselves -- below
+// -qmax the fraction y - f is negative and never draws the step up, at or
+// above qmax it is at least 1 and always does -- so no clamp is needed after
+// the step, and everywhere else this is the plain floor. The fraction
+// fr = RN(y - f) is rounded once, as defined. The draw u = (top >> 9) 2^-23 is
+// on the 2^-23 grid, so u < fr exactly when 1 + u < RU(1 + fr): both sides
+// are floats in the same binade or RU(1 + fr) has left it (fr >= 1 - 2^-24:
+// always up; fr < 0: never). The comparison writes 1.0f or 0.0f, added to the
+// floor.
+template <int BITS>
+__device__ __forceinline__ float2 sr_round(float2 x, float2 inv, float2 kb, uint32_t top0,
+                                           uint32_t top1) {
+    constexpr float QMAX = Q<BITS>::kMax;
+    float2 tb = fma2_rm(x, inv, kb);
+    tb.x = fminf(fmaxf(tb.x, kb.x - QMAX), kb.x + (QMAX - 1.0f));
+    tb.y = fminf(fmaxf(tb.y, kb.y - QMAX), kb.y + (QMAX - 1.0f));
+    const float2 fr = fma2(x, inv, sub2(kb, tb));       // y - f, one rounding (kb - tb = -f exactly)
+    const float2 g = add2_rp(fr, f2(1.0f));
+    return add2(tb, make_float2(set_lt(sr_unit1(top0), g.x), set_lt(sr_unit1(top1), g.y)));
+}
+
+// Bounded Directional Rounding of two elements (key rows i, i+1 of one
+// column). deq: their values before the update; s_new: the new scale.
+//
+// n = rint(y) comes out biased (kb + n) from one multiply-add; -n = kb - nb
+// exactly. The update a = RN(x - deq) and the move b = RN(p - deq),
+// p = RN(n s'), enter only through their signs (a rounded difference of two
+// floats is zero only when they are equal, and has their difference's sign),
+// and so does d = RN(y - n). A reversal (a and b of opposite signs) takes
+// ceil(y) when the update is positive and floor(y) when it is negative;
+// ceil = n + 1 exactly when d > 0, floor = n - 1 exactly when d < 0. With
+// e = RN(deq - p) = -b the code therefore moves up when min(a, e, d) > 0 and
+// down when max(a, e, d) < 0: one three-input minimum and maximum, each
+// compared into 1.0f or 0.0f.
+//
+// No clamp to [-qmax, qmax] is needed afterwards. A step up from n = qmax
+// needs y > qmax, and only x = A itself (the column's absmax) reaches it,
+// when A * inv > qmax; it also needs p < deq < x = A. For every significand
+// of A where A * inv > qmax (qmax 7 and 127, all 2^23 of them; the
+// quantities scale exactly with A's exponent over the range used), p is at
+// least the float just below A, so no deq lies strictly between: the step
+// never happens. Mirrored, the same holds for a step down from -qmax.
+//
+// deq and p are products. Their differences are taken with the scalar
+// __fsub_rn / __fadd_rn, which the compiler never contracts with the
+// multiply before them:
+// a two-wide subtraction of a two-wide product was seen contracted into one
+// fused multiply-add, which keeps the product unrounded and turns an exact
+// tie (x == deq or deq == p, difference 0) into a nonzero sign.
+template <int BITS>
+__device__ __forceinline__ float2 bdr_round(float2 x, float2 inv, float2 deq, float2 s_new,
+                                            float2 kb) {
+    const float2 nb = fma2(x, inv, kb);
+    const float2 nn = sub2(kb, nb);                     // -n
+    const float2 d = fma2(x, inv, nn);
+    const float2 mp = mul2(nn, s_new);                  // -p
+    const float2 a = make_float2(__fsub_rn(x.x, deq.x), __fsub_rn(x.y, deq.y));
+    const float2 e = make_float2(__fadd_rn(deq.x, mp.x), __fadd_rn(deq.y, mp.y));   // deq - p
+    const float2 up = make_float2(set_gt(min3(a.x, e.x, d.x), 0.0f),
+                                  set_gt(min3(a.y, e.y, d.y), 0.0f));
+    const float2 dn = make_float2(set_lt(max3(a.x, e.x, d.x), 0.0f),
+                                  set_lt(max3(a.y, e.y, d.y), 0.0f));
+    return add2(nb, sub2(up, dn));
+}
+
 // Codes of two elements (key rows i, i+1 of value column j; i even), returned
 // as the floats kb + code (kb: word_bias of the two elements' word positions)
 // whose low bits are the stored byte (nibble). inv, s_new: the column's values
@@ -303,57 +411,24 @@ __device__ __forceinline__ void new_scales(float A0, float A1, float2& snew, flo
 template <int MODE, int BITS, bool HASH64 = false>
 __device__ __forceinline__ float2 round_rows(float2 x, float2 inv, float2 deq, float2 s_new,
                                              float2 kb, uint64_t hkey, uint32_t i, uint32_t j) {
-    constexpr float QMAX = Q<BITS>::kMax;
     if constexpr (MODE == kRTN) {
         // |x*inv| <= qmax (1 + 2^-24) since inv = RN(qmax/A) and |x| <= A:
         // the nearest integer never leaves [-qmax, qmax], no clamp needed.
         return fma2(x, inv, kb);
-    } else {
-        float2 c;
-        if constexpr (MODE == kSR) {
-            // floor(x*inv): the exact product plus 1.5*2^23, rounded toward
-            // minus infinity, lands on the integer below it (|x*inv| < 2^22)
-            const float2 f = add2(fma2_rm(x, inv, f2(kRound)), f2(-kRound));
-            const float2 fr = fma2(x, inv, neg2(f));                      // fraction, rounded once
-            const float2 f1 = add2(f, f2(1.0f));
-            float u0, u1;
-            if constexpr (HASH64) {
-                u0 = element_uniform_u64(hkey, i, j);
-                u1 = element_uniform_u64(hkey, i + 1, j);
-            } else {
-                const HashColumn hc = hash_column(hkey, j);
-                const uint32_t khi = static_cast<uint32_t>(hkey >> 32) ^ i;
-                u0 = hash_uniform(khi, hc);
-                u1 = hash_uniform(khi ^ 1u, hc);                         // row i + 1 (i even)
-            }
-            c.x = u0 < fr.x ? f1.x : f.x;
-            c.y = u1 < fr.y ? f1.y : f.y;
+    } else if constexpr (MODE == kSR) {
+        uint32_t t0, t1;
+        if constexpr (HASH64) {
+            t0 = element_top_u64(hkey, i, j);
+            t1 = element_top_u64(hkey, i + 1, j);
         } else {
-            const float2 n = add2(fma2(x, inv, f2(kRound)), f2(-kRound));  // nearest integer
-            const float2 d = fma2(x, inv, neg2(n));                          // sign of x*inv - n
-            // The update a = RN(x - deq) and the move b = RN(p - deq),
-            // p = RN(n s'), enter only through their signs. A reversal (a
-            // and b of opposite signs) takes ceil(x*inv) when the update is
-            // positive and floor(x*inv) when it is negative; ceil = n + 1
-            // exactly when d > 0, floor = n - 1 exactly when d < 0. So the
-            // code moves up when a > 0, b < 0 and d > 0, i.e. when
-            // min(a, -b, d) > 0, and down when max(a, -b, d) < 0: one
-            // three-input minimum or maximum and one compare each, no
-            // branches. (The subtractions are exact in sign: a rounded
-            // difference of two floats is zero only when they are equal.)
-            const float2 p = mul2(n, s_new);
-            const float2 a = add2(x, neg2(deq));
-            const float2 nb = add2(deq, neg2(p));                         // -b
-            const bool up0 = min3(a.x, nb.x, d.x) > 0.0f;
-            const bool dn0 = max3(a.x, nb.x, d.x) < 0.0f;
-            const bool up1 = min3(a.y, nb.y, d.y) > 0.0f;
-            const bool dn1 = max3(a.y, nb.y, d.y) < 0.0f;
-            c.x = up0 ? n.x + 1.0f : (dn0 ? n.x - 1.0f : n.x);
-            c.y = up1 ? n.y + 1.0f : (dn1 ? n.y - 1.0f : n.y);
+            const HashColumn hc = hash_column(hkey, j);
+            const uint32_t khi = static_cast<uint32_t>(hkey >> 32) ^ i;
+            t0 = hash_top(khi, hc);
+            t1 = hash_top(khi ^ 1u, hc);                                // row i + 1 (i even)
         }
-        c.x = fminf(fmaxf(c.x, -QMAX), QMAX);
-        c.y = fminf(fmaxf(c.y, -QMAX), QMAX);
-        return add2(c, kb);
+        return sr_round<BITS>(x, inv, kb, t0, t1);
+    } else {
+        return bdr_round<BITS>(x, inv, deq, s_new, kb);
     }
 }
 
@@ -659,6 +734,105 @@ struct TileCursor : TileLayout {
 // x[r+1][c0], x[r][c1], x[r+1][c1]) per row pair r and lane) or recomputed
 // from the codes, scales, k, gates and w, by the same operations in the same
 // order, so bit for bit the same values.
+//
+// SR draws come from the group's row table (rtab: per row pair of the group
+// the SrRow values of its two rows) when the tile's low-sum carry is the same
+// for all columns (rowtab), else from the whole per-element hash.
+template <int GROUP, int GATE, int MODE, int BITS, int IO, bool STAGE, bool ROWTAB>
+__device__ __forceinline__ void round_pass(const uint8_t* __restrict__ cs, int ubase, float2 sc,
+                                           const uint8_t* __restrict__ ks,
+                                           const float* __restrict__ gs, float gscalar, float2 w,
+                                           float2 inv, float2 snew, uint8_t* __restrict__ gcodes,
+                                           uint64_t hkey, int row0, uint32_t j0, int lane,
+                                           const float4* __restrict__ xs,
+                                           const uint4* __restrict__ rtab) {
+    using G = PairGeo<GROUP, BITS>;
+    constexpr float BIAS = Q<BITS>::kBias;
+    constexpr int RPUH = G::RPU / 2;              // row pairs per unit
+    const float2 s0 = f2(sc.x), s1 = f2(sc.y);
+    const float2 w0 = f2(w.x), w1 = f2(w.y);
+    const float2 gsc = f2(gscalar);
+    const float2 inv0 = f2(inv.x), inv1 = f2(inv.y);
+    const float2 sn0 = f2(snew.x), sn1 = f2(snew.y);
+    // SR column parts of the draw: row-table form (clo only) or the whole hash
+    const uint32_t khi = static_cast<uint32_t>(hkey >> 32);
+    const HashColumn hc0 = hash_column(hkey, j0), hc1 = hash_column(hkey, j0 + 1);
+
+    constexpr bool DECODE = MODE == kBDR || !STAGE;   // this pass reads the old codes
+#pragma unroll 1
+    for (int un = 0; un < G::UNITS; ++un) {
+        uint32_t ow[4];
+        uint32_t wd[4] = {0u, 0u, 0u, 0u};
+        if constexpr (DECODE) {
+            const uint4 raw = lds_unit(cs, ubase + un, lane);
+            wd[0] = raw.x; wd[1] = raw.y; wd[2] = raw.z; wd[3] = raw.w;
+        }
+        float kk[STAGE ? 1 : G::RPU], gg[STAGE || GATE != kGatePerKey ? 1 : G::RPU];
+        if constexpr (!STAGE) {
+            ld_rows<IO, G::RPU>(ks, un * G::RPU, kk);
+            if constexpr (GATE == kGatePerKey) ld_smem_rows<G::RPU>(gs + un * G::RPU, gg);
+        }
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+            float f[G::EPW];
+            if constexpr (DECODE) decode_word_biased<BITS>(wd[wi], f);
+            float t[G::EPW];
+#pragma unroll
+            for (int rp = 0; rp < G::RPW / 2; ++rp) {
+                const int rl = wi * G::RPW + 2 * rp;
+                float2 dq0 = f2(0.0f), dq1 = f2(0.0f);
+                if constexpr (DECODE) {
+                    dq0 = mul2(add2(make_float2(f[4 * rp], f[4 * rp + 2]), f2(-(kTwo23 + BIAS))), s0);
+                    dq1 = mul2(add2(make_float2(f[4 * rp + 1], f[4 * rp + 3]), f2(-(kTwo23 + BIAS))), s1);
+                }
+                float4 xv;
+                if constexpr (STAGE) {
+                    xv = xs[(un * RPUH + rl / 2) * 32 + lane];
+                } else {
+                    // the first loop's x, recomputed by the same operations
+                    const float2 kr = make_float2(kk[rl], kk[rl + 1]);
+                    const float2 gr = GATE == kGatePerKey ? make_float2(gg[rl], gg[rl + 1]) : gsc;
+                    const float2 x0 = fma2(gr, dq0, mul2(kr, w0));
+                    const float2 x1 = fma2(gr, dq1, mul2(kr, w1));
+                    xv = make_float4(x0.x, x0.y, x1.x, x1.y);
+                }
+                const float2 kb0 = make_float2(word_bias<BITS>(4 * rp), word_bias<BITS>(4 * rp + 2));
+                const float2 kb1 = make_float2(word_bias<BITS>(4 * rp + 1), word_bias<BITS>(4 * rp + 3));
+                float2 t0, t1;
+                if constexpr (MODE == kSR) {
+                    uint32_t a0, a1, b0, b1;          // tops: column 0 rows i, i+1; column 1
+                    if constexpr (ROWTAB) {
+                        const uint4 rt = rtab[un * RPUH + rl / 2];
+                        a0 = hash_top_row(hc0.clo, rt.x, rt.y);
+                        a1 = hash_top_row(hc0.clo, rt.z, rt.w);
+                        b0 = hash_top_row(hc1.clo, rt.x, rt.y);
+                        b1 = hash_top_row(hc1.clo, rt.z, rt.w);
+                    } else {
+                        const uint32_t ki = khi ^ static_cast<uint32_t>(row0 + un * G::RPU + rl);
+                        a0 = hash_top(ki, hc0);
+                        a1 = hash_top(ki ^ 1u, hc0);
+                        b0 = hash_top(ki, hc1);
+                        b1 = hash_top(ki ^ 1u, hc1);
+                    }
+                    t0 = sr_round<BITS>(make_float2(xv.x, xv.y), inv0, kb0, a0, a1);
+                    t1 = sr_round<BITS>(make_float2(xv.z, xv.w), inv1, kb1, b0, b1);
+                } else {
+                    t0 = round_rows<MODE, BITS>(make_float2(xv.x, xv.y), inv0, dq0, sn0, kb0, 0ull,
+                                                0u, 0u);
+                    t1 = round_rows<MODE, BITS>(make_float2(xv.z, xv.w), inv1, dq1, sn1, kb1, 0ull,
+                                                0u, 0u);
+                }
+                t[4 * rp] = t0.x;
+                t[4 * rp + 2] = t0.y;
+                t[4 * rp + 1] = t1.x;
+                t[4 * rp + 3] = t1.y;
+            }
+            ow[wi] = encode_word<BITS>(t);
+        }
+        st_cs_u4(gcodes + ((ubase + un) * 32 + lane) * 16, ow[0], ow[1], ow[2], ow[3]);
+    }
+}
+
 template <int GROUP, int GATE, int MODE, int BITS, int IO, bool STAGE>
 __device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int ubase, float2 sc,
                                              const uint8_t* __restrict__ qs,
@@ -666,7 +840,8 @@ __device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int
                                              const float* __restrict__ gs, float gscalar,
                                              float2 w, float2& o, uint8_t* __restrict__ gcodes,
                                              float* __restrict__ gscale, uint64_t hkey, int row0,
-                                             uint32_t j0, int lane, float4* __restrict__ xs) {
+                                             uint32_t j0, int lane, float4* __restrict__ xs,
+                                             const uint4* __restrict__ rtab, bool rowtab) {
     using G = PairGeo<GROUP, BITS>;
     constexpr float BIAS = Q<BITS>::kBias;
     constexpr int RPUH = G::RPU / 2;              // row pairs per unit
@@ -712,63 +887,14 @@ __device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int
     float2 snew, inv;
     new_scales<BITS>(a0, b0, snew, inv);
     st_cs_f2(gscale, snew);
-    const float2 inv0 = f2(inv.x), inv1 = f2(inv.y);
-    const float2 sn0 = f2(snew.x), sn1 = f2(snew.y);
-
-    constexpr bool DECODE = MODE == kBDR || !STAGE;   // phase 2 reads the old codes
-#pragma unroll 1
-    for (int un = 0; un < G::UNITS; ++un) {
-        uint32_t ow[4];
-        uint32_t wd[4] = {0u, 0u, 0u, 0u};
-        if constexpr (DECODE) {
-            const uint4 raw = lds_unit(cs, ubase + un, lane);
-            wd[0] = raw.x; wd[1] = raw.y; wd[2] = raw.z; wd[3] = raw.w;
-        }
-        float kk[STAGE ? 1 : G::RPU], gg[STAGE || GATE != kGatePerKey ? 1 : G::RPU];
-        if constexpr (!STAGE) {
-            ld_rows<IO, G::RPU>(ks, un * G::RPU, kk);
-            if constexpr (GATE == kGatePerKey) ld_smem_rows<G::RPU>(gs + un * G::RPU, gg);
-        }
-#pragma unroll
-        for (int wi = 0; wi < 4; ++wi) {
-            float f[G::EPW];
-            if constexpr (DECODE) decode_word_biased<BITS>(wd[wi], f);
-            float t[G::EPW];
-#pragma unroll
-            for (int rp = 0; rp < G::RPW / 2; ++rp) {
-                const int rl = wi * G::RPW + 2 * rp;
-                float2 dq0 = f2(0.0f), dq1 = f2(0.0f);
-                if constexpr (DECODE) {
-                    dq0 = mul2(add2(make_float2(f[4 * rp], f[4 * rp + 2]), f2(-(kTwo23 + BIAS))), s0);
-                    dq1 = mul2(add2(make_float2(f[4 * rp + 1], f[4 * rp + 3]), f2(-(kTwo23 + BIAS))), s1);
-                }
-                float4 xv;
-                if constexpr (STAGE) {
-                    xv = xs[(un * RPUH + rl / 2) * 32 + lane];
-                } else {
-                    // the first loop's x, recomputed by the same operations
-                    const float2 kr = make_float2(kk[rl], kk[rl + 1]);
-                    const float2 gr = GATE == kGatePerKey ? make_float2(gg[rl], gg[rl + 1]) : gsc;
-                    const float2 x0 = fma2(gr, dq0, mul2(kr, w0));
-                    const float2 x1 = fma2(gr, dq1, mul2(kr, w1));
-                    xv = make_float4(x0.x, x0.y, x1.x, x1.y);
-                }
-                const uint32_t i = static_cast<uint32_t>(row0 + un * G::RPU + rl);
-                const float2 kb0 = make_float2(word_bias<BITS>(4 * rp), word_bias<BITS>(4 * rp + 2));
-                const float2 kb1 = make_float2(word_bias<BITS>(4 * rp + 1), word_bias<BITS>(4 * rp + 3));
-                const float2 t0 = round_rows<MODE, BITS>(make_float2(xv.x, xv.y), inv0, dq0, sn0,
-                                                         kb0, hkey, i, j0);
-                const float2 t1 = round_rows<MODE, BITS>(make_float2(xv.z, xv.w), inv1, dq1, sn1,
-                                                         kb1, hkey, i, j0 + 1);
-                t[4 * rp] = t0.x;
-                t[4 * rp + 2] = t0.y;
-                t[4 * rp + 1] = t1.x;
-                t[4 * rp + 3] = t1.y;
-            }
-            ow[wi] = encode_word<BITS>(t);
-        }
-        st_cs_u4(gcodes + ((ubase + un) * 32 + lane) * 16, ow[0], ow[1], ow[2], ow[3]);
-    }
+    if (MODE == kSR && rowtab)
+        round_pass<GROUP, GATE, MODE, BITS, IO, STAGE, true>(cs, ubase, sc, ks, gs, gscalar, w,
+                                                            inv, snew, gcodes, hkey, row0, j0,
+                                                            lane, xs, rtab);
+    else
+        round_pass<GROUP, GATE, MODE, BITS, IO, STAGE, false>(cs, ubase, sc, ks, gs, gscalar, w,
+                                                             inv, snew, gcodes, hkey, row0, j0,
+                                                             lane, xs, rtab);
 }
 
 // Fill `slot` with group g of the cursor's tile (lane 0 only); with the
@@ -857,6 +983,8 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE, UPD) * 32, 1)
     float* cvt = reinterpret_cast<float*>(wsm + hdr + NS * S::kBytes);   // bf16 widened (CVT)
     float4* xs = reinterpret_cast<float4*>(wsm + hdr + NS * S::kBytes +
                                            S::cvt_bytes(p.d_k));              // SR, BDR
+    uint2* rtab2 = reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(xs) + S::kTabOff);  // SR
+    const uint4* rtab = reinterpret_cast<const uint4*>(rtab2);
     constexpr int IOR = S::CVT ? kIoF32 : IO;     // element type the pair code reads
     constexpr int ESR = IOR == kIoBF16 ? 2 : 4;
     const int ntw = gw < p.ntiles ? (p.ntiles - gw + W - 1) / W : 0;   // this warp's tiles
@@ -878,8 +1006,11 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE, UPD) * 32, 1)
     itc.init(p, gw, W);
     if (K > 0) itc.load(p, GROUP * DV);
 
+    // p.inject (error-path tests): n + 1 issues copies for the warp's first n
+    // items only, so a later wait runs out
+    const int64_t kmax = p.inject ? static_cast<int64_t>(p.inject - 1) : K;
     auto issue_next = [&]() {
-        if (ki < K && !p.inject) {
+        if (ki < K && ki < kmax) {
             if (lane == 0)
                 issue_item<C, GROUP, GATE, IO, INS>(p, wsm, is.slot, itc, it_g,
                                                wsm + 128 + (it_n & 1) * tib, pol_state, pol_in);
@@ -918,6 +1049,8 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE, UPD) * 32, 1)
                                                           static_cast<uint32_t>(ti.b),
                                                           static_cast<uint32_t>(ti.h))
                                           : 0ull;
+        uint32_t hcarry = 0;
+        const bool rowtab = MODE == kSR && sr_tile_carry(hkey, DV, &hcarry);
 
         // the tile's first group
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[ic.slot], ic.par, p.timeout_ns));
@@ -1033,6 +1166,18 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE, UPD) * 32, 1)
             float* gscale = p.scales + (static_cast<int64_t>(tile) * G + g) * DV + lane * C;
             uint8_t* gcodes = gcodes_tile + ti.goff(g, GROUP * DV / 2);
             const bool int8g = ti.bits(g) == 8;
+            if constexpr (MODE == kSR) {
+                // the group's row table of the element hash (the previous
+                // group's readers finished at the warp barrier ending it)
+                if (rowtab) {
+                    for (int r = lane; r < GROUP; r += 32) {
+                        const SrRow rr = sr_row(static_cast<uint32_t>(hkey >> 32),
+                                                static_cast<uint32_t>(g * GROUP + r), hcarry);
+                        rtab2[r] = make_uint2(rr.sh, rr.p);
+                    }
+                    __syncwarp();
+                }
+            }
             // The column pairs run one after the other through one copy of the
             // (large) pair code; the pairs' w and o rotate through (wp, op).
             float2 wp = w[0], op = o[0], wq = w[P - 1], oq = o[P - 1];
@@ -1046,12 +1191,12 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE, UPD) * 32, 1)
                         pair_step_xs<GROUP, GATE, MODE, 8, IOR, ST>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc,
                                                                qs, ks, gs, gscalar, wp, op, gcodes,
                                                                gscale + 2 * pc, hkey, g * GROUP, j0,
-                                                               lane, xs);
+                                                               lane, xs, rtab, rowtab);
                     else
                         pair_step_xs<GROUP, GATE, MODE, 4, IOR, ST>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc,
                                                                qs, ks, gs, gscalar, wp, op, gcodes,
                                                                gscale + 2 * pc, hkey, g * GROUP, j0,
-                                                               lane, xs);
+                                                               lane, xs, rtab, rowtab);
                 } else {
                     if (int8g)
                         pair_step<GROUP, GATE, MODE, 8, IOR>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs, ks,

@@ -79,6 +79,7 @@ _SIGS = {
     "lrs_precision_map": [ctypes.c_int32, _P, ctypes.c_int32, _P],
     "lrs_sync": [_P],
     "lrs_debug_inject_timeout": [ctypes.c_int32, ctypes.c_int32],
+    "lrs_debug_inject_timeout_after": [ctypes.c_int32, ctypes.c_int32],
 }
 
 
@@ -281,3 +282,7 @@ def lrs_sync(stream=None):
 
 def lrs_debug_inject_timeout(enable, timeout_us=1000):
     _check(lib().lrs_debug_inject_timeout(1 if enable else 0, timeout_us))
+
+
+def lrs_debug_inject_timeout_after(items_copied, timeout_us=1000):
+    _check(lib().lrs_debug_inject_timeout_after(items_copied, timeout_us))

@@ -306,6 +306,47 @@ def test_timed_out_wait_reports_and_leaves_state_untouched():
         pair.free()
 
 
+def test_timeout_on_a_later_group_leaves_a_partial_tile_and_checkpoint_restores():
+    # Each warp copies in only its first (tile, group) item, so its wait for
+    # the second one runs out after the first group of its first tile was
+    # written: the documented partial state. Restoring the checkpoint makes
+    # the next step exact again.
+    w = I.Workload("timeout_after", "gla", 8, 4, 128, 128, 32, 2, I.ROUND_RTN, "int8",
+                   s0_std=0.02, gate_mu=-4.0, seed_id=82)
+    pm = np.full(4, 8, np.uint8)
+    pair = P.Pair(w, pm)
+    G = w.d_k // w.group
+    gbytes = w.group * w.d_v                  # one int8 group block of a tile
+    try:
+        pair.init(I.initial_state(w, device="cuda"))
+        raw0, sc0 = _snapshot(pair.st)
+        x = I.step_inputs(w, 0, device="cuda")
+        lrs.lrs_debug_inject_timeout_after(1, 2000)      # waits give up after 2 ms
+        lrs.lrs_decode_step(pair.st, pair.st.state_codes, pair.st.scales, pair.st.prec_map,
+                            x["q"], x["k"], x["v"], x["gates"], None, pair.out, 0, 0, w.mode)
+        with pytest.raises(lrs.LrsError) as e:
+            lrs.lrs_sync()
+        assert e.value.status == lrs.LRS_ERR_DEVICE_TIMEOUT
+        raw1, sc1 = _snapshot(pair.st)
+        s0 = sc0.reshape(w.batch * w.heads, G, w.d_v)
+        s1 = sc1.reshape(w.batch * w.heads, G, w.d_v)
+        c0 = raw0.reshape(w.batch * w.heads, G, gbytes)
+        c1 = raw1.reshape(w.batch * w.heads, G, gbytes)
+        # 32 tiles, one per warp: every tile got its first group and no other
+        np.testing.assert_array_equal(s1[:, 1:], s0[:, 1:])
+        np.testing.assert_array_equal(c1[:, 1:], c0[:, 1:])
+        assert not np.array_equal(s1[:, 0], s0[:, 0])
+        assert not np.array_equal(c1[:, 0], c0[:, 0])
+        # restore the checkpoint; the context works and the step is exact
+        lrs.lrs_state_copy_raw(pair.st, raw0, sc0, False)
+        o_gpu, o_ref = pair.step(x, 0, 0)
+        P.check_out(o_gpu, o_ref, "after restore")
+        pair.compare_state("after restore")
+    finally:
+        lrs.lrs_debug_inject_timeout_after(-1, 0)
+        pair.free()
+
+
 def test_decay_means_and_precision_map_match_oracle():
     for name in ("mamba2_mixed_sr_b128h64", "gdn_mixed_sr_h32_128"):
         w = I.WORKLOADS[name]
