@@ -220,10 +220,10 @@ lrs_status lrs_chunk_step(const lrs_state *st, void *state_codes, float *scales,
                           const float *v, const float *gates, const float *beta, float *out,
                           uint64_t seed, uint64_t step, int32_t mode, void *stream);
 
-/* The decode step with a Low-Rank Bypass buffer ([LRB/BDR] abstract: small
- * updates accumulate in a compact low-rank buffer whose sufficiently large
- * elements are merged into the state from time to time). The sources fix no
- * rank, period or threshold; this entry point takes:
+/* The decode step with a Low-Rank Bypass buffer ([LRB/BDR] abstract, Low-Rank
+ * Bypass). The sources fix no rank, period or threshold; this entry point
+ * keeps rank-r fp32 factors of the step's updates beside the quantized state,
+ * merges them every r-th step with the threshold RN(s_old / 2), and takes:
  *   - buffer L = U V^T of rank `rank` (1..8): U [B][H][rank][d_k] and
  *     V [B][H][rank][d_v], fp32 device memory owned by the caller, zero at
  *     the start, updated in place; step mod rank components are filled before

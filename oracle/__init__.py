@@ -49,6 +49,8 @@ def lib():
         L.orc_lrb_step.restype = i32
         L.orc_lrb_step_pg.argtypes = L.orc_lrb_step.argtypes
         L.orc_lrb_step_pg.restype = i32
+        L.orc_bdr_additive_step.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P, P]
+        L.orc_bdr_additive_step.restype = i32
         L.orc_bf16_rne.argtypes = [ctypes.c_float]
         L.orc_bf16_rne.restype = ctypes.c_uint16
         L.orc_bf16_rne_array.argtypes = [i64, P, P]
@@ -205,6 +207,21 @@ def fp32_step(S, q, k, v, gates, beta, *, update_kind, gate_kind, nthreads=1):
                              _p(gates), _p(beta), _p(out), nthreads)
     if rc != 0:
         raise ValueError("orc_fp32_step rejected its arguments (%d)" % rc)
+    return out
+
+
+def bdr_additive_step(codes, scales, q, k, v, gates, *, group, qmax):
+    """Study of the other BDR reading (update = the additive term k_i w_j):
+    one gated step with per-key gates, one width for all tiles; codes and
+    scales updated in place. Returns out f32 [n][d_v]. Not a library step."""
+    n, d_k, d_v = codes.shape
+    assert codes.dtype == np.int8 and scales.dtype == np.float32
+    q, k, v, gates = map(_f32, (q, k, v, gates))
+    out = np.zeros((n, d_v), np.float32)
+    rc = lib().orc_bdr_additive_step(n, d_k, d_v, group, qmax, _p(codes), _p(scales), _p(q),
+                                     _p(k), _p(v), _p(gates), _p(out))
+    if rc != 0:
+        raise ValueError("orc_bdr_additive_step rejected its arguments (%d)" % rc)
     return out
 
 

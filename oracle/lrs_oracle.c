@@ -409,10 +409,9 @@ int orc_chunk_step_pg(int ntiles, const int32_t *tile_b, const int32_t *tile_h, 
 
 /* ------------------------------------------------- Low-Rank Bypass --- */
 
-/* [LRB/BDR] Low-Rank Bypass: small updates are accumulated in a compact
- * low-rank buffer and the buffer's sufficiently large elements are merged
- * into the state from time to time. The sources give neither the rank, the
- * merge period nor the threshold; the readings taken here:
+/* [LRB/BDR] abstract, Low-Rank Bypass. The sources give neither the rank,
+ * the merge period nor the threshold; the readings taken here (rank-r fp32
+ * factors, a merge every r-th step, threshold RN(s_old / 2)):
  *   - buffer L = sum_l U_l V_l^T, l < r, U_l in R^{d_k}, V_l in R^{d_v}, fp32;
  *     the effective state is deq(S_q) + L;
  *   - each step appends the step's rank-1 update k w^T as the next component
@@ -703,3 +702,69 @@ int orc_precision_map(int heads, const double *means, int n_int8, uint8_t *prec_
     }
     return 0;
 }
+
+/* ------------------------------------------ BDR reading study (additive) --- */
+
+int orc_bdr_additive_step(int ntiles, int d_k, int d_v, int group, int qmax, int8_t *codes,
+                          float *scales, const float *q, const float *k, const float *v,
+                          const float *gates, float *out)
+{
+    if (ntiles < 0 || d_k <= 0 || d_v <= 0 || group <= 0 || d_k % group != 0) return -1;
+    if (qmax != 127 && qmax != 7) return -1;
+    size_t n = (size_t)d_k * d_v;
+    int G = d_k / group;
+    float *deq = (float *)malloc(n * sizeof(float));
+    float *kw = (float *)malloc(n * sizeof(float));
+    float *x = (float *)malloc(n * sizeof(float));
+    if (!deq || !kw || !x) {
+        free(deq); free(kw); free(x);
+        return -2;
+    }
+    for (int t = 0; t < ntiles; ++t) {
+        int8_t *c = codes + (size_t)t * n;
+        float *s = scales + (size_t)t * G * d_v;
+        const float *qt = q + (size_t)t * d_k, *kt = k + (size_t)t * d_k;
+        const float *vt = v + (size_t)t * d_v, *gt = gates + (size_t)t * d_k;
+        /* dequantize, update (w = v), output -- as orc_step's gated form */
+        for (int i = 0; i < d_k; ++i)
+            for (int j = 0; j < d_v; ++j) {
+                deq[i * d_v + j] = (float)c[i * d_v + j] * s[(i / group) * d_v + j];
+                kw[i * d_v + j] = kt[i] * vt[j];
+                x[i * d_v + j] = fmaf(gt[i], deq[i * d_v + j], kw[i * d_v + j]);
+            }
+        for (int j = 0; j < d_v; ++j) {
+            float acc = 0.0f;
+            for (int i = 0; i < d_k; ++i) acc = fmaf(qt[i], x[i * d_v + j], acc);
+            out[(size_t)t * d_v + j] = acc;
+        }
+        /* new scales as orc_step; codes with the additive term as the update */
+        for (int g = 0; g < G; ++g)
+            for (int j = 0; j < d_v; ++j) {
+                float A = 0.0f;
+                for (int i = g * group; i < (g + 1) * group; ++i)
+                    if (fabsf(x[i * d_v + j]) > A) A = fabsf(x[i * d_v + j]);
+                float s_new = 0.0f, inv = 0.0f;
+                if (A >= ORC_TINY) {
+                    s_new = A / (float)qmax;
+                    inv = (float)qmax / A;
+                }
+                s[g * d_v + j] = s_new;
+                for (int i = g * group; i < (g + 1) * group; ++i) {
+                    size_t e = (size_t)i * d_v + j;
+                    double y = (double)x[e] * (double)inv;
+                    double c0 = rint(y), cc = c0;
+                    float m = (float)c0 * s_new - deq[e];
+                    if (kw[e] > 0.0f && m < 0.0f)
+                        cc = ceil(y);
+                    else if (kw[e] < 0.0f && m > 0.0f)
+                        cc = floor(y);
+                    if (cc > qmax) cc = qmax;
+                    if (cc < -qmax) cc = -qmax;
+                    c[e] = (int8_t)cc;
+                }
+            }
+    }
+    free(deq); free(kw); free(x);
+    return 0;
+}
+

@@ -134,6 +134,20 @@ int orc_lrb_step_pg(int ntiles, const int32_t *tile_b, const int32_t *tile_h,
                     const float *gates, const float *beta, float *out, uint64_t seed,
                     uint64_t step, float *x_out);
 
+/* A study of the Bounded Directional Rounding reading (not a step the
+ * library implements). [LRB/BDR] says a stored element can move opposite to
+ * "its update" and that BDR rounds such elements toward the update. The
+ * library reads the update as the element's whole change x - deq this step.
+ * This function takes the other reading, the additive term k_i w_j alone
+ * (decay excluded), for the gated update with per-key gates and one code
+ * width (qmax 127 or 7) for every tile: deq, x, out and the new scales as in
+ * orc_step; then c0 = rint(y), move m = RN(RN(c0 s') - deq), and c = ceil(y)
+ * when k_i w_j > 0 > m, floor(y) when k_i w_j < 0 < m, else c0; clamped.
+ * Single-threaded. */
+int orc_bdr_additive_step(int ntiles, int d_k, int d_v, int group, int qmax, int8_t *codes,
+                          float *scales, const float *q, const float *k, const float *v,
+                          const float *gates, float *out);
+
 /* bfloat16 (the upper half of binary32: sign, 8 exponent bits, 7 fraction
  * bits) nearest to x, ties to the even fraction; NaN becomes a quiet NaN of the
  * same sign. Returns the 16-bit pattern. */

@@ -1,9 +1,8 @@
 // lrb_kernel.cuh -- the decode step with a Low-Rank Bypass buffer.
 //
-// "Preserving Updates in Low-Bit Recurrent State Quantization" (abstract):
-// small updates are accumulated in a compact low-rank buffer and the buffer's
-// sufficiently large elements are merged into the state from time to time.
-// The readings (the sources give neither rank, period nor threshold): each
+// "Preserving Updates in Low-Bit Recurrent State Quantization" (abstract,
+// Low-Rank Bypass). The readings (the sources give neither rank, period nor
+// threshold): each
 // step's rank-1 update k w^T is appended to a rank-r fp32 buffer L = U V^T
 // (U [r][d_k], V [r][d_v] per tile) instead of the quantized state; older
 // components decay with the state; the delta rule and the output read the

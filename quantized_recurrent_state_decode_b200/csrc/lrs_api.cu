@@ -216,11 +216,13 @@ const void* find_step_kernel(int C, int group, int update_kind, int gate_kind, i
 
 int step_warp_smem(int C, int group, int update_kind, int gate_kind, int slots, int mode, int io,
                    int d_k) {
-    const bool xs = stage_x(mode, update_kind);
+    const bool xs = stage_x(mode, update_kind), tab = mode == kSR;
 #define LRS_SLOT_IO(CC, GG, IO)                                                                   \
-    if (update_kind == kDelta) return Slot<CC, GG, kGate, IO, true>::warp_bytes(slots, xs, d_k);   \
-    return gate_kind == kGatePerKey ? Slot<CC, GG, kGatePerKey, IO>::warp_bytes(slots, xs, d_k)   \
-                                    : Slot<CC, GG, kGate, IO>::warp_bytes(slots, xs, d_k);
+    if (update_kind == kDelta)                                                                  \
+        return Slot<CC, GG, kGate, IO, true>::warp_bytes(slots, xs, tab, d_k);                  \
+    return gate_kind == kGatePerKey                                                             \
+               ? Slot<CC, GG, kGatePerKey, IO>::warp_bytes(slots, xs, tab, d_k)                 \
+               : Slot<CC, GG, kGate, IO>::warp_bytes(slots, xs, tab, d_k);
 #define LRS_SLOT(CC, GG)                                                                     \
     if (C == CC && group == GG) {                                                            \
         if (io == kStepIoBF16) {                                                             \

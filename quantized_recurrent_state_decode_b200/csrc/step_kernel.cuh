@@ -84,7 +84,8 @@ struct StepParams {
 //   [0, 128) mbarriers | v (d_v elements, one buffer: read before the tile's
 //   groups are, refilled with the next tile's first group) | slots of kBytes:
 //     codes | scales (d_v fp32) | q, k (GROUP elements each)
-// In both, SR and BDR add the x staging buffer at the end.
+// In both, the variants that stage x add the staging buffer after the slots
+// (and the widened inputs), and SR adds its row table after that.
 template <int C, int GROUP, int GATE, int IO = kIoF32, bool INS = false>
 struct Slot {
     static constexpr int DV = 32 * C;
@@ -95,10 +96,8 @@ struct Slot {
     static constexpr int kK = kQ + GROUP * ES;                    // INS only
     static constexpr int kBytes = INS ? kK + GROUP * ES : kQ;
     static_assert(kBytes % 16 == 0, "slot alignment");
-    // x staging (SR, BDR): 16 B per row pair and lane; then, for SR, the
-    // group's row table of the element hash (8 B per key row)
-    static constexpr int kTabOff = GROUP * 256;
-    static constexpr int kXsBytes = kTabOff + GROUP * 8;
+    static constexpr int kXsBytes = GROUP * 256;   // x staging: 16 B per row pair and lane
+    static constexpr int kTabBytes = GROUP * 8;    // SR: the group's row table of the hash
     // offsets inside a tile-input buffer (!INS)
     __host__ __device__ static int in_k(int d_k) { return d_k * ES; }
     __host__ __device__ static int in_g(int d_k) { return 2 * d_k * ES; }
@@ -116,9 +115,10 @@ struct Slot {
     // into a buffer after the slots: q, k (d_k each), v (d_v)
     static constexpr bool CVT = IO == kIoBF16 && !INS;
     __host__ __device__ static int cvt_bytes(int d_k) { return CVT ? (2 * d_k + DV) * 4 : 0; }
-    static int warp_bytes(int slots, bool xs, int d_k) {
-        return (header(d_k) + slots * kBytes + cvt_bytes(d_k) + (xs ? kXsBytes : 0) + 127) / 128 *
-               128;
+    // [header | slots | widened inputs (CVT) | x staging (xs) | row table (tab)]
+    static int warp_bytes(int slots, bool xs, bool tab, int d_k) {
+        return (header(d_k) + slots * kBytes + cvt_bytes(d_k) + (xs ? kXsBytes : 0) +
+                (tab ? kTabBytes : 0) + 127) / 128 * 128;
     }
 };
 
@@ -982,8 +982,9 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE, UPD) * 32, 1)
     const int in_k = S::in_k(p.d_k), in_g = S::in_g(p.d_k), in_v = S::in_v(p.d_k);
     float* cvt = reinterpret_cast<float*>(wsm + hdr + NS * S::kBytes);   // bf16 widened (CVT)
     float4* xs = reinterpret_cast<float4*>(wsm + hdr + NS * S::kBytes +
-                                           S::cvt_bytes(p.d_k));              // SR, BDR
-    uint2* rtab2 = reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(xs) + S::kTabOff);  // SR
+                                           S::cvt_bytes(p.d_k));              // staging variants
+    uint2* rtab2 = reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(xs) +
+                                            (stage_x(MODE, UPD) ? S::kXsBytes : 0));  // SR
     const uint4* rtab = reinterpret_cast<const uint4*>(rtab2);
     constexpr int IOR = S::CVT ? kIoF32 : IO;     // element type the pair code reads
     constexpr int ESR = IOR == kIoBF16 ? 2 : 4;

@@ -219,3 +219,59 @@ def _embed(fx, key, n, rows, fill):
     a = np.full(n, fill, np.float32)
     a[rows] = [float(c) for c in fx[key]]
     return a
+
+
+_U64 = np.uint64
+
+
+def _splitmix64(z):
+    z = z + _U64(0x9E3779B97F4A7C15)
+    z = (z ^ (z >> _U64(30))) * _U64(0xBF58476D1CE4E5B9)
+    z = (z ^ (z >> _U64(27))) * _U64(0x94D049BB133111EB)
+    return z ^ (z >> _U64(31))
+
+
+def _column_varying_carry_seed(B, H, d_v, step):
+    """The first seed for which some tile's hash key k2 = m(m(m(seed) ^ step)
+    ^ (b<<32 | h)) has a low half whose sum with the golden gamma's low half
+    carries for some value columns j < d_v and not for others (about one tile
+    in 2^32 / d_v)."""
+    bh = ((np.arange(B, dtype=np.uint64)[:, None] << _U64(32)) |
+          np.arange(H, dtype=np.uint64)[None, :]).reshape(-1)
+    wrap = (1 << 32) - 0x7F4A7C15
+    for s0 in range(0, 1 << 22, 4096):
+        seeds = np.arange(s0, s0 + 4096, dtype=np.uint64)
+        k1 = _splitmix64(_splitmix64(seeds) ^ _U64(step))
+        lo = _splitmix64(k1[:, None] ^ bh[None, :]) & _U64(0xFFFFFFFF)
+        kmin, kmax = lo & _U64(~(d_v - 1) & 0xFFFFFFFF), lo | _U64(d_v - 1)
+        hit = np.argwhere((kmin < wrap) & (kmax >= wrap))
+        if len(hit):
+            si, t = hit[0]
+            seed = int(seeds[si])
+            # the chain, recomputed by the oracle's SplitMix64
+            k = oracle.splitmix64(oracle.splitmix64(oracle.splitmix64(seed) ^ step) ^
+                                  int(bh[t]))
+            assert (k & 0xFFFFFFFF) == int(lo[si, t])
+            return seed, int(t)
+    raise AssertionError("no seed found")
+
+
+@pytest.mark.parametrize("d_v,prec", [(128, "int8"), (64, "int4")])
+def test_sr_tile_whose_hash_carry_varies_across_columns(d_v, prec):
+    # The kernel draws most tiles' numbers from a per-row table that assumes
+    # the same carry in every column; a tile where it differs takes the whole
+    # per-element hash. Find such a tile and compare the step with the oracle.
+    w = _small("gla", 64, 16, 128, d_v, 32, I.ROUND_SR, prec, steps=1)
+    step = 5
+    seed, tile = _column_varying_carry_seed(w.batch, w.heads, d_v, step)
+    pm = np.full(w.heads, 8 if prec == "int8" else 4, np.uint8)
+    pair = P.Pair(w, pm)
+    try:
+        pair.init(I.initial_state(w, device="cuda"))
+        x = I.step_inputs(w, 0, device="cuda")
+        o_gpu, o_ref = pair.step(x, step, seed)
+        P.check_out(o_gpu, o_ref, "carry tile %d" % tile)
+        pair.compare_state("carry tile %d" % tile)
+    finally:
+        pair.free()
+
