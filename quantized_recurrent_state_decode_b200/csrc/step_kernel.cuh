@@ -244,59 +244,31 @@ __device__ __forceinline__ void decode_word_biased(uint32_t w, float (&f)[32 / B
     }
 }
 
-// Rounded codes leave the rounding as floats 2^23 + B_n + code, whose bit
-// patterns are 0x4B000000 + B_n + code (B_n + code in [1, 2^23)), with the
-// stored byte (nibble) in the low bits. word_bias<BITS>(n) is 2^23 + B_n for
-// element n of a 32-bit word. Packing (encode_word) adds the patterns
-// shifted to their positions modulo 2^32; only the unshifted pattern (and,
-// for int4, the one shifted by 4) keeps any of 0x4B000000. B_n is the
-// offset-binary bias (128, 8) except at two positions whose extra amounts
-// cancel those leftovers: int8 elements 2 and 3 take 384 and 308 (adding
-// 1 and 180 to the top byte: 0x4B + 1 + 180 = 256), int4 elements 6 and 3
-// (nibbles 5 and 6) take 24 and 12 (adding 1 and 4 to nibble 6, against
-// 0x4B + 0xB0 from the two low patterns). Every B_n is even, so rounding
-// 2^23 + B_n + y to nearest-even breaks a tie of y the same way as rint.
+// Rounded codes leave the rounding as floats 2^23 + B + code, whose bit
+// patterns are 0x4B000000 + B + code with the stored byte (nibble) in their
+// low byte: B is the offset-binary bias (128 for int8, 8 for int4), so the
+// low byte is code + B in [1, 255] (int4: [1, 15], its high nibble 0). B is
+// even, so rounding 2^23 + B + y to nearest-even breaks a tie of y the same
+// way as rint. word_bias<BITS>(n) is 2^23 + B for element n of a word.
 template <int BITS>
-__host__ __device__ constexpr float word_bias(int n) {
-    if constexpr (BITS == 8) {
-        return kTwo23 + (n == 2 ? 384.0f : n == 3 ? 308.0f : 128.0f);
-    } else {
-        return kTwo23 + (n == 3 ? 12.0f : n == 6 ? 24.0f : 8.0f);
-    }
+__host__ __device__ constexpr float word_bias(int) {
+    return kTwo23 + (BITS == 8 ? 128.0f : 8.0f);
 }
 
 // Pack the stored bytes (nibbles) of 4 (8) rounded codes into one word with
-// integer multiply-adds on their bit patterns, modulo 2^32: a pattern
-// shifted left by 8 (4) bits or more keeps only its low bits, and the high
-// bits that remain cancel by the choice of word_bias (see above). The
-// multiply-adds run on the fused-multiply-add pipe beside the byte permutes
-// of the decode.
+// byte permutes on the integer pipe (the multiply-add pipe is the busier one
+// in the step): int8 takes the low byte of each pattern; int4 gathers the
+// low bytes of elements 0-3 and 4-7 and adds the second word shifted by 4
+// (byte n = element n | element n+4 << 4).
 template <int BITS>
 __device__ __forceinline__ uint32_t encode_word(const float (&t)[32 / BITS]) {
-    uint32_t r;
     if constexpr (BITS == 8) {
-        asm("{\n\t.reg .u32 a;\n\t"
-            "mad.lo.u32 a, %2, 256, %1;\n\t"
-            "mad.lo.u32 a, %3, 65536, a;\n\t"
-            "mad.lo.u32 %0, %4, 16777216, a;\n\t}"
-            : "=r"(r)
-            : "r"(__float_as_uint(t[0])), "r"(__float_as_uint(t[1])), "r"(__float_as_uint(t[2])),
-              "r"(__float_as_uint(t[3])));
+        return pack_low_bytes(t[0], t[1], t[2], t[3]);
     } else {
-        asm("{\n\t.reg .u32 a;\n\t"
-            "mad.lo.u32 a, %2, 16, %1;\n\t"
-            "mad.lo.u32 a, %3, 256, a;\n\t"
-            "mad.lo.u32 a, %4, 4096, a;\n\t"
-            "mad.lo.u32 a, %5, 65536, a;\n\t"
-            "mad.lo.u32 a, %6, 1048576, a;\n\t"
-            "mad.lo.u32 a, %7, 16777216, a;\n\t"
-            "mad.lo.u32 %0, %8, 268435456, a;\n\t}"
-            : "=r"(r)
-            : "r"(__float_as_uint(t[0])), "r"(__float_as_uint(t[4])), "r"(__float_as_uint(t[1])),
-              "r"(__float_as_uint(t[5])), "r"(__float_as_uint(t[2])), "r"(__float_as_uint(t[6])),
-              "r"(__float_as_uint(t[3])), "r"(__float_as_uint(t[7])));
+        const uint32_t lo = pack_low_bytes(t[0], t[1], t[2], t[3]);
+        const uint32_t hi = pack_low_bytes(t[4], t[5], t[6], t[7]);
+        return lo + (hi << 4);
     }
-    return r;
 }
 
 template <int BITS> struct Q;

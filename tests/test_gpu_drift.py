@@ -34,3 +34,10 @@ def test_drift_series_small_batch():
     assert res["rtn"][1] == res["bdr"][1]
     # int4 requantization leaves a visible error once the state has been rounded
     assert res["rtn"][1] > 0.0 and res["sr"][1] > 0.0
+    # S0 = 0: with the bypass the quantized part stays zero until the first
+    # merge (after step `rank`, whose output is read before the merge), so up
+    # to t = rank = 4 the output differs from the fp32 state's only by the
+    # order of fp32 roundings
+    for n in ("lrb4_rtn", "lrb4_bdr"):
+        assert max(res[n][:3]) <= 1e-6, (n, res[n])
+        assert res[n][3] > 1e-3, (n, res[n])        # merged and rounded from t = 8 on

@@ -1,13 +1,16 @@
 """The allocation-free host-buffer step (lrs_decode_step_host_noalloc).
 
-Callers that cannot allocate device memory when they step -- code running
-during CUDA graph capture, or processes whose device memory belongs to a fixed
-pool -- use this entry point; its scratch is a static array in the library.
-This test runs it through the C ABI next to the allocating entry point
+Callers that must not allocate device memory when they step -- a process
+whose device memory belongs to another allocator or to a fixed pool sized at
+start-up, or a latency-critical path that cannot pay for a cudaMalloc --
+use this entry point; its scratch is a static array in the library. This test
+runs it through the C ABI next to the allocating entry point
 (lrs_decode_step_host) on two states with the same start, for two calls in a
 row, and requires identical outputs and states (the same bit-exact bar as the
-other parity tests). It sits in a file pytest collects last and works both
-alone in a fresh process and after the other tests.
+other parity tests): round to nearest, stochastic rounding and BDR, per-head
+and per-(head, scale group) widths, the gated and the delta-rule update. It
+sits in a file pytest collects last and works both alone in a fresh process
+and after the other tests.
 """
 import numpy as np
 import pytest
@@ -26,16 +29,24 @@ def _snapshot(st):
     return raw, sc
 
 
-@pytest.mark.parametrize("family,mode,pm", [
-    ("gla", I.ROUND_RTN, [8, 8, 4, 4]),
-    ("gdn", I.ROUND_SR, [8, 4, 8, 4]),
+# per-(head, scale group) widths of the 4 heads x 4 groups states
+PG = [[8, 4, 4, 8], [4, 4, 8, 8], [8, 8, 8, 4], [4, 8, 4, 4]]
+
+
+@pytest.mark.parametrize("family,mode,pm,d_k", [
+    ("gla", I.ROUND_RTN, [8, 8, 4, 4], 128),
+    ("gdn", I.ROUND_SR, [8, 4, 8, 4], 128),
+    ("gla", I.ROUND_BDR, [4, 8, 8, 4], 128),
+    ("gdn", I.ROUND_BDR, [8, 4, 4, 8], 64),
+    ("gla", I.ROUND_SR, PG, 128),
+    ("gdn", I.ROUND_BDR, PG, 128),
 ])
-def test_noalloc_step_matches_allocating_step(family, mode, pm):
-    w = I.Workload("noalloc_" + family, family, 9, 4, 128, 128, 32, 2, mode, "mixed",
+def test_noalloc_step_matches_allocating_step(family, mode, pm, d_k):
+    w = I.Workload("noalloc_" + family, family, 9, 4, d_k, 128, 32, 2, mode, "mixed",
                    s0_std=0.02, gate_mu=4.0 if family == "gdn" else -4.0, seed_id=95)
     pm = np.array(pm, np.uint8)
     shp = lrs.shape(w.batch, w.heads, w.d_k, w.d_v, w.group, w.update_kind, w.gate_kind)
-    a = lrs.lrs_state_alloc(shp, pm)
+    a = lrs.lrs_state_alloc(shp, pm)          # [H] or [H][G] widths
     b = lrs.lrs_state_alloc(shp, pm)
     try:
         S0 = I.initial_state(w, device="cuda")
