@@ -670,6 +670,10 @@ def run_configs(dev, stream, n=64):
                                           "hbm_frac": fb / (ms_f / 1e3) / 1e9 / peak,
                                           "layers_rotated": Lf},
                     "speedup_vs_fp32_state": ms_f / ms})
+                # the NEXT rows on the same states and inputs, in the same mode
+                rows[-1]["lrb"] = run_lrb_extra(w, w, states, xs, out, seed, stream, L, NI, m,
+                                                dev, pm)
+                rows[-1]["chunk"] = run_chunk_extra(w, w, states, seed, stream, L, m, dev, pm)
         for st in states:
             lrs.lrs_state_free(st)
         del Ss, xs, out

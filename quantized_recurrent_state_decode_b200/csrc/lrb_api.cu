@@ -17,16 +17,6 @@ namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// LRS_LRB_KERNEL=tile selects the one-CTA-per-tile kernel for every rank (for
-// comparisons); by default ranks up to 4 use the streaming kernel.
-bool lrs_stream_enabled() {
-    static const bool on = [] {
-        const char* e = getenv("LRS_LRB_KERNEL");
-        return !(e && std::string(e) == "tile");
-    }();
-    return on;
-}
-
 lrs::ChunkKernel find_lrb(int d_k, int d_v, int group, int update_kind, int gate_kind, int mode) {
     switch (mode) {
         case LRS_ROUND_RTN: return lrs::find_lrb_kernel_rtn(d_k, d_v, group, update_kind, gate_kind);
@@ -71,12 +61,13 @@ const void* find_lrb_stream(int C, int group, int update_kind, int gate_kind, in
     }
 }
 
-int lrb_stream_warp_smem(int C, int group, int gate_kind, int slots, int d_k, bool staged) {
-#define LRS_LRB_SLOT(CC, GG)                                                                  \
-    if (C == CC && group == GG)                                                               \
-        return gate_kind == lrs::kGatePerKey                                                  \
-                   ? lrs::LrbSlot<CC, GG, lrs::kGatePerKey>::warp_bytes(slots, d_k, staged)    \
-                   : lrs::LrbSlot<CC, GG, lrs::kGate>::warp_bytes(slots, d_k, staged);
+int lrb_stream_warp_smem(int C, int group, int gate_kind, int slots, int d_k, bool staged,
+                         bool tab) {
+#define LRS_LRB_SLOT(CC, GG)                                                                       \
+    if (C == CC && group == GG)                                                                    \
+        return gate_kind == lrs::kGatePerKey                                                       \
+                   ? lrs::LrbSlot<CC, GG, lrs::kGatePerKey>::warp_bytes(slots, d_k, staged, tab)    \
+                   : lrs::LrbSlot<CC, GG, lrs::kGate>::warp_bytes(slots, d_k, staged, tab);
     LRS_LRB_SLOT(4, 16)
     LRS_LRB_SLOT(4, 32)
     LRS_LRB_SLOT(2, 16)
@@ -104,7 +95,8 @@ lrs_status launch_lrb_stream(const lrs_state* st, void* state_codes, float* scal
     int slots = sh.update_kind == LRS_UPDATE_DELTA ? G : std::min(2, G);
     slots = std::max(1, std::min(slots, lrs::kMaxSlots));
     const int warp_smem =
-        lrb_stream_warp_smem(C, sh.group, sh.gate_kind, slots, sh.d_k, lrs::lrb_staged(mode, merge));
+        lrb_stream_warp_smem(C, sh.group, sh.gate_kind, slots, sh.d_k, lrs::lrb_staged(mode, merge),
+                             mode == LRS_ROUND_SR);
     constexpr int kSmemLimit = 227 * 1024;
     const int warps = std::min(lrs::lrb_max_warps(mode, merge, sh.group), kSmemLimit / warp_smem);
     if (warps < 1) return LRS_ERR_UNSUPPORTED;
@@ -198,7 +190,7 @@ lrs_status lrs_lrb_step(const lrs_state* st, void* state_codes, float* scales,
         return lrs::api_fail(LRS_ERR_INVALID_ARG, "beta is NULL");
     const int64_t ntiles0 = static_cast<int64_t>(sh.batch) * sh.heads;
     if (ntiles0 == 0) return lrs::api_ok();
-    if (rank <= lrs::kLrbStreamMaxRank && lrs_stream_enabled()) {
+    if (rank <= lrs::kLrbStreamMaxRank) {
         unsigned* err = nullptr;
         int sms = 0;
         s = lrs::device_error_word(&err, &sms);

@@ -34,7 +34,8 @@ struct LrbStreamParams {
     int32_t rank, m;      // rank, components filled before the step (step mod rank)
 };
 
-// Per-warp shared memory: barriers | two tile-input buffers | slots | x staging.
+// Per-warp shared memory: barriers | two tile-input buffers | slots | x
+// staging | SR row table.
 // Tile-input buffer: q, k, [gate] (d_k fp32 each) | v (d_v) | U (4 rows of
 // d_k) | V (4 rows of d_v).
 template <int C, int GROUP, int GATE>
@@ -44,6 +45,7 @@ struct LrbSlot {
     static constexpr int kScales = kCodes;
     static constexpr int kBytes = kScales + DV * 4;
     static constexpr int kXsBytes = GROUP * 256;
+    static constexpr int kTabBytes = GROUP * 8;    // SR: the group's row table of the hash
     __host__ __device__ static int in_k(int d_k) { return d_k * 4; }
     __host__ __device__ static int in_g(int d_k) { return 2 * d_k * 4; }
     __host__ __device__ static int in_v(int d_k) {
@@ -55,8 +57,9 @@ struct LrbSlot {
         return (in_vb(d_k) + kLrbStreamMaxRank * DV * 4 + 15) / 16 * 16;
     }
     __host__ __device__ static int header(int d_k) { return 128 + 2 * tile_in_bytes(d_k); }
-    static int warp_bytes(int slots, int d_k, bool staged) {
-        return (header(d_k) + slots * kBytes + (staged ? kXsBytes : 0) + 127) / 128 * 128;
+    static int warp_bytes(int slots, int d_k, bool staged, bool tab) {
+        return (header(d_k) + slots * kBytes + (staged ? kXsBytes : 0) + (tab ? kTabBytes : 0) +
+                127) / 128 * 128;
     }
 };
 
@@ -114,7 +117,8 @@ __device__ __forceinline__ void pair_step_lrb(const uint8_t* __restrict__ cs, in
                                               uint32_t j0, int lane, float4* __restrict__ xs,
                                               bool merge, int R, const float* __restrict__ Ut,
                                               int dk, const float (&vc0)[kLrbStreamMaxRank],
-                                              const float (&vc1)[kLrbStreamMaxRank]) {
+                                              const float (&vc1)[kLrbStreamMaxRank],
+                                              const uint4* __restrict__ rtab, bool rowtab) {
     using G = PairGeo<GROUP, BITS>;
     constexpr float BIAS = Q<BITS>::kBias;
     constexpr int RPUH = G::RPU / 2;
@@ -187,6 +191,20 @@ __device__ __forceinline__ void pair_step_lrb(const uint8_t* __restrict__ cs, in
     float2 snew, inv;
     new_scales<BITS>(a0, b0, snew, inv);
     st_cs_f2(gscale, snew);
+    if constexpr (MODE == kSR) {
+        // SR stages x: the decode step's rounding pass, with the row table of
+        // the hash when the tile's carry allows it
+        static_assert(STAGE, "SR stages x");
+        if (rowtab)
+            round_pass<GROUP, GATE, kSR, BITS, kIoF32, true, true>(
+                cs, ubase, sc, nullptr, gs, gscalar, f2(0.0f), inv, snew, gcodes, hkey, row0, j0,
+                lane, xs, rtab);
+        else
+            round_pass<GROUP, GATE, kSR, BITS, kIoF32, true, false>(
+                cs, ubase, sc, nullptr, gs, gscalar, f2(0.0f), inv, snew, gcodes, hkey, row0, j0,
+                lane, xs, rtab);
+        return;
+    }
     const float2 inv0 = f2(inv.x), inv1 = f2(inv.y);
     const float2 sn0 = f2(snew.x), sn1 = f2(snew.y);
 
@@ -426,6 +444,9 @@ __global__ void __launch_bounds__(lrb_max_warps(MODE, MERGE, GROUP) * 32, 1)
     const int hdr = S::header(dk), tib = S::tile_in_bytes(dk);
     const int in_k = S::in_k(dk), in_g = S::in_g(dk), in_v = S::in_v(dk), in_u = S::in_u(dk);
     float4* xs = reinterpret_cast<float4*>(wsm + hdr + NS * S::kBytes);
+    uint2* rtab2 = reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(xs) +
+                                            (lrb_staged(MODE, MERGE) ? S::kXsBytes : 0));  // SR
+    const uint4* rtab = reinterpret_cast<const uint4*>(rtab2);
     const int ntw = gw < p.ntiles ? (p.ntiles - gw + W - 1) / W : 0;
     const int64_t K = static_cast<int64_t>(ntw) * G;
     const int R = lp.rank, m = lp.m;
@@ -476,6 +497,8 @@ __global__ void __launch_bounds__(lrb_max_warps(MODE, MERGE, GROUP) * 32, 1)
                                                           static_cast<uint32_t>(ti.b),
                                                           static_cast<uint32_t>(ti.h))
                                           : 0ull;
+        uint32_t hcarry = 0;
+        const bool rowtab = MODE == kSR && sr_tile_carry(hkey, DV, &hcarry);
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[ic.slot], ic.par, p.timeout_ns));
         if (!ok) break;
         if (!ti.ok) {
@@ -624,6 +647,18 @@ __global__ void __launch_bounds__(lrb_max_warps(MODE, MERGE, GROUP) * 32, 1)
             uint8_t* gcodes = gcodes_tile + ti.goff(g, GROUP * DV / 2);
             const bool int8g = ti.bits(g) == 8;
             const float* Ug = Ut + g * GROUP;
+            if constexpr (MODE == kSR) {
+                // the group's row table of the hash (the previous group's
+                // readers finished at the warp barrier ending it)
+                if (rowtab) {
+                    for (int r = lane; r < GROUP; r += 32) {
+                        const SrRow rr = sr_row(static_cast<uint32_t>(hkey >> 32),
+                                                static_cast<uint32_t>(g * GROUP + r), hcarry);
+                        rtab2[r] = make_uint2(rr.sh, rr.p);
+                    }
+                    __syncwarp();
+                }
+            }
             float2 op = o[0], oq = o[P - 1];
 #pragma unroll 1
             for (int pc = 0; pc < P; ++pc) {
@@ -651,12 +686,12 @@ __global__ void __launch_bounds__(lrb_max_warps(MODE, MERGE, GROUP) * 32, 1)
                     pair_step_lrb<GROUP, GATE, MODE, 8, lrb_staged(MODE, MERGE)>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs, gs,
                                                         gscalar, op, gcodes, gscale + 2 * pc, hkey,
                                                         g * GROUP, j0, lane, xs, merge, R, Ug, dk,
-                                                        vc0, vc1);
+                                                        vc0, vc1, rtab, rowtab);
                 else
                     pair_step_lrb<GROUP, GATE, MODE, 4, lrb_staged(MODE, MERGE)>(sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs, gs,
                                                         gscalar, op, gcodes, gscale + 2 * pc, hkey,
                                                         g * GROUP, j0, lane, xs, merge, R, Ug, dk,
-                                                        vc0, vc1);
+                                                        vc0, vc1, rtab, rowtab);
                 if constexpr (P == 2) {
                     const float2 to = op;
                     op = oq; oq = to;
