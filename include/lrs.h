@@ -60,8 +60,11 @@ typedef enum {
     LRS_ERR_DEVICE_TIMEOUT = 6, /* a kernel gave up waiting for its copies */
     LRS_ERR_DEVICE_LAYOUT = 7,  /* the precision map passed to a step does not
                                    fit the state's tile layout */
-    LRS_ERR_DEVICE_RANGE = 8    /* lrs_state_import_codes met a code outside
+    LRS_ERR_DEVICE_RANGE = 8,   /* lrs_state_import_codes met a code outside
                                    [-qmax, qmax] */
+    LRS_ERR_DEVICE_BOUNDS = 9   /* bounds-checked debug build only: a step
+                                   kernel index fell outside its buffer (the
+                                   access was skipped) */
 } lrs_status;
 
 typedef enum { LRS_ROUND_RTN = 0, LRS_ROUND_SR = 1, LRS_ROUND_BDR = 2 } lrs_round_mode;

@@ -151,6 +151,8 @@ lrs_status launch_lrb_stream(const lrs_state* st, void* state_codes, float* scal
     p.warp_smem = warp_smem;
     p.slots = slots;
     p.inject = lrs::take_injected_timeout(&p.timeout_ns) ? 1 : 0;
+    p.code_bytes = st->code_bytes;
+    p.scale_count = st->scale_count;
     lp.U = U;
     lp.V = V;
     lp.rank = rank;

@@ -306,6 +306,7 @@ const char* lrs_status_string(lrs_status s) {
         case LRS_ERR_DEVICE_TIMEOUT: return "LRS_ERR_DEVICE_TIMEOUT";
         case LRS_ERR_DEVICE_LAYOUT: return "LRS_ERR_DEVICE_LAYOUT";
         case LRS_ERR_DEVICE_RANGE: return "LRS_ERR_DEVICE_RANGE";
+        case LRS_ERR_DEVICE_BOUNDS: return "LRS_ERR_DEVICE_BOUNDS";
     }
     return "LRS_ERR_UNKNOWN";
 }
@@ -490,6 +491,8 @@ static lrs_status decode_step_io(const lrs_state* st, void* state_codes, float* 
     p.warp_smem = ls.warp_smem;
     p.slots = ls.slots;
     p.inject = 0;
+    p.code_bytes = st->code_bytes;
+    p.scale_count = st->scale_count;
     {
         std::lock_guard<std::mutex> lk(g_inject_mu);
         if (g_inject) {
@@ -747,6 +750,9 @@ lrs_status lrs_sync(void* stream) {
         return fail(LRS_ERR_DEVICE_TIMEOUT, "a step kernel timed out waiting for its copies");
     if (flags & lrs::kErrLayout)
         return fail(LRS_ERR_DEVICE_LAYOUT, "prec_map does not fit the state's tile layout");
+    if (flags & lrs::kErrBounds)
+        return fail(LRS_ERR_DEVICE_BOUNDS, "a step kernel index fell outside its buffer "
+                    "(bounds-checked build)");
     return fail(LRS_ERR_DEVICE_RANGE, "an imported code was outside [-qmax, qmax]");
 }
 

@@ -150,6 +150,8 @@ extern "C" lrs_status lrs_decode_step_host_noalloc(const lrs_state* st, const fl
     p.slots = ls.slots;
     p.warp_smem = ls.warp_smem;
     p.inject = 0;
+    p.code_bytes = st->code_bytes;
+    p.scale_count = st->scale_count;
     void* args[] = {&p};
     if ((e = cudaLaunchKernel(ls.fn, dim3(grid), dim3(ls.warps * 32), args, ls.smem, cs)) !=
         cudaSuccess) {

@@ -68,6 +68,8 @@ struct StepParams {
     int32_t slots;       // ring slots per warp, 1..min(G, 16); the delta rule needs G
     int32_t warp_smem;   // bytes of shared memory per warp
     int32_t inject;      // error-path tests: 0, or n + 1 to issue copies for n items per warp
+    int64_t code_bytes;  // bytes of the code buffer and floats of the scale buffer
+    int64_t scale_count; // (read by the bounds-checked build only)
 };
 
 // Shared-memory layout of one warp (ES = bytes of a q, k, v element).
@@ -897,6 +899,22 @@ __device__ __forceinline__ void issue_item(const StepParams& p, uint8_t* wsm, in
     } else if (g == 0) {
         total += S::tile_in_payload(dk);
     }
+    if constexpr (kBoundsCheck) {
+        // the slot and the tile-input buffer inside the warp's shared memory;
+        // the group's codes and scales and the tile's rows inside their buffers
+        const int64_t coff = tc.code_off + tc.goff(g, GROUP * DV / 2);
+        const bool ok =
+            in_bounds(sm + S::kBytes <= wsm + p.warp_smem && (INS || slot < p.slots) &&
+                          (INS || tin + S::tile_in_payload(dk) <= wsm + S::header(dk)) &&
+                          coff >= 0 && coff + cbytes <= p.code_bytes &&
+                          (static_cast<int64_t>(tile) * p.G + g + 1) * DV <= p.scale_count &&
+                          tile < p.ntiles,
+                      p.err);
+        if (!ok) {
+            mbar_arrive(bar);
+            return;
+        }
+    }
     mbar_arrive_expect_tx(bar, total);
     bulk_g2s(sm, p.codes + tc.code_off + tc.goff(g, GROUP * DV / 2), cbytes, bar, pol_state);
     bulk_g2s(sm + S::kScales, p.scales + (static_cast<int64_t>(tile) * p.G + g) * DV, DV * 4, bar,
@@ -1057,9 +1075,18 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE, UPD) * 32, 1)
             }
         }
 
-        if (!ti.ok) {
-            // no copies were made for this tile: record the mismatch and skip it
-            if (lane == 0) atomicOr(p.err, kErrLayout);
+        bool inside = true;      // the tile's codes and scales inside their buffers
+        if constexpr (kBoundsCheck) {
+            const int64_t tbytes = ti.goff(G, GROUP * DV / 2);
+            inside = !ti.ok || in_bounds(ti.code_off >= 0 && ti.code_off + tbytes <= p.code_bytes &&
+                                             (static_cast<int64_t>(tile) + 1) * G * DV <=
+                                                 p.scale_count,
+                                         p.err);
+        }
+        if (!ti.ok || !inside) {
+            // a layout mismatch (no copies were made) or, in the bounds-checked
+            // build, a tile outside its buffers: record it and skip the tile
+            if (lane == 0 && !ti.ok) atomicOr(p.err, kErrLayout);
             for (int g = 0; g < G; ++g) {
                 if (g > 0) {
                     ok = __all_sync(0xffffffffu,
@@ -1158,6 +1185,22 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE, UPD) * 32, 1)
             for (int pc = 0; pc < P; ++pc) {
                 const float2 sc = *reinterpret_cast<const float2*>(ss + 2 * pc);
                 const uint32_t j0 = static_cast<uint32_t>(lane * C + 2 * pc);
+                if constexpr (kBoundsCheck) {
+                    // this pair's units of the slot and of the state, and its scales
+                    const int units = int8g ? PairGeo<GROUP, 8>::UNITS : PairGeo<GROUP, 4>::UNITS;
+                    const int64_t end = (static_cast<int64_t>(pc) + 1) * units * 512;
+                    if (!in_bounds(end <= S::kCodes &&
+                                       (gcodes - p.codes) + end <= p.code_bytes &&
+                                       (gscale - p.scales) + 2 * pc + 2 <= p.scale_count &&
+                                       j0 + 2 <= static_cast<uint32_t>(DV),
+                                   p.err)) {
+                        if constexpr (P == 2) {
+                            const float2 tw = wp, to = op;
+                            wp = wq; op = oq; wq = tw; oq = to;
+                        }
+                        continue;
+                    }
+                }
                 if constexpr (MODE != kRTN) {
                     constexpr bool ST = stage_x(MODE, UPD);
                     if (int8g)
@@ -1195,6 +1238,7 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE, UPD) * 32, 1)
         }
         if (!ok) break;
         const int64_t oi = static_cast<int64_t>(tile) * DV + lane * C;
+        if (!in_bounds(oi + C <= static_cast<int64_t>(p.ntiles) * DV, p.err)) continue;
         if constexpr (IO == kIoF32) {
             float* op = static_cast<float*>(p.out) + oi;
             if constexpr (P == 2) {

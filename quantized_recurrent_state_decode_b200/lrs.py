@@ -20,6 +20,7 @@ LRS_ERR_CUDA = 5
 LRS_ERR_DEVICE_TIMEOUT = 6
 LRS_ERR_DEVICE_LAYOUT = 7
 LRS_ERR_DEVICE_RANGE = 8
+LRS_ERR_DEVICE_BOUNDS = 9
 
 LRS_ROUND_RTN, LRS_ROUND_SR, LRS_ROUND_BDR = 0, 1, 2
 LRS_UPDATE_GATED, LRS_UPDATE_DELTA = 0, 1
@@ -81,6 +82,15 @@ _SIGS = {
     "lrs_debug_inject_timeout": [ctypes.c_int32, ctypes.c_int32],
     "lrs_debug_inject_timeout_after": [ctypes.c_int32, ctypes.c_int32],
 }
+
+
+def use_library(path):
+    """Load another build of the library (e.g. the bounds-checked
+    liblrs_checked.so) instead of liblrs.so; only before the first call."""
+    global LIB_PATH
+    if _lib is not None:
+        raise RuntimeError("the library is already loaded from %s" % LIB_PATH)
+    LIB_PATH = path
 
 
 def lib():
