@@ -250,8 +250,11 @@ lrs_status step_launch_shape(const lrs_shape& sh, int mode, int io, int device, 
     if (!fn) return fail(LRS_ERR_UNSUPPORTED, "no compiled kernel for this shape and mode");
     // ring slots per warp: the delta rule keeps a whole tile resident; the
     // gated forms stream a few groups ahead (at most G, so that the single v
-    // buffer is never overwritten before it is read)
-    int slots = sh.update_kind == LRS_UPDATE_DELTA ? G : std::min(kDefaultSlots, G);
+    // buffer is never overwritten before it is read); gated SR streams one
+    // group ahead through a single slot released early (sr_early_release)
+    int slots = sh.update_kind == LRS_UPDATE_DELTA
+                    ? G
+                    : std::min(sr_early_release(mode, sh.update_kind) ? 1 : kDefaultSlots, G);
     slots = std::max(1, std::min(slots, kMaxSlots));
     const int warp_smem = step_warp_smem(C, sh.group, sh.update_kind, sh.gate_kind, slots, mode,
                                          io, sh.d_k);

@@ -39,11 +39,19 @@ constexpr int kMaxSlots = 16;
 __host__ __device__ constexpr bool stage_x(int mode, int upd) {
     return mode == kSR || (mode == kBDR && upd == kDelta);
 }
+// SR of the gated forms runs a ring of one slot per warp, released early: its
+// rounding loop reads only the staged values, so the slot is free for the
+// next group's copy once the last column pair's first loop has read it. The
+// one-slot ring leaves shared memory for 12 warps beside the staging buffer.
+__host__ __device__ constexpr bool sr_early_release(int mode, int upd) {
+    return mode == kSR && upd == kGated;
+}
 // Launch bound of a step variant in warps: 12 (at most 168 registers a thread)
 // where the live state fits, 8 (255 registers) for the wider groups and for
-// the staging variants, whose buffer leaves shared memory for 8 warps.
+// the other staging variants, whose buffer leaves shared memory for 8 warps
+// beside a ring of several slots.
 __host__ __device__ constexpr int step_max_warps(int group, int mode, int upd) {
-    return (stage_x(mode, upd) || group > 32) ? 8 : 12;
+    return ((stage_x(mode, upd) && !sr_early_release(mode, upd)) || group > 32) ? 8 : 12;
 }
 constexpr float kTiny = 0x1p-100f;               // absmax below this: stored as zero
 
@@ -807,15 +815,16 @@ __device__ __forceinline__ void round_pass(const uint8_t* __restrict__ cs, int u
     }
 }
 
+// The first loop of pair_step_xs: x, the output, the absmax (and the staged
+// x); then the new scales, stored, and their inverses.
 template <int GROUP, int GATE, int MODE, int BITS, int IO, bool STAGE>
-__device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int ubase, float2 sc,
-                                             const uint8_t* __restrict__ qs,
-                                             const uint8_t* __restrict__ ks,
-                                             const float* __restrict__ gs, float gscalar,
-                                             float2 w, float2& o, uint8_t* __restrict__ gcodes,
-                                             float* __restrict__ gscale, uint64_t hkey, int row0,
-                                             uint32_t j0, int lane, float4* __restrict__ xs,
-                                             const uint4* __restrict__ rtab, bool rowtab) {
+__device__ __forceinline__ void pair_pass1_xs(const uint8_t* __restrict__ cs, int ubase, float2 sc,
+                                              const uint8_t* __restrict__ qs,
+                                              const uint8_t* __restrict__ ks,
+                                              const float* __restrict__ gs, float gscalar,
+                                              float2 w, float2& o, float* __restrict__ gscale,
+                                              int lane, float4* __restrict__ xs, float2& snew,
+                                              float2& inv) {
     using G = PairGeo<GROUP, BITS>;
     constexpr float BIAS = Q<BITS>::kBias;
     constexpr int RPUH = G::RPU / 2;              // row pairs per unit
@@ -858,9 +867,20 @@ __device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int
         }
     }
 
-    float2 snew, inv;
     new_scales<BITS>(a0, b0, snew, inv);
     st_cs_f2(gscale, snew);
+}
+
+// The rounding loop of pair_step_xs, from the first loop's snew and inv.
+template <int GROUP, int GATE, int MODE, int BITS, int IO, bool STAGE>
+__device__ __forceinline__ void pair_round_xs(const uint8_t* __restrict__ cs, int ubase, float2 sc,
+                                              const uint8_t* __restrict__ ks,
+                                              const float* __restrict__ gs, float gscalar,
+                                              float2 w, float2 snew, float2 inv,
+                                              uint8_t* __restrict__ gcodes, uint64_t hkey,
+                                              int row0, uint32_t j0, int lane,
+                                              const float4* __restrict__ xs,
+                                              const uint4* __restrict__ rtab, bool rowtab) {
     if (MODE == kSR && rowtab)
         round_pass<GROUP, GATE, MODE, BITS, IO, STAGE, true>(cs, ubase, sc, ks, gs, gscalar, w,
                                                             inv, snew, gcodes, hkey, row0, j0,
@@ -869,6 +889,23 @@ __device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int
         round_pass<GROUP, GATE, MODE, BITS, IO, STAGE, false>(cs, ubase, sc, ks, gs, gscalar, w,
                                                              inv, snew, gcodes, hkey, row0, j0,
                                                              lane, xs, rtab);
+}
+
+template <int GROUP, int GATE, int MODE, int BITS, int IO, bool STAGE>
+__device__ __forceinline__ void pair_step_xs(const uint8_t* __restrict__ cs, int ubase, float2 sc,
+                                             const uint8_t* __restrict__ qs,
+                                             const uint8_t* __restrict__ ks,
+                                             const float* __restrict__ gs, float gscalar,
+                                             float2 w, float2& o, uint8_t* __restrict__ gcodes,
+                                             float* __restrict__ gscale, uint64_t hkey, int row0,
+                                             uint32_t j0, int lane, float4* __restrict__ xs,
+                                             const uint4* __restrict__ rtab, bool rowtab) {
+    float2 snew, inv;
+    pair_pass1_xs<GROUP, GATE, MODE, BITS, IO, STAGE>(cs, ubase, sc, qs, ks, gs, gscalar, w, o,
+                                                      gscale, lane, xs, snew, inv);
+    pair_round_xs<GROUP, GATE, MODE, BITS, IO, STAGE>(cs, ubase, sc, ks, gs, gscalar, w, snew, inv,
+                                                      gcodes, hkey, row0, j0, lane, xs, rtab,
+                                                      rowtab);
 }
 
 // Fill `slot` with group g of the cursor's tile (lane 0 only); with the
@@ -1016,6 +1053,14 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE, UPD) * 32, 1)
         }
     };
     for (int s = 0; s < NS; ++s) issue_next();
+    // the consumer is done with its slot: hand it to the next item's copy
+    auto release_slot = [&]() {
+        ++kc;
+        ic.advance(NS);
+        __syncwarp();
+        if (lane == 0) fence_proxy_async_smem();
+        issue_next();
+    };
 
     float nscal = 0.0f, nbeta = 0.0f;
     if (ntw > 0) {
@@ -1181,6 +1226,8 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE, UPD) * 32, 1)
             // The column pairs run one after the other through one copy of the
             // (large) pair code; the pairs' w and o rotate through (wp, op).
             float2 wp = w[0], op = o[0], wq = w[P - 1], oq = o[P - 1];
+            constexpr bool EARLY = sr_early_release(MODE, UPD);
+            bool released = false;   // the slot, after the last pair's first loop (EARLY)
 #pragma unroll 1
             for (int pc = 0; pc < P; ++pc) {
                 const float2 sc = *reinterpret_cast<const float2*>(ss + 2 * pc);
@@ -1201,7 +1248,31 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE, UPD) * 32, 1)
                         continue;
                     }
                 }
-                if constexpr (MODE != kRTN) {
+                if constexpr (EARLY) {
+                    // first loop; the slot's last reader done, the next copy
+                    // is issued; then the rounding loop on the staged values
+                    float2 snew, inv;
+                    if (int8g)
+                        pair_pass1_xs<GROUP, GATE, MODE, 8, IOR, true>(
+                            sm, pc * PairGeo<GROUP, 8>::UNITS, sc, qs, ks, gs, gscalar, wp, op,
+                            gscale + 2 * pc, lane, xs, snew, inv);
+                    else
+                        pair_pass1_xs<GROUP, GATE, MODE, 4, IOR, true>(
+                            sm, pc * PairGeo<GROUP, 4>::UNITS, sc, qs, ks, gs, gscalar, wp, op,
+                            gscale + 2 * pc, lane, xs, snew, inv);
+                    if (pc == P - 1) {
+                        release_slot();
+                        released = true;
+                    }
+                    if (int8g)
+                        pair_round_xs<GROUP, GATE, MODE, 8, IOR, true>(
+                            sm, pc * PairGeo<GROUP, 8>::UNITS, sc, ks, gs, gscalar, wp, snew, inv,
+                            gcodes, hkey, g * GROUP, j0, lane, xs, rtab, rowtab);
+                    else
+                        pair_round_xs<GROUP, GATE, MODE, 4, IOR, true>(
+                            sm, pc * PairGeo<GROUP, 4>::UNITS, sc, ks, gs, gscalar, wp, snew, inv,
+                            gcodes, hkey, g * GROUP, j0, lane, xs, rtab, rowtab);
+                } else if constexpr (MODE != kRTN) {
                     constexpr bool ST = stage_x(MODE, UPD);
                     if (int8g)
                         pair_step_xs<GROUP, GATE, MODE, 8, IOR, ST>(sm, pc * PairGeo<GROUP, 8>::UNITS, sc,
@@ -1230,11 +1301,7 @@ __global__ void __launch_bounds__(step_max_warps(GROUP, MODE, UPD) * 32, 1)
             }
             o[0] = op;
             o[P - 1] = P == 2 ? oq : op;
-            ++kc;
-            ic.advance(NS);
-            __syncwarp();
-            if (lane == 0) fence_proxy_async_smem();
-            issue_next();
+            if (!released) release_slot();
         }
         if (!ok) break;
         const int64_t oi = static_cast<int64_t>(tile) * DV + lane * C;
