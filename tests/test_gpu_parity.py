@@ -66,6 +66,14 @@ def test_ragged_tile_counts(B, H):
     P.run_parity(w, w.steps, check_every=1)
 
 
+@pytest.mark.parametrize("B,H", [(1, 1), (1, 7), (37, 3), (149, 8)])
+def test_ragged_tile_counts_gated_sr(B, H):
+    # the gated SR launch (a one-slot ring handed to the next copy after the
+    # last pair's first loop) on tile counts below and between warp multiples
+    w = _small("gla", B, H, 128, 128, 32, I.ROUND_SR, "mixed", steps=3)
+    P.run_parity(w, w.steps, check_every=1)
+
+
 def test_zero_batch_is_a_no_op():
     w = _small("gla", 0, 4, 64, 64, 32, I.ROUND_RTN, "int8", steps=1)
     st = lrs.lrs_state_alloc(P.make_shape(w), np.full(4, 8, np.uint8))
